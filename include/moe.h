@@ -1,0 +1,332 @@
+/*
+ * libmoe -- one mixture-of-experts feed-forward layer, forward and backward,
+ * on one NVIDIA B200 (sm_100a).  Plain C ABI: pointers, sizes, a CUDA stream.
+ *
+ * Passages cited below (page title, section):
+ *  [OC3-ja]  "Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ"
+ *            (agentlenshq.com), section "ルーティングと計算の最適化": routed
+ *            tokens are written directly into the experts' input buffers
+ *            ("rowwise" dispatch), routing metadata stays on the GPU so the
+ *            CPU is never a bottleneck, and many small per-expert matmuls are
+ *            batched into one grouped GEMM.  Section "MXFP8による精度最適化":
+ *            MXFP8 as the low-precision format of the expert feed-forward
+ *            compute.  Section "実証されたスケール": random routing used to
+ *            stress the system.
+ *  [OC3-hu]  "Az Ai2 megnyitotta az Olmo-core 3 MoE-tréningrendszerét"
+ *            (aihirek.info), first section: 8 -> 128 experts with four chosen
+ *            per token; section "Billió paraméteres tesztek, nyílt
+ *            hozzáférés": rowwise dispatch, GPU-resident routing, grouped GEMM.
+ *  [OC3-th]  "เปิดตัว Olmo-core 3 ..." (ai4bro.com), section on scaling and
+ *            optimising MoE training: GPU-resident routing lets the CPU queue
+ *            work without waiting for copies.
+ *  [JUPITER] "PyTorch、欧州の公共スパコンで約1兆パラメータMoEを訓練"
+ *            (cctest.ai), model paragraph: 384 experts, top-8, hidden 6144.
+ *
+ * The layer (its formulas are not printed on the pages; this is the layer
+ * definition the library implements):
+ *   logits  L = x W_r (+ b)                       x [T,d] bf16, W_r [d,E] fp32
+ *   top-k   k largest logits per token, ties -> lower expert index
+ *   gates   softmax over the k chosen logits (= softmax over E, renormalised)
+ *   expert  y_e(x) = (silu(x W1[e]) * (x W3[e])) W2[e]
+ *   out[t]  = sum_j gates[t,j] * y_{topk[t,j]}(x[t])
+ *
+ * Conventions for every call:
+ *  - Asynchronous and stream-ordered on `stream`; never synchronises the
+ *    host, never allocates device memory.  The caller owns every buffer.
+ *  - Device pointers unless stated otherwise; 16-byte aligned.
+ *  - bf16 arrays are passed as `void*` (IEEE bfloat16 bit patterns).
+ *  - All matrices row-major.  Weight layout: W1, W3 [E,d,F]; W2 [E,F,d];
+ *    W_r [d,E].
+ *  - Returns MOE_OK, or an error code with nothing enqueued (argument
+ *    errors) or after a failed launch (MOE_ERR_CUDA).  moe_last_error()
+ *    gives a message for the calling thread.
+ *  - Data errors found on the device (an expert index out of range, a
+ *    duplicate expert in a token, a pipeline wait that gave up) are OR-ed
+ *    into the caller's `int32_t* dev_status` word (MOE_DEV_* bits; may be
+ *    NULL), which the caller reads whenever it chooses.  No kernel traps.
+ *
+ * Routing metadata (bit-exact, GPU resident):
+ *   counts[E]     assignments per expert
+ *   offsets[E+1]  exclusive scan of counts
+ *   poff[E+1]     exclusive scan of counts rounded up to `align` (= 128):
+ *                 group e occupies rows [poff[e], poff[e+1]) of every
+ *                 expert-contiguous buffer; its first counts[e] rows are real,
+ *                 the rest are zero pad rows
+ *   dst[T,k]      permuted row of assignment (t,j) =
+ *                 poff[e] + #{t' < t : expert e chosen by t'}  (stable)
+ *   src[A_pad_max] token of each permuted row, -1 for pad rows
+ *   A_pad_max     = T*k + E*(align-1), the host-known bound on poff[E]
+ *
+ * MX (MXFP8) tensors: codes are E4M3FN bytes with the shape of the source;
+ * one E8M0 scale byte per 32 elements along the GEMM's K axis, with
+ * X = 2^(floor(log2 amax) - 8), round-to-nearest-even, saturation at 448;
+ * an all-zero block gets byte 0.  Scales are stored in the tensor-core
+ * layout: for a source [R, C] quantised along axis a (a = 0: blocks along a
+ * row, K = C, MN = R; a = 1: blocks down a column, K = R, MN = C), the scale
+ * of (mn, kb) (kb = K index / 32) sits at byte
+ *   ((mn/128) * (K/128) + kb/4) * 512 + (mn%32)*16 + ((mn/32)%4)*4 + kb%4.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t (NULL = legacy default) */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* a size, pointer, alignment or mode is not accepted */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+  MOE_ERR_WORKSPACE = 3,    /* workspace / context smaller than the query says */
+  MOE_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  MOE_ERR_TIMEOUT = 5,      /* reserved: host-visible form of MOE_DEV_TIMEOUT */
+  MOE_ERR_DEVICE_DATA = 6   /* reserved: host-visible form of the MOE_DEV_* data bits */
+} moe_status_t;
+
+/* bits OR-ed into *dev_status by kernels */
+#define MOE_DEV_BAD_EXPERT 0x1  /* a given expert index is outside [0, E) */
+#define MOE_DEV_DUP_EXPERT 0x2  /* a token lists the same expert twice */
+#define MOE_DEV_TIMEOUT 0x4     /* a GEMM pipeline wait gave up (bounded spin) */
+#define MOE_DEV_NONFINITE 0x8   /* a router logit was NaN or infinite */
+
+typedef enum { MOE_ROUTE_ROUTER = 0, MOE_ROUTE_GIVEN = 1 } moe_route_mode;
+typedef enum { MOE_BF16 = 0, MOE_MXFP8 = 1 } moe_dtype;
+typedef enum {
+  MOE_EPI_NONE = 0,       /* C = A B */
+  MOE_EPI_SWIGLU = 1,     /* fwd GEMM1: C = silu(A W1) * (A W3), aux = [A W1 | A W3] */
+  MOE_EPI_SWIGLU_BWD = 2  /* dgrad of GEMM2 fused with the SwiGLU backward */
+} moe_epilogue;
+
+/* Message for the last failed call on this thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+/* Library version string. */
+MOE_API const char* moe_version(void);
+
+/* ------------------------------------------------------------------ route
+ * Router and GPU-resident routing metadata ([OC3-ja] "ルーティングと計算の最適化":
+ * metadata kept on the GPU; [OC3-th]: the CPU queues work without waiting
+ * for copies; [OC3-hu] first section / [JUPITER]: k experts per token).
+ *
+ * mode MOE_ROUTE_ROUTER: logits = x W_r (+ bias) in fp32, top-k (ties to the
+ *   lower index, slot j = j-th largest), gates = softmax of the k chosen
+ *   logits (fp32); writes topk_idx [T,k] and gates [T,k].
+ * mode MOE_ROUTE_GIVEN: topk_idx and gates are INPUTS (random-routing stress
+ *   workload, [OC3-ja] "実証されたスケール"); x and W_r are not read.  An index
+ *   outside [0,E) or a repeat inside a token sets MOE_DEV_BAD_EXPERT /
+ *   MOE_DEV_DUP_EXPERT and that assignment is dropped (dst = -1).
+ * Both modes then write counts, offsets, poff, dst and src (see above).
+ *   logits: optional [T,E] fp32 copy of the router logits (ROUTER mode).
+ *   align must be 128.  Router mode needs E <= 512, k <= min(E, 16),
+ *   d % 8 == 0; given mode E <= 4096.
+ *   ws: device workspace of at least moe_route_workspace_size(T, E) bytes.
+ */
+MOE_API size_t moe_route_workspace_size(int T, int E);
+MOE_API moe_status_t moe_route(const void* x, const float* Wr, const float* bias, int T, int d,
+                       int E, int k, int align, int mode, int32_t* topk_idx, float* gates,
+                       int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* dst,
+                       int32_t* src, int A_pad_max, float* logits, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- permute
+ * Rowwise dispatch ([OC3-ja] "ルーティングと計算の最適化": routed tokens are
+ * written directly into the experts' input buffers): Xp[dst[t,j]] = x[t]
+ * for every assignment, and every pad row of every group is zeroed.
+ *   x [T,d] bf16; Xp [A_pad_max,d] bf16; d % 8 == 0.
+ *   Xq / Xs (both NULL or both set): additionally writes the MX codes of Xp
+ *   [A_pad_max,d] and its scales along d (axis 0) -- MX requires d % 128 == 0.
+ */
+MOE_API moe_status_t moe_permute(const void* x, const int32_t* dst, const int32_t* offsets,
+                         const int32_t* poff, int T, int k, int d, int E, int A_pad_max,
+                         void* Xp, uint8_t* Xq, uint8_t* Xs, moe_stream_t stream);
+
+/* ------------------------------------------------------------- mx_quantize
+ * MX quantiser ([OC3-ja] "MXFP8による精度最適化"; rule in the file header).
+ *   in [rows, cols] bf16.  axis 0: blocks of 32 along each row (K = cols);
+ *   axis 1: blocks of 32 down each column (K = rows).  rows % 128 == 0 and
+ *   cols % 128 == 0.  `poff` is accepted for documentation of grouped use:
+ *   with axis 1 every group start must be a multiple of 128 (true for the
+ *   routing metadata above), so no block crosses a group; it may be NULL.
+ *   codes [rows, cols] u8; scales rows*cols/32 bytes in the layout above.
+ *   `nrows_dev` (nullable device int): rows at and beyond *nrows_dev are
+ *   skipped (their codes and scales are left as they are).
+ */
+MOE_API moe_status_t mx_quantize(const void* in, int rows, int cols, int axis, const int32_t* poff,
+                         int E, const int32_t* nrows_dev, uint8_t* codes, uint8_t* scales,
+                         moe_stream_t stream);
+
+/* ------------------------------------------------------- grouped GEMMs
+ * Grouped GEMM over the expert groups of the routing metadata ([OC3-ja]
+ * "ルーティングと計算の最適化": many small per-expert matmuls as one grouped
+ * GEMM).  tcgen05 tensor cores, TMEM accumulators, TMA-fed shared-memory
+ * pipeline, persistent CTAs walking a device-side tile schedule read from
+ * poff (no host sync).  fp32 accumulation, bf16 outputs.
+ *
+ * Rows of group e are [poff[e], poff[e+1]); poff[E] <= A_pad_max; every
+ * poff entry is a multiple of 128.  Shapes: K % 64 == 0 (BF16) or
+ * K % 128 == 0 (MXFP8); N % 256 == 0 (N % 128 for SWIGLU halves).
+ *
+ * moe_grouped_gemm_fwd: for every row r of group e,
+ *   EPI_NONE:   C[r, :N]  = A[r, :K] B[e]             B [E,K,N]
+ *   EPI_SWIGLU: H1 = A[r] B[e], H3 = A[r] B3[e]        B, B3 [E,K,N], N = F
+ *               C[r, :F] = silu(H1) * H3; aux (nullable) [A_pad_max, 2F]
+ *               receives [H1 | H3] in bf16.
+ *   dt == MOE_MXFP8: A, B, B3 are MX codes with scales A_sc (axis 0 of A),
+ *   B_sc / B3_sc (axis 1 of the [E*K, N] view).
+ */
+MOE_API moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc, const void* B,
+                                  const uint8_t* B_sc, const void* B3, const uint8_t* B3_sc,
+                                  const int32_t* poff, int E, int A_pad_max, int N, int K,
+                                  int epilogue, void* C, void* aux, int32_t* dev_status,
+                                  moe_stream_t stream);
+
+/* moe_grouped_gemm_dgrad: gradient through B[e] (B [E,K,N] as in fwd):
+ *   EPI_NONE, B3 == NULL: dA[r, :K] = dC[r, :N] B[e]^T
+ *   EPI_NONE, B3 != NULL: dC has 2N columns; dA = dC[:, :N] B[e]^T + dC[:, N:] B3[e]^T
+ *   EPI_SWIGLU_BWD (B = W2 [E,F,d], so K = F, N = d): dh = dC B[e]^T and,
+ *     with aux = [H1 | H3] [A_pad_max, 2F] from the forward,
+ *     dA[r, :F]  = dh * H3 * s * (1 + H1 (1 - s)),  s = sigmoid(H1)
+ *     dA[r, F:]  = dh * silu(H1)                     (dA is [A_pad_max, 2F])
+ *   dt == MOE_MXFP8: dC codes with dC_sc along its columns (axis 0); B / B3
+ *   codes with scales along N, i.e. axis 0 of the [E*K, N] view.
+ */
+MOE_API moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc,
+                                    const void* B, const uint8_t* B_sc, const void* B3,
+                                    const uint8_t* B3_sc, const int32_t* poff, int E,
+                                    int A_pad_max, int N, int K, int epilogue, const void* aux,
+                                    void* dA, int32_t* dev_status, moe_stream_t stream);
+
+/* moe_grouped_gemm_wgrad: weight gradient, reduction over the rows of each
+ * group:  dB[e][:K, :N] = A_e^T dC_e, A [A_pad_max, K], dC [A_pad_max, N].
+ *   dB3 != NULL: dC has 2N columns; dB[e] = A_e^T dC_e[:, :N] and
+ *   dB3[e] = A_e^T dC_e[:, N:].  Empty groups give zero gradients.
+ *   Pad rows must be zero in A or dC (they are, for buffers written by this
+ *   library).  dt == MOE_MXFP8: A and dC codes with scales down the columns
+ *   (axis 1).
+ */
+MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, const void* dC,
+                                    const uint8_t* dC_sc, const int32_t* poff, int E,
+                                    int A_pad_max, int K, int N, void* dB, void* dB3,
+                                    int32_t* dev_status, moe_stream_t stream);
+
+/* -------------------------------------------------- unpermute / combine
+ * Gate-weighted combine (the unpermute half of the rowwise dispatch of
+ * [OC3-ja]): out[t] = sum_{j<k} gates[t,j] * Y[dst[t,j]], fp32 sum in slot
+ * order, bf16 result.  gates == NULL gives the plain sum.  dst entries < 0
+ * contribute nothing.  d % 8 == 0.
+ */
+MOE_API moe_status_t moe_unpermute_combine(const void* Y, const float* gates, const int32_t* dst,
+                                   int T, int k, int d, void* out, moe_stream_t stream);
+
+/* Backward of the combine: for each assignment (t,j) with r = dst[t,j]
+ *   dY[r]    = bf16(gates[t,j] * dout[t]);  pad rows of dY are zeroed
+ *   dg[t,j]  = <dout[t], Y[r]>  (fp32)
+ *   and, when dl != NULL (router mode), the logit gradient of the chosen
+ *   experts dl[t,j] = g_j (dg_j - sum_i g_i dg_i) (fp32), also scattered to
+ *   dl_rows[r] (nullable, [A_pad_max] fp32, pad rows untouched).
+ */
+MOE_API moe_status_t moe_combine_bwd(const void* dout, const void* Y, const float* gates,
+                             const int32_t* dst, const int32_t* offsets, const int32_t* poff,
+                             int T, int k, int d, int E, void* dY, float* dg, float* dl,
+                             float* dl_rows, moe_stream_t stream);
+
+/* Backward of the dispatch: dx[t] = sum_j dXp[dst[t,j]]
+ *   (+ sum_j dl[t,j] W_r[:, topk_idx[t,j]] when Wr != NULL: the router's
+ *   input gradient), fp32 sum, bf16 result.  ws: at least
+ *   moe_unpermute_sum_workspace_size(d, E) bytes (a transposed W_r).
+ */
+MOE_API size_t moe_unpermute_sum_workspace_size(int d, int E);
+MOE_API moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst, const int32_t* topk_idx,
+                               const float* dl, const float* Wr, int T, int k, int d, int E,
+                               void* dx, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Router weight gradient: dWr[i, e] = sum over the real rows r of group e
+ * of x[src[r], i] * dl_rows[r]  (= x^T dL with dL nonzero only at the chosen
+ * experts), fp32 [d, E].
+ */
+MOE_API moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const float* dl_rows,
+                              const int32_t* offsets, const int32_t* poff, int T, int d, int E,
+                              float* dWr, moe_stream_t stream);
+
+/* --------------------------------------------------------------- layer
+ * The whole layer: route -> permute -> GEMM1+SwiGLU -> GEMM2 -> combine, and
+ * its backward.  All saved tensors live in the caller's context buffer
+ * `ctx` of at least moe_layer_ctx_bytes(desc) bytes (256-byte aligned).
+ */
+typedef struct {
+  int T, d, E, k, F;
+  int align;       /* must be 128 */
+  int route_mode;  /* moe_route_mode */
+  int dtype;       /* moe_dtype of the grouped GEMMs */
+} moe_layer_desc;
+
+typedef struct {
+  const float* Wr;         /* [d,E] fp32 (router mode) */
+  const float* bias;       /* [E] fp32, nullable (router mode, constant) */
+  const void* W1;          /* [E,d,F] bf16 */
+  const void* W3;          /* [E,d,F] bf16 */
+  const void* W2;          /* [E,F,d] bf16 */
+  const int32_t* topk_idx; /* [T,k], given mode */
+  const float* gates;      /* [T,k], given mode */
+} moe_layer_weights;
+
+typedef struct {
+  void* dW1;   /* [E,d,F] bf16 */
+  void* dW3;   /* [E,d,F] bf16 */
+  void* dW2;   /* [E,F,d] bf16 */
+  float* dWr;  /* [d,E] fp32 (router mode; nullable) */
+} moe_layer_grads;
+
+/* Pointers into a context buffer (for inspection and tests). */
+typedef struct {
+  int32_t *topk_idx, *counts, *offsets, *poff, *dst, *src;
+  float *gates, *logits, *dg, *dl, *dl_rows;
+  void *Xp, *H13, *h, *Y, *dY, *dA13, *dXp;        /* bf16 */
+  uint8_t *Xp_q, *Xp_s, *W13_q, *W13_s, *W2_q, *W2_s, *h_q, *h_s;  /* MX (fwd) */
+  uint8_t *dY_q, *dY_s, *W13t_q, *W13t_s, *W2t_q, *W2t_s, *dA_q, *dA_s;  /* MX (bwd) */
+  uint8_t *hT_q, *hT_s, *dYT_q, *dYT_s, *XpT_q, *XpT_s, *dAT_q, *dAT_s;  /* MX (wgrad) */
+  void* ws;
+  size_t ws_bytes;
+  int A_pad_max;
+} moe_ctx_view;
+
+MOE_API size_t moe_layer_ctx_bytes(const moe_layer_desc* desc);
+MOE_API moe_status_t moe_layer_ctx_view(const moe_layer_desc* desc, void* ctx, moe_ctx_view* view);
+
+MOE_API moe_status_t moe_layer_fwd(const moe_layer_desc* desc, const moe_layer_weights* w,
+                           const void* x, void* out, void* ctx, size_t ctx_bytes,
+                           int32_t* dev_status, moe_stream_t stream);
+
+MOE_API moe_status_t moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_weights* w,
+                           const void* x, void* ctx, size_t ctx_bytes, const void* dout,
+                           void* dx, moe_layer_grads* grads, int32_t* dev_status,
+                           moe_stream_t stream);
+
+/* One training step of the layer from HOST buffers: copies x and dout
+ * (pinned host memory recommended) to the device buffers x_dev / dout_dev,
+ * runs moe_layer_fwd and moe_layer_bwd, and copies out and dx back to
+ * out_host / dx_host (all copies cudaMemcpyAsync on `stream`; the call
+ * returns once they are enqueued -- synchronise the stream before reading
+ * the host outputs).
+ */
+MOE_API moe_status_t moe_layer_step_host(const moe_layer_desc* desc, const moe_layer_weights* w,
+                                 const void* x_host, const void* dout_host, void* out_host,
+                                 void* dx_host, void* x_dev, void* dout_dev, void* out_dev,
+                                 void* dx_dev, void* ctx, size_t ctx_bytes,
+                                 moe_layer_grads* grads, int32_t* dev_status,
+                                 moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

@@ -1,0 +1,89 @@
+// Shared device/host helpers of libmoe (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libmoe targets sm_100a (B200) only"
+#endif
+
+namespace moe {
+
+// ---------------------------------------------------------------- host side
+void set_error(const char* fmt, ...);
+
+#define MOE_CHECK_ARG(cond, ...)                     \
+  do {                                               \
+    if (!(cond)) {                                   \
+      ::moe::set_error(__VA_ARGS__);                 \
+      return MOE_ERR_INVALID_ARG;                    \
+    }                                                \
+  } while (0)
+
+#define MOE_CHECK_LAUNCH(what)                                                   \
+  do {                                                                           \
+    cudaError_t e_ = cudaGetLastError();                                         \
+    if (e_ != cudaSuccess) {                                                     \
+      ::moe::set_error("%s: %s", what, cudaGetErrorString(e_));                  \
+      return MOE_ERR_CUDA;                                                       \
+    }                                                                            \
+  } while (0)
+
+#define MOE_TRY(expr)                         \
+  do {                                        \
+    moe_status_t s_ = (expr);                 \
+    if (s_ != MOE_OK) return s_;              \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int num_sms();
+
+// ---------------------------------------------------------------- device side
+__device__ __forceinline__ void report(int32_t* status, int32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// 8 bf16 <-> 8 fp32 through one 16-byte vector
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 v;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace moe

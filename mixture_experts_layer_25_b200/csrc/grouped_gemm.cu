@@ -1,0 +1,693 @@
+// Grouped GEMM over expert groups on the 5th-generation tensor cores.
+//
+// Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ, section
+// "ルーティングと計算の最適化": the many small per-expert matmuls are batched
+// into one grouped GEMM; section "MXFP8による精度最適化": MXFP8 for the expert
+// feed-forward compute.
+//
+// Design (sm_100a):
+//  * persistent CTAs (one per SM), 192 threads: warp 0 issues TMA loads,
+//    warp 1 issues tcgen05.mma (one thread) and owns TMEM, warps 2..5 are
+//    the epilogue (one accumulator row per thread, TMEM -> registers ->
+//    global).
+//  * tile 128 x 256, fp32 accumulators in TMEM (two buffers for BF16, so the
+//    epilogue of tile i overlaps the main loop of tile i+1), a 4-stage
+//    shared-memory ring fed by TMA with 128-byte swizzle.
+//  * device-side tile schedule read from poff: "rows" mode walks the
+//    128-row tiles of the expert-contiguous buffer (every group starts on a
+//    multiple of 128, so a tile never mixes experts) times the N tiles;
+//    "wgrad" mode walks (expert, M tile, N tile) and reduces over the rows
+//    of the expert's group.
+//  * every mbarrier wait is bounded; a wait that gives up raises
+//    MOE_DEV_TIMEOUT in the caller's status word and the CTA drains and
+//    exits.
+//  * MXFP8: E4M3 operands with kind::mxf8f6f4.block_scale; the E8M0 scales
+//    of each stage are bulk-copied to shared memory and moved into TMEM
+//    with tcgen05.cp; one accumulator buffer (TMEM also holds the scales).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace gg {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr int A_BYTES = BM * 128;   // 128-byte rows (64 bf16 or 128 fp8 of K)
+constexpr int B_BYTES = BN * 128;
+constexpr int SFA_BYTES = 512;      // 128 rows x 4 scale bytes
+constexpr int SFB_BYTES = 1024;     // 256 rows x 4 scale bytes
+constexpr int MAX_E = 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+
+enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2 };
+enum BLoad { B_MN = 0, B_MN_DUAL_N = 1, B_K = 2, B_K_DUAL_K = 3 };
+
+struct Params {
+  const int32_t* poff;
+  int E;
+  int wgrad;          // 0: rows mode; 1: weight-gradient mode
+  int n_tiles;        // tiles along N
+  int m_tiles_w;      // wgrad: M tiles (K_out / 128)
+  int num_kb;         // rows mode: K blocks per tile
+  int b_rows_per_e;   // rows of the B tensor map per expert (rows mode)
+  int k_split;        // B_K_DUAL_K: first K index taken from B3
+  // MX scales (byte pointers into the tensor-core scale layout)
+  const uint8_t* a_sc; int a_sc_kchunks;
+  const uint8_t* b_sc; const uint8_t* b3_sc; int b_sc_kchunks;
+  // epilogue
+  __nv_bfloat16* C; long long ldc;
+  __nv_bfloat16* C2; int n_split;
+  __nv_bfloat16* aux; long long ld_aux; int half;
+  long long c_expert_stride;
+  int32_t* status;
+};
+
+struct Tile {
+  int e, row0, m0, nt, nkb, krow0;
+};
+
+__device__ __forceinline__ int find_expert(const int* poff_s, int E, int row) {
+  int lo = 0, hi = E - 1;       // largest e with poff[e] <= row
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (poff_s[mid] <= row) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ Tile decode(const Params& p, const int* poff_s, int tile) {
+  Tile t;
+  if (!p.wgrad) {
+    const int mt = tile / p.n_tiles;
+    t.nt = tile - mt * p.n_tiles;
+    t.row0 = mt * BM;
+    t.e = find_expert(poff_s, p.E, t.row0);
+    t.m0 = t.row0;
+    t.nkb = p.num_kb;
+    t.krow0 = 0;
+  } else {
+    const int per_e = p.m_tiles_w * p.n_tiles;
+    t.e = tile / per_e;
+    const int rem = tile - t.e * per_e;
+    const int mt = rem / p.n_tiles;
+    t.nt = rem - mt * p.n_tiles;
+    t.m0 = mt * BM;
+    t.row0 = 0;
+    t.krow0 = poff_s[t.e];
+    t.nkb = -1;   // set by the caller from the group size and BK
+  }
+  return t;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) { return pack2(a, b); }
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+template <bool MX>
+__device__ __forceinline__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
+  if constexpr (!MX) {
+    return (1u << 4)              // D: fp32
+           | (1u << 7)            // A: bf16
+           | (1u << 10)           // B: bf16
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  } else {
+    return (0u << 7) | (0u << 10)   // A, B: E4M3
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(BN >> 3) << 17) | (1u << 23)   // scales: E8M0
+           | ((uint32_t)(BM >> 4) << 24);
+  }
+}
+
+template <bool MX, bool A_MN, int BLOAD, int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB3, const Params p) {
+  constexpr int ELEM = MX ? 1 : 2;
+  constexpr int BK = 128 / ELEM;                 // K per stage (128-byte rows)
+  constexpr int MMA_K = MX ? 32 : 16;
+  constexpr int KSTEPS = BK / MMA_K;             // 4
+  constexpr bool B_MNMAJOR = (BLOAD == B_MN || BLOAD == B_MN_DUAL_N);
+  constexpr int MN_CHUNK = 128 / ELEM;           // MN elements per 128-byte swizzle row
+  constexpr int MN_CHUNK_BYTES = BK * 128;       // one box of an MN-major operand
+  constexpr int ACC_BUFS = MX ? 1 : 2;
+  constexpr int SF_COL0 = 256 * ACC_BUFS;        // TMEM column of the first scale stage
+  constexpr uint32_t TMEM_COLS = MX ? 512 : 512;
+  constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + (MX ? SFA_BYTES + SFB_BYTES : 0);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int poff_s[MAX_E + 1];
+  __shared__ volatile int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;                                  // STAGES x A_BYTES
+  uint8_t* sB = smem + STAGES * A_BYTES;               // STAGES x B_BYTES
+  uint8_t* sSF = sB + STAGES * B_BYTES;                // STAGES x (SFA + SFB), MX only
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) poff_s[i] = p.poff[i];
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    mbar_init(&drain_bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&tmA);
+    tma_prefetch(&tmB);
+    if (BLOAD == B_MN_DUAL_N || BLOAD == B_K_DUAL_K) tma_prefetch(&tmB3);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+
+  const int total = p.wgrad ? p.E * p.m_tiles_w * p.n_tiles : (poff_s[p.E] / BM) * p.n_tiles;
+  auto group_kb = [&](const Tile& t) {
+    return p.wgrad ? (poff_s[t.e + 1] - poff_s[t.e]) / BK : t.nkb;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0;               // stages that ever received a load
+      uint32_t last_parity = 0;        // parity of the last load per stage (bit s)
+      for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+        const Tile t = decode(p, poff_s, tile);
+        const int nkb = group_kb(t);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
+          uint64_t* fb = &full_bar[stage];
+          mbar_arrive_expect_tx(fb, STAGE_TX);
+          uint8_t* a_dst = sA + stage * A_BYTES;
+          uint8_t* b_dst = sB + stage * B_BYTES;
+          // A operand
+          if constexpr (!A_MN) {
+            tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
+          } else {
+#pragma unroll
+            for (int i = 0; i < BM / MN_CHUNK; ++i)
+              tma_load_2d(a_dst + i * MN_CHUNK_BYTES, &tmA, fb, t.m0 + i * MN_CHUNK,
+                          t.krow0 + kb * BK);
+          }
+          // B operand
+          const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
+          if constexpr (BLOAD == B_MN) {
+#pragma unroll
+            for (int i = 0; i < BN / MN_CHUNK; ++i)
+              tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * BN + i * MN_CHUNK,
+                          brow + kb * BK);
+          } else if constexpr (BLOAD == B_MN_DUAL_N) {
+            constexpr int HALF_CHUNKS = (BN / 2) / MN_CHUNK;
+#pragma unroll
+            for (int i = 0; i < HALF_CHUNKS; ++i) {
+              tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * (BN / 2) + i * MN_CHUNK,
+                          brow + kb * BK);
+              tma_load_2d(b_dst + (HALF_CHUNKS + i) * MN_CHUNK_BYTES, &tmB3, fb,
+                          t.nt * (BN / 2) + i * MN_CHUNK, brow + kb * BK);
+            }
+          } else if constexpr (BLOAD == B_K) {
+            tma_load_2d(b_dst, &tmB, fb, kb * BK, brow + t.nt * BN);
+          } else {
+            const int k = kb * BK;
+            if (k < p.k_split) tma_load_2d(b_dst, &tmB, fb, k, brow + t.nt * BN);
+            else tma_load_2d(b_dst, &tmB3, fb, k - p.k_split, brow + t.nt * BN);
+          }
+          if constexpr (MX) {
+            uint8_t* sf = sSF + stage * (SFA_BYTES + SFB_BYTES);
+            // A scales: one 512-byte chunk (128 MN rows x 4 K blocks)
+            long long ca;
+            if constexpr (!A_MN) ca = (long long)(t.row0 / 128) * p.a_sc_kchunks + kb;
+            else ca = (long long)(t.m0 / 128) * p.a_sc_kchunks + (t.krow0 / 128 + kb);
+            bulk_load(sf, p.a_sc + ca * 512, SFA_BYTES, fb);
+            // B scales: two chunks (N rows 0..127 and 128..255 of the tile)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint8_t* base = p.b_sc;
+              long long cb;
+              if constexpr (BLOAD == B_MN) {
+                const long long nb = (long long)(t.nt * BN) / 128 + h;
+                cb = nb * p.b_sc_kchunks + (brow / 128 + kb);
+              } else if constexpr (BLOAD == B_MN_DUAL_N) {
+                base = h ? p.b3_sc : p.b_sc;
+                cb = (long long)t.nt * p.b_sc_kchunks + (brow / 128 + kb);
+              } else if constexpr (BLOAD == B_K) {
+                cb = ((long long)(brow + t.nt * BN) / 128 + h) * p.b_sc_kchunks + kb;
+              } else {
+                const int k = kb * BK;
+                int kk = kb;
+                if (k >= p.k_split) { base = p.b3_sc; kk = (k - p.k_split) / BK; }
+                cb = ((long long)(brow + t.nt * BN) / 128 + h) * p.b_sc_kchunks + kk;
+              }
+              bulk_load(sf + SFA_BYTES + h * 512, base + cb * 512, 512, fb);
+            }
+          }
+          used |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // drain: every load this thread issued has landed before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (used & (1u << s)) {
+          volatile int no_abort = 0;
+          mbar_wait(&full_bar[s], (last_parity >> s) & 1, &no_abort, p.status, kWaitLimitNs);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t IDESC = make_idesc<MX>(A_MN, B_MNMAJOR);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+      for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x, ++it) {
+        const Tile t = decode(p, poff_s, tile);
+        const int nkb = group_kb(t);
+        const int acc = ACC_BUFS == 2 ? (it & 1) : 0;
+        const uint32_t acc_par = ACC_BUFS == 2 ? ((it >> 1) & 1) : (it & 1);
+        if (!mbar_wait(&acc_empty[acc], acc_par ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * 256;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, p.status, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = a_base + stage * A_BYTES, sb = b_base + stage * B_BYTES;
+          uint32_t sfa_t = 0, sfb_t = 0;
+          if constexpr (MX) {
+            const uint32_t sf = smem_u32(sSF + stage * (SFA_BYTES + SFB_BYTES));
+            sfa_t = tmem_base + SF_COL0 + stage * 12;
+            sfb_t = sfa_t + 4;
+            tmem_cp_32x128b_warpx4(sfa_t, smem_desc(sf, 0, 128, 0));
+            tmem_cp_32x128b_warpx4(sfb_t, smem_desc(sf + SFA_BYTES, 0, 128, 0));
+            tmem_cp_32x128b_warpx4(sfb_t + 4, smem_desc(sf + SFA_BYTES + 512, 0, 128, 0));
+          }
+#pragma unroll
+          for (int ks = 0; ks < KSTEPS; ++ks) {
+            uint64_t ad, bd;
+            if constexpr (!A_MN) ad = smem_desc(sa + ks * 32, 16, 1024, 2);
+            else ad = smem_desc(sa + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
+            if constexpr (!B_MNMAJOR) bd = smem_desc(sb + ks * 32, 16, 1024, 2);
+            else bd = smem_desc(sb + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
+            const uint32_t accum = (kb > 0 || ks > 0) ? 1u : 0u;
+            if constexpr (!MX) {
+              mma_bf16(d_tmem, ad, bd, IDESC, accum);
+            } else {
+              const uint32_t id = IDESC | ((uint32_t)ks << 4) | ((uint32_t)ks << 29);
+              mma_mxf8(d_tmem, ad, bd, id, accum, sfa_t, sfb_t);
+            }
+          }
+          mma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (nkb > 0) mma_commit(&acc_full[acc]);
+        else mbar_arrive(&acc_full[acc]);      // empty group: the epilogue writes zeros
+      }
+      // drain: all issued MMAs have completed before TMEM is released
+      mma_commit(&drain_bar);
+      volatile int no_abort = 0;
+      mbar_wait(&drain_bar, 0, &no_abort, p.status, kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = q * 32 + lane;            // accumulator row of this thread
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const Tile t = decode(p, poff_s, tile);
+      const int nkb = group_kb(t);
+      const int acc = ACC_BUFS == 2 ? (it & 1) : 0;
+      const uint32_t acc_par = ACC_BUFS == 2 ? ((it >> 1) & 1) : (it & 1);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_par, &abort_flag, p.status, kWaitLimitNs);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256;
+      const bool empty = nkb <= 0;
+
+      if constexpr (EPI == EPI_STORE) {
+        __nv_bfloat16* out;
+        const int n0 = t.nt * BN;
+        if (!p.wgrad) {
+          out = p.C + (long long)(t.row0 + r) * p.ldc + n0;
+        } else if (p.C2 && n0 >= p.n_split) {
+          out = p.C2 + (long long)t.e * p.c_expert_stride + (long long)(t.m0 + r) * p.ldc +
+                (n0 - p.n_split);
+        } else {
+          out = p.C + (long long)t.e * p.c_expert_stride + (long long)(t.m0 + r) * p.ldc + n0;
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          if (!empty) {
+            tmem_ld32(tbase + c, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          uint4* o = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 w;
+            w.x = bf16x2_bits(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+            w.y = bf16x2_bits(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+            w.z = bf16x2_bits(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+            w.w = bf16x2_bits(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+            o[i] = w;
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        // accumulator columns [0,128) = A W1, [128,256) = A W3 for the output
+        // columns [nt*128, nt*128 + 128)
+        const long long row = t.row0 + r;
+        const int n0 = t.nt * (BN / 2);
+        __nv_bfloat16* hout = p.C + row * p.ldc + n0;
+        __nv_bfloat16* a1 = p.aux ? p.aux + row * p.ld_aux + n0 : nullptr;
+        __nv_bfloat16* a3 = p.aux ? p.aux + row * p.ld_aux + p.half + n0 : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c, g);
+          tmem_ld32(tbase + BN / 2 + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint4 hw, gw, uw;
+            uint32_t* hp = &hw.x;
+            uint32_t* gp = &gw.x;
+            uint32_t* up = &uw.x;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float g0 = __uint_as_float(g[8 * i + 2 * j]);
+              const float g1 = __uint_as_float(g[8 * i + 2 * j + 1]);
+              const float u0 = __uint_as_float(u[8 * i + 2 * j]);
+              const float u1 = __uint_as_float(u[8 * i + 2 * j + 1]);
+              hp[j] = bf16x2_bits(silu_f(g0) * u0, silu_f(g1) * u1);
+              gp[j] = bf16x2_bits(g0, g1);
+              up[j] = bf16x2_bits(u0, u1);
+            }
+            reinterpret_cast<uint4*>(hout + c)[i] = hw;
+            if (a1) {
+              reinterpret_cast<uint4*>(a1 + c)[i] = gw;
+              reinterpret_cast<uint4*>(a3 + c)[i] = uw;
+            }
+          }
+        }
+      } else {  // EPI_SWIGLU_BWD: accumulator = dh for columns [nt*256, +256)
+        const long long row = t.row0 + r;
+        const int n0 = t.nt * BN;
+        const __nv_bfloat16* h1 = p.aux + row * p.ld_aux + n0;
+        const __nv_bfloat16* h3 = p.aux + row * p.ld_aux + p.half + n0;
+        __nv_bfloat16* d1 = p.C + row * p.ldc + n0;
+        __nv_bfloat16* d3 = p.C + row * p.ldc + p.half + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float f1[8], f3[8], o1[8], o3[8];
+            unpack8(reinterpret_cast<const uint4*>(h1 + c)[i], f1);
+            unpack8(reinterpret_cast<const uint4*>(h3 + c)[i], f3);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float dh = __uint_as_float(v[8 * i + j]);
+              const float z = f1[j];
+              const float s = 1.0f / (1.0f + __expf(-z));
+              o1[j] = dh * f3[j] * s * (1.0f + z * (1.0f - s));
+              o3[j] = dh * z * s;
+            }
+            reinterpret_cast<uint4*>(d1 + c)[i] = pack8(o1);
+            reinterpret_cast<uint4*>(d3 + c)[i] = pack8(o3);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [outer, inner] array of 1- or 2-byte elements,
+// box {box_inner, box_outer}, 128-byte swizzle.
+moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner,
+                      uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) {
+    set_error("cuTensorMapEncodeTiled unavailable");
+    return MOE_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (%d): inner %llu outer %llu box %u x %u", (int)r,
+              (unsigned long long)inner, (unsigned long long)outer, box_inner, box_outer);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+constexpr size_t smem_bytes(bool mx) {
+  return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + (mx ? SFA_BYTES + SFB_BYTES : 0));
+}
+
+template <bool MX, bool A_MN, int BLOAD, int EPI>
+moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3,
+                    const Params& p, int max_tiles, cudaStream_t s) {
+  auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI>;
+  const size_t smem = smem_bytes(MX);
+  static bool attr = false;   // one per instantiation
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+      set_error("grouped_gemm: smem attribute: %s", cudaGetErrorString(e));
+      return MOE_ERR_CUDA;
+    }
+    attr = true;
+  }
+  const int grid = max(1, min(num_sms(), max_tiles));
+  kern<<<grid, NUM_THREADS, smem, s>>>(a, b, b3, p);
+  MOE_CHECK_LAUNCH("grouped_gemm");
+  return MOE_OK;
+}
+
+}  // namespace gg
+}  // namespace moe
+
+using namespace moe;
+using namespace moe::gg;
+
+static Params base_params(const int32_t* poff, int E, int32_t* status) {
+  Params p{};
+  p.poff = poff;
+  p.E = E;
+  p.status = status;
+  return p;
+}
+
+extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc,
+                                             const void* B, const uint8_t* B_sc, const void* B3,
+                                             const uint8_t* B3_sc, const int32_t* poff, int E,
+                                             int A_pad_max, int N, int K, int epilogue, void* C,
+                                             void* aux, int32_t* dev_status,
+                                             moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool mx = dt == MOE_MXFP8;
+  MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_fwd: bad dtype");
+  MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_fwd: E must be in [1, %d]", MAX_E);
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_fwd: A_pad_max %% 128");
+  MOE_CHECK_ARG(K > 0 && K % (mx ? 128 : 64) == 0, "gemm_fwd: K %% %d", mx ? 128 : 64);
+  MOE_CHECK_ARG(A && B && C && poff, "gemm_fwd: null pointer");
+  MOE_CHECK_ARG(!mx || (A_sc && B_sc), "gemm_fwd: MX needs scales");
+  const int eb = mx ? 1 : 2;
+  Params p = base_params(poff, E, dev_status);
+  p.num_kb = K / (128 / eb);
+  p.b_rows_per_e = K;
+  p.a_sc = A_sc;
+  p.a_sc_kchunks = K / 128;
+  p.b_sc = B_sc;
+  p.b3_sc = B3_sc;
+  p.b_sc_kchunks = (int)((long long)E * K / 128);
+  p.C = static_cast<__nv_bfloat16*>(C);
+  CUtensorMap ma, mb, mb3;
+  MOE_TRY(make_map(&ma, A, eb, K, A_pad_max, 128 / eb, BM));
+  if (epilogue == MOE_EPI_NONE) {
+    MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_fwd: N %% 256");
+    p.n_tiles = N / BN;
+    p.ldc = N;
+    MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+    return mx ? launch<true, false, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
+              : launch<false, false, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
+  }
+  MOE_CHECK_ARG(epilogue == MOE_EPI_SWIGLU, "gemm_fwd: epilogue must be NONE or SWIGLU");
+  MOE_CHECK_ARG(B3 && (!mx || B3_sc), "gemm_fwd: SWIGLU needs B3 (W3)");
+  MOE_CHECK_ARG(N > 0 && N % 128 == 0, "gemm_fwd: SWIGLU needs F %% 128");
+  p.n_tiles = N / (BN / 2);
+  p.ldc = N;
+  p.aux = static_cast<__nv_bfloat16*>(aux);
+  p.ld_aux = 2LL * N;
+  p.half = N;
+  MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  MOE_TRY(make_map(&mb3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+  return mx ? launch<true, false, B_MN_DUAL_N, EPI_SWIGLU>(ma, mb, mb3, p, max_tiles, s)
+            : launch<false, false, B_MN_DUAL_N, EPI_SWIGLU>(ma, mb, mb3, p, max_tiles, s);
+}
+
+extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc,
+                                               const void* B, const uint8_t* B_sc,
+                                               const void* B3, const uint8_t* B3_sc,
+                                               const int32_t* poff, int E, int A_pad_max, int N,
+                                               int K, int epilogue, const void* aux, void* dA,
+                                               int32_t* dev_status, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool mx = dt == MOE_MXFP8;
+  MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_dgrad: bad dtype");
+  MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_dgrad: E must be in [1, %d]", MAX_E);
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_dgrad: A_pad_max %% 128");
+  MOE_CHECK_ARG(N > 0 && N % (mx ? 128 : 64) == 0, "gemm_dgrad: N %% %d", mx ? 128 : 64);
+  MOE_CHECK_ARG(K > 0 && K % 256 == 0, "gemm_dgrad: K %% 256");
+  MOE_CHECK_ARG(dC && B && dA && poff, "gemm_dgrad: null pointer");
+  MOE_CHECK_ARG(!mx || (dC_sc && B_sc), "gemm_dgrad: MX needs scales");
+  const int eb = mx ? 1 : 2;
+  const bool dual = B3 != nullptr;
+  MOE_CHECK_ARG(!dual || epilogue == MOE_EPI_NONE, "gemm_dgrad: B3 only with EPI_NONE");
+  MOE_CHECK_ARG(!(dual && mx) || B3_sc, "gemm_dgrad: MX needs B3 scales");
+  const int Ktot = dual ? 2 * N : N;    // reduction length over dC's columns
+  Params p = base_params(poff, E, dev_status);
+  p.num_kb = Ktot / (128 / eb);
+  p.b_rows_per_e = K;
+  p.k_split = N;
+  p.n_tiles = K / BN;
+  p.a_sc = dC_sc;
+  p.a_sc_kchunks = Ktot / 128;
+  p.b_sc = B_sc;
+  p.b3_sc = B3_sc;
+  p.b_sc_kchunks = N / 128;
+  p.C = static_cast<__nv_bfloat16*>(dA);
+  CUtensorMap ma, mb, mb3;
+  MOE_TRY(make_map(&ma, dC, eb, Ktot, A_pad_max, 128 / eb, BM));
+  MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, BN));
+  const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+  if (epilogue == MOE_EPI_SWIGLU_BWD) {
+    MOE_CHECK_ARG(aux != nullptr, "gemm_dgrad: SWIGLU_BWD needs aux = [H1|H3]");
+    p.aux = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(aux));
+    p.ld_aux = 2LL * K;
+    p.half = K;
+    p.ldc = 2LL * K;
+    return mx ? launch<true, false, B_K, EPI_SWIGLU_BWD>(ma, mb, mb, p, max_tiles, s)
+              : launch<false, false, B_K, EPI_SWIGLU_BWD>(ma, mb, mb, p, max_tiles, s);
+  }
+  MOE_CHECK_ARG(epilogue == MOE_EPI_NONE, "gemm_dgrad: epilogue must be NONE or SWIGLU_BWD");
+  p.ldc = K;
+  if (!dual)
+    return mx ? launch<true, false, B_K, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
+              : launch<false, false, B_K, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
+  MOE_TRY(make_map(&mb3, B3, eb, N, (uint64_t)E * K, 128 / eb, BN));
+  return mx ? launch<true, false, B_K_DUAL_K, EPI_STORE>(ma, mb, mb3, p, max_tiles, s)
+            : launch<false, false, B_K_DUAL_K, EPI_STORE>(ma, mb, mb3, p, max_tiles, s);
+}
+
+extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc,
+                                               const void* dC, const uint8_t* dC_sc,
+                                               const int32_t* poff, int E, int A_pad_max, int K,
+                                               int N, void* dB, void* dB3, int32_t* dev_status,
+                                               moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool mx = dt == MOE_MXFP8;
+  MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_wgrad: bad dtype");
+  MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_wgrad: E must be in [1, %d]", MAX_E);
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_wgrad: A_pad_max %% 128");
+  MOE_CHECK_ARG(K > 0 && K % 128 == 0, "gemm_wgrad: K %% 128");
+  MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_wgrad: N %% 256");
+  MOE_CHECK_ARG(A && dC && dB && poff, "gemm_wgrad: null pointer");
+  MOE_CHECK_ARG(!mx || (A_sc && dC_sc), "gemm_wgrad: MX needs scales");
+  const int eb = mx ? 1 : 2;
+  const int Ncols = dB3 ? 2 * N : N;
+  Params p = base_params(poff, E, dev_status);
+  p.wgrad = 1;
+  p.m_tiles_w = K / BM;
+  p.n_tiles = Ncols / BN;
+  p.a_sc = A_sc;
+  p.a_sc_kchunks = A_pad_max / 128;
+  p.b_sc = dC_sc;
+  p.b_sc_kchunks = A_pad_max / 128;
+  p.C = static_cast<__nv_bfloat16*>(dB);
+  p.C2 = static_cast<__nv_bfloat16*>(dB3);
+  p.n_split = dB3 ? N : Ncols;
+  p.ldc = N;
+  p.c_expert_stride = (long long)K * N;
+  CUtensorMap ma, mb;
+  MOE_TRY(make_map(&ma, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
+  MOE_TRY(make_map(&mb, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  const int max_tiles = E * p.m_tiles_w * p.n_tiles;
+  return mx ? launch<true, true, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
+            : launch<false, true, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
+}

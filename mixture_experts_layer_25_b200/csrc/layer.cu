@@ -1,0 +1,257 @@
+// The whole MoE feed-forward layer, forward and backward, composed from the
+// library's calls on one stream with no host synchronisation.
+//
+// Forward:  route -> permute (rowwise dispatch) -> GEMM1 + SwiGLU -> GEMM2
+//           -> gate-weighted combine.
+// Backward: combine bwd (dY = g dout, dg, dl) -> GEMM2 dgrad fused with the
+//           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad -> GEMM1 wgrad ->
+//           unpermute-sum (+ router input grad) -> router weight grad.
+// In MXFP8 mode every GEMM operand is quantised along that GEMM's K first
+// (weights included, inside the step).
+#include "common.cuh"
+
+namespace {
+
+struct Layout {
+  size_t off = 0;
+  char* base = nullptr;
+  template <class T>
+  T* take(size_t count) {
+    off = moe::round_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+bool desc_ok(const moe_layer_desc* L) {
+  if (!L) return false;
+  if (L->T <= 0 || L->d <= 0 || L->E <= 0 || L->k <= 0 || L->F <= 0) return false;
+  if (L->align != 128 || L->k > L->E || L->k > 16) return false;
+  if (L->d % 256 || L->F % 256) return false;
+  if (L->route_mode != MOE_ROUTE_ROUTER && L->route_mode != MOE_ROUTE_GIVEN) return false;
+  if (L->dtype != MOE_BF16 && L->dtype != MOE_MXFP8) return false;
+  if (L->route_mode == MOE_ROUTE_ROUTER && L->E > 512) return false;
+  if (L->E > 1024) return false;
+  return true;
+}
+
+int a_pad_max(const moe_layer_desc* L) {
+  const long long a = (long long)L->T * L->k + (long long)L->E * (L->align - 1);
+  return (int)((a + 127) / 128 * 128);
+}
+
+size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
+  Layout l;
+  l.base = static_cast<char*>(base);
+  moe_ctx_view x{};
+  const size_t T = L->T, d = L->d, E = L->E, k = L->k, F = L->F;
+  const size_t A = a_pad_max(L);
+  x.A_pad_max = (int)A;
+  x.topk_idx = l.take<int32_t>(T * k);
+  x.gates = l.take<float>(T * k);
+  x.logits = L->route_mode == MOE_ROUTE_ROUTER ? l.take<float>(T * E) : nullptr;
+  x.counts = l.take<int32_t>(E);
+  x.offsets = l.take<int32_t>(E + 1);
+  x.poff = l.take<int32_t>(E + 1);
+  x.dst = l.take<int32_t>(T * k);
+  x.src = l.take<int32_t>(A);
+  x.dg = l.take<float>(T * k);
+  x.dl = l.take<float>(T * k);
+  x.dl_rows = l.take<float>(A);
+  x.Xp = l.take<__nv_bfloat16>(A * d);
+  x.H13 = l.take<__nv_bfloat16>(A * 2 * F);
+  x.h = l.take<__nv_bfloat16>(A * F);
+  x.Y = l.take<__nv_bfloat16>(A * d);
+  x.dXp = x.Y;   // Y is dead once the combine backward has run
+  x.dY = l.take<__nv_bfloat16>(A * d);
+  x.dA13 = l.take<__nv_bfloat16>(A * 2 * F);
+  if (L->dtype == MOE_MXFP8) {
+    x.Xp_q = l.take<uint8_t>(A * d);       x.Xp_s = l.take<uint8_t>(A * d / 32);
+    x.W13_q = l.take<uint8_t>(2 * E * d * F); x.W13_s = l.take<uint8_t>(2 * E * d * F / 32);
+    x.W2_q = l.take<uint8_t>(E * F * d);   x.W2_s = l.take<uint8_t>(E * F * d / 32);
+    x.h_q = l.take<uint8_t>(A * F);        x.h_s = l.take<uint8_t>(A * F / 32);
+    x.dY_q = l.take<uint8_t>(A * d);       x.dY_s = l.take<uint8_t>(A * d / 32);
+    x.W2t_q = l.take<uint8_t>(E * F * d);  x.W2t_s = l.take<uint8_t>(E * F * d / 32);
+    x.dA_q = l.take<uint8_t>(A * 2 * F);   x.dA_s = l.take<uint8_t>(A * 2 * F / 32);
+    x.W13t_q = l.take<uint8_t>(2 * E * d * F); x.W13t_s = l.take<uint8_t>(2 * E * d * F / 32);
+    x.hT_q = l.take<uint8_t>(A * F);       x.hT_s = l.take<uint8_t>(A * F / 32);
+    x.dYT_q = l.take<uint8_t>(A * d);      x.dYT_s = l.take<uint8_t>(A * d / 32);
+    x.XpT_q = l.take<uint8_t>(A * d);      x.XpT_s = l.take<uint8_t>(A * d / 32);
+    x.dAT_q = l.take<uint8_t>(A * 2 * F);  x.dAT_s = l.take<uint8_t>(A * 2 * F / 32);
+  }
+  const size_t ws_route = moe_route_workspace_size(L->T, L->E);
+  const size_t ws_unperm = moe_unpermute_sum_workspace_size(L->d, L->E);
+  x.ws_bytes = ws_route > ws_unperm ? ws_route : ws_unperm;
+  x.ws = l.take<uint8_t>(x.ws_bytes);
+  if (v) *v = x;
+  return moe::round_up(l.off, 256);
+}
+
+template <class T>
+T* bf(void* p) { return static_cast<T*>(p); }
+
+}  // namespace
+
+using moe::set_error;
+
+extern "C" size_t moe_layer_ctx_bytes(const moe_layer_desc* desc) {
+  if (!desc_ok(desc)) return 0;
+  return layout(desc, nullptr, nullptr);
+}
+
+extern "C" moe_status_t moe_layer_ctx_view(const moe_layer_desc* desc, void* ctx,
+                                           moe_ctx_view* view) {
+  MOE_CHECK_ARG(desc_ok(desc), "moe_layer_ctx_view: bad layer description");
+  MOE_CHECK_ARG(ctx && view, "moe_layer_ctx_view: null pointer");
+  layout(desc, ctx, view);
+  return MOE_OK;
+}
+
+static moe_status_t check_common(const moe_layer_desc* L, const moe_layer_weights* w, void* ctx,
+                                 size_t ctx_bytes) {
+  MOE_CHECK_ARG(desc_ok(L),
+                "moe_layer: bad description (align 128, d %% 256, F %% 256, k <= min(E,16), "
+                "router mode E <= 512, E <= 1024)");
+  MOE_CHECK_ARG(w && w->W1 && w->W3 && w->W2, "moe_layer: missing expert weights");
+  if (L->route_mode == MOE_ROUTE_ROUTER) MOE_CHECK_ARG(w->Wr, "moe_layer: router mode needs Wr");
+  else MOE_CHECK_ARG(w->topk_idx && w->gates, "moe_layer: given mode needs topk_idx and gates");
+  MOE_CHECK_ARG(ctx && (reinterpret_cast<uintptr_t>(ctx) & 255) == 0,
+                "moe_layer: ctx must be 256-byte aligned");
+  const size_t need = moe_layer_ctx_bytes(L);
+  if (ctx_bytes < need) {
+    set_error("moe_layer: ctx %zu < %zu bytes", ctx_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_weights* w,
+                                      const void* x, void* out, void* ctx, size_t ctx_bytes,
+                                      int32_t* dev_status, moe_stream_t stream) {
+  MOE_TRY(check_common(L, w, ctx, ctx_bytes));
+  MOE_CHECK_ARG(x && out, "moe_layer_fwd: null x/out");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  moe_ctx_view c;
+  layout(L, ctx, &c);
+  const int T = L->T, d = L->d, E = L->E, k = L->k, F = L->F, A = c.A_pad_max;
+  const bool mx = L->dtype == MOE_MXFP8;
+
+  if (L->route_mode == MOE_ROUTE_GIVEN) {
+    if (cudaMemcpyAsync(c.topk_idx, w->topk_idx, sizeof(int32_t) * T * k, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(c.gates, w->gates, sizeof(float) * T * k, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+      set_error("moe_layer_fwd: copy of the given routing failed");
+      return MOE_ERR_CUDA;
+    }
+  }
+  MOE_TRY(moe_route(x, w->Wr, w->bias, T, d, E, k, L->align, L->route_mode, c.topk_idx, c.gates,
+                    c.counts, c.offsets, c.poff, c.dst, c.src, A, c.logits, c.ws, c.ws_bytes,
+                    dev_status, stream));
+  if (!mx) {
+    MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, nullptr, nullptr, stream));
+    MOE_TRY(moe_grouped_gemm_fwd(MOE_BF16, c.Xp, nullptr, w->W1, nullptr, w->W3, nullptr, c.poff,
+                                 E, A, F, d, MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_fwd(MOE_BF16, c.h, nullptr, w->W2, nullptr, nullptr, nullptr, c.poff,
+                                 E, A, d, F, MOE_EPI_NONE, c.Y, nullptr, dev_status, stream));
+  } else {
+    const int32_t* nrows = c.poff + E;
+    uint8_t* W1q = c.W13_q; uint8_t* W3q = c.W13_q + (size_t)E * d * F;
+    uint8_t* W1s = c.W13_s; uint8_t* W3s = c.W13_s + (size_t)E * d * F / 32;
+    MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, c.Xp_q, c.Xp_s, stream));
+    // weights along the fwd GEMMs' K: W1/W3 down d, W2 down F
+    MOE_TRY(mx_quantize(w->W1, E * d, F, 1, nullptr, E, nullptr, W1q, W1s, stream));
+    MOE_TRY(mx_quantize(w->W3, E * d, F, 1, nullptr, E, nullptr, W3q, W3s, stream));
+    MOE_TRY(mx_quantize(w->W2, E * F, d, 1, nullptr, E, nullptr, c.W2_q, c.W2_s, stream));
+    MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.Xp_q, c.Xp_s, W1q, W1s, W3q, W3s, c.poff, E, A, F, d,
+                                 MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
+    MOE_TRY(mx_quantize(c.h, A, F, 0, c.poff, E, nrows, c.h_q, c.h_s, stream));
+    MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.h_q, c.h_s, c.W2_q, c.W2_s, nullptr, nullptr, c.poff,
+                                 E, A, d, F, MOE_EPI_NONE, c.Y, nullptr, dev_status, stream));
+  }
+  return moe_unpermute_combine(c.Y, c.gates, c.dst, T, k, d, out, stream);
+}
+
+extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w,
+                                      const void* x, void* ctx, size_t ctx_bytes,
+                                      const void* dout, void* dx, moe_layer_grads* G,
+                                      int32_t* dev_status, moe_stream_t stream) {
+  MOE_TRY(check_common(L, w, ctx, ctx_bytes));
+  MOE_CHECK_ARG(x && dout && dx && G && G->dW1 && G->dW3 && G->dW2, "moe_layer_bwd: null pointer");
+  const bool router = L->route_mode == MOE_ROUTE_ROUTER;
+  moe_ctx_view c;
+  layout(L, ctx, &c);
+  const int T = L->T, d = L->d, E = L->E, k = L->k, F = L->F, A = c.A_pad_max;
+  const bool mx = L->dtype == MOE_MXFP8;
+
+  MOE_TRY(moe_combine_bwd(dout, c.Y, c.gates, c.dst, c.offsets, c.poff, T, k, d, E, c.dY, c.dg,
+                          router ? c.dl : nullptr, router ? c.dl_rows : nullptr, stream));
+  if (!mx) {
+    MOE_TRY(moe_grouped_gemm_dgrad(MOE_BF16, c.dY, nullptr, w->W2, nullptr, nullptr, nullptr,
+                                   c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
+                                   dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, E, A, F, d,
+                                   G->dW2, nullptr, dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_dgrad(MOE_BF16, c.dA13, nullptr, w->W1, nullptr, w->W3, nullptr,
+                                   c.poff, E, A, F, d, MOE_EPI_NONE, nullptr, c.dXp, dev_status,
+                                   stream));
+    MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, E, A, d, F,
+                                   G->dW1, G->dW3, dev_status, stream));
+  } else {
+    const int32_t* nrows = c.poff + E;
+    uint8_t* W1q = c.W13t_q; uint8_t* W3q = c.W13t_q + (size_t)E * d * F;
+    uint8_t* W1s = c.W13t_s; uint8_t* W3s = c.W13t_s + (size_t)E * d * F / 32;
+    // GEMM2 dgrad: K = d.  dY along d, W2 along d (rows of the [E*F, d] view)
+    MOE_TRY(mx_quantize(c.dY, A, d, 0, c.poff, E, nrows, c.dY_q, c.dY_s, stream));
+    MOE_TRY(mx_quantize(w->W2, E * F, d, 0, nullptr, E, nullptr, c.W2t_q, c.W2t_s, stream));
+    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dY_q, c.dY_s, c.W2t_q, c.W2t_s, nullptr, nullptr,
+                                   c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
+                                   dev_status, stream));
+    // GEMM2 wgrad: K = rows of the group.  h and dY down their columns
+    MOE_TRY(mx_quantize(c.h, A, F, 1, c.poff, E, nrows, c.hT_q, c.hT_s, stream));
+    MOE_TRY(mx_quantize(c.dY, A, d, 1, c.poff, E, nrows, c.dYT_q, c.dYT_s, stream));
+    MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff, E, A, F,
+                                   d, G->dW2, nullptr, dev_status, stream));
+    // GEMM1 dgrad: K = 2F.  dA13 along 2F, W1/W3 along F
+    MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 0, c.poff, E, nrows, c.dA_q, c.dA_s, stream));
+    MOE_TRY(mx_quantize(w->W1, E * d, F, 0, nullptr, E, nullptr, W1q, W1s, stream));
+    MOE_TRY(mx_quantize(w->W3, E * d, F, 0, nullptr, E, nullptr, W3q, W3s, stream));
+    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, W1q, W1s, W3q, W3s, c.poff, E, A, F,
+                                   d, MOE_EPI_NONE, nullptr, c.dXp, dev_status, stream));
+    // GEMM1 wgrad: K = rows of the group.  Xp and dA13 down their columns
+    MOE_TRY(mx_quantize(c.Xp, A, d, 1, c.poff, E, nrows, c.XpT_q, c.XpT_s, stream));
+    MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 1, c.poff, E, nrows, c.dAT_q, c.dAT_s, stream));
+    MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff, E, A, d,
+                                   F, G->dW1, G->dW3, dev_status, stream));
+  }
+  MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, c.topk_idx, router ? c.dl : nullptr,
+                            router ? w->Wr : nullptr, T, k, d, E, dx, c.ws, c.ws_bytes, stream));
+  if (router && G->dWr)
+    MOE_TRY(moe_router_wgrad(x, c.src, c.dl_rows, c.offsets, c.poff, T, d, E, G->dWr, stream));
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_layer_weights* w,
+                                            const void* x_host, const void* dout_host,
+                                            void* out_host, void* dx_host, void* x_dev,
+                                            void* dout_dev, void* out_dev, void* dx_dev,
+                                            void* ctx, size_t ctx_bytes, moe_layer_grads* G,
+                                            int32_t* dev_status, moe_stream_t stream) {
+  MOE_TRY(check_common(L, w, ctx, ctx_bytes));
+  MOE_CHECK_ARG(x_host && dout_host && out_host && dx_host && x_dev && dout_dev && out_dev && dx_dev,
+                "moe_layer_step_host: null pointer");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)L->T * L->d * 2;
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    set_error("moe_layer_step_host: host-to-device copy failed");
+    return MOE_ERR_CUDA;
+  }
+  MOE_TRY(moe_layer_fwd(L, w, x_dev, out_dev, ctx, ctx_bytes, dev_status, stream));
+  MOE_TRY(moe_layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream));
+  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    set_error("moe_layer_step_host: device-to-host copy failed");
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}

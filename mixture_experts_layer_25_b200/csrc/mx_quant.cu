@@ -1,0 +1,218 @@
+// MX (MXFP8) quantiser: E4M3 codes with one E8M0 scale per 32 elements.
+//
+// Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ, section
+// "MXFP8による精度最適化": MXFP8 for the expert feed-forward compute.  Rule
+// (OCP MX): X = 2^(floor(log2 amax) - 8), code = RNE-saturating E4M3 of v/X,
+// an all-zero block gets scale byte 0.
+//
+// For a bf16 block, floor(log2 amax) is the exponent field of amax minus
+// 127, so the scale byte is max(expfield(amax) - 8, 0), and 1/X is the fp32
+// number with exponent field 254 - byte (exact power-of-two scaling).
+// Scales go to the tensor-core layout (see the library header).
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ size_t sf_offset(int mn, int kb, int kchunks) {
+  return ((size_t)(mn >> 7) * kchunks + (kb >> 2)) * 512 + (mn & 31) * 16 + ((mn >> 5) & 3) * 4 +
+         (kb & 3);
+}
+
+__device__ __forceinline__ uint32_t scale_byte(float amax) {
+  const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
+  return ef > 8 ? (uint32_t)(ef - 8) : 0u;
+}
+
+__device__ __forceinline__ float inv_scale(uint32_t byte) {
+  return __uint_as_float((254u - byte) << 23);
+}
+
+// 8 values -> 8 E4M3 codes (memory order)
+__device__ __forceinline__ uint2 encode8(const float* f, float inv) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+        make_float2(f[2 * i] * inv, f[2 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    w[i] = (uint32_t)c;
+  }
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// ------------------------------------------- blocks along rows (axis 0)
+// one warp per 256-column segment of one row; 4 lanes per 32-element block
+__global__ void mx_quant_rows_kernel(const uint4* __restrict__ in, int rows, int cols,
+                                     const int32_t* __restrict__ nrows_dev,
+                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int segs = (cols + 255) / 256;
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)rows * segs) return;
+  const int row = (int)(w / segs), seg = (int)(w % segs);
+  if (nrows_dev && row >= *nrows_dev) return;
+  const int col = seg * 256 + lane * 8;
+  const bool active = col < cols;
+  float f[8];
+  float amax = 0.f;
+  if (active) {
+    unpack8(in[((size_t)row * cols + col) / 8], f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  }
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  if (!active) return;
+  const uint32_t b = scale_byte(amax);
+  *reinterpret_cast<uint2*>(codes + (size_t)row * cols + col) = encode8(f, inv_scale(b));
+  if ((lane & 3) == 0) scales[sf_offset(row, col / 32, cols / 128)] = (uint8_t)b;
+}
+
+// ------------------------------------------ blocks down columns (axis 1)
+// one warp per (32-row block, 256-column segment); 8 columns per lane
+__global__ void mx_quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols,
+                                     const int32_t* __restrict__ nrows_dev,
+                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int segs = (cols + 255) / 256;
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= (long long)(rows / 32) * segs) return;
+  const int rb = (int)(w / segs), seg = (int)(w % segs);
+  const int r0 = rb * 32;
+  if (nrows_dev && r0 >= *nrows_dev) return;
+  const int col = seg * 256 + lane * 8;
+  if (col >= cols) return;
+  float amax[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int r = 0; r < 32; ++r) {
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(in + (size_t)(r0 + r) * cols + col), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax[i] = fmaxf(amax[i], fabsf(f[i]));
+  }
+  uint32_t b[8];
+  float inv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    b[i] = scale_byte(amax[i]);
+    inv[i] = inv_scale(b[i]);
+    scales[sf_offset(col + i, rb, rows / 128)] = (uint8_t)b[i];
+  }
+  for (int r = 0; r < 32; ++r) {
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(in + (size_t)(r0 + r) * cols + col), f);
+    uint32_t wv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+          make_float2(f[2 * i] * inv[2 * i], f[2 * i + 1] * inv[2 * i + 1]), __NV_SATFINITE,
+          __NV_E4M3);
+      wv[i] = (uint32_t)c;
+    }
+    *reinterpret_cast<uint2*>(codes + (size_t)(r0 + r) * cols + col) =
+        make_uint2(wv[0] | (wv[1] << 16), wv[2] | (wv[3] << 16));
+  }
+}
+
+// -------------------------------------------- permute fused with MX codes
+constexpr int kMaxK = 16;
+constexpr int kWarps = 8;
+
+__global__ void __launch_bounds__(32 * kWarps)
+permute_mx_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
+                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
+                  int k, int d, int tok_blocks, uint4* __restrict__ Xp, uint8_t* __restrict__ Xq,
+                  uint8_t* __restrict__ Xs) {
+  const int d8 = d / 8;
+  if ((int)blockIdx.x >= tok_blocks) {
+    // pad rows of one group: bf16 zeros, zero codes, scale byte 0
+    const int e = blockIdx.x - tok_blocks;
+    const int r0 = poff[e] + (offsets[e + 1] - offsets[e]);
+    const int r1 = poff[e + 1];
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (size_t i = threadIdx.x; i < (size_t)(r1 - r0) * d8; i += blockDim.x) {
+      Xp[(size_t)r0 * d8 + i] = z;
+      reinterpret_cast<uint2*>(Xq)[(size_t)r0 * d8 + i] = make_uint2(0, 0);
+    }
+    const int nkb = d / 32;
+    for (int i = threadIdx.x; i < (r1 - r0) * nkb; i += blockDim.x)
+      Xs[sf_offset(r0 + i / nkb, i % nkb, d / 128)] = 0;
+    return;
+  }
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int r[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) r[j] = j < k ? dst[(size_t)t * k + j] : -1;
+  for (int seg = 0; seg * 256 < d; ++seg) {
+    const int col = seg * 256 + lane * 8;
+    const bool active = col < d;
+    float f[8];
+    float amax = 0.f;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (active) {
+      v = ldg_stream(x + (size_t)t * d8 + col / 8);
+      unpack8(v, f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    if (!active) continue;
+    const uint32_t b = scale_byte(amax);
+    const uint2 c = encode8(f, inv_scale(b));
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      Xp[(size_t)r[j] * d8 + col / 8] = v;
+      *reinterpret_cast<uint2*>(Xq + (size_t)r[j] * d + col) = c;
+      if ((lane & 3) == 0) Xs[sf_offset(r[j], col / 32, d / 128)] = (uint8_t)b;
+    }
+  }
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+moe_status_t moe_permute_mx_launch(const void* x, const int32_t* dst, const int32_t* offsets,
+                                   const int32_t* poff, int T, int k, int d, int E, int A_pad_max,
+                                   void* Xp, uint8_t* Xq, uint8_t* Xs, cudaStream_t s) {
+  MOE_CHECK_ARG(d % 128 == 0 && A_pad_max % 128 == 0, "moe_permute: MX needs d %% 128 == 0");
+  MOE_CHECK_ARG(aligned16(Xq) && aligned16(Xs), "moe_permute: unaligned MX buffers");
+  const int tok_blocks = (T + kWarps - 1) / kWarps;
+  permute_mx_kernel<<<tok_blocks + E, 32 * kWarps, 0, s>>>(
+      static_cast<const uint4*>(x), dst, offsets, poff, T, k, d, tok_blocks,
+      static_cast<uint4*>(Xp), Xq, Xs);
+  MOE_CHECK_LAUNCH("permute_mx");
+  return MOE_OK;
+}
+
+extern "C" moe_status_t mx_quantize(const void* in, int rows, int cols, int axis,
+                                    const int32_t* poff, int E, const int32_t* nrows_dev,
+                                    uint8_t* codes, uint8_t* scales, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  (void)poff;
+  (void)E;
+  MOE_CHECK_ARG(rows > 0 && cols > 0 && rows % 128 == 0 && cols % 128 == 0,
+                "mx_quantize: rows and cols must be multiples of 128");
+  MOE_CHECK_ARG(axis == 0 || axis == 1, "mx_quantize: axis must be 0 or 1");
+  MOE_CHECK_ARG(in && codes && scales && aligned16(in) && aligned16(codes),
+                "mx_quantize: null or unaligned pointer");
+  const int segs = (cols + 255) / 256;
+  const int warps_per_block = 8;
+  if (axis == 0) {
+    const long long warps = (long long)rows * segs;
+    const long long blocks = (warps + warps_per_block - 1) / warps_per_block;
+    mx_quant_rows_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, s>>>(
+        static_cast<const uint4*>(in), rows, cols, nrows_dev, codes, scales);
+  } else {
+    const long long warps = (long long)(rows / 32) * segs;
+    const long long blocks = (warps + warps_per_block - 1) / warps_per_block;
+    mx_quant_cols_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(in), rows, cols, nrows_dev, codes, scales);
+  }
+  MOE_CHECK_LAUNCH("mx_quantize");
+  return MOE_OK;
+}

@@ -1,0 +1,355 @@
+// Rowwise dispatch into expert-contiguous buffers, the gate-weighted
+// combine, and their backward passes (HBM-bound gathers/scatters).
+//
+// Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ, section
+// "ルーティングと計算の最適化": routed tokens are written straight into the
+// experts' input buffers.  Every kernel moves whole token rows with 16-byte
+// vector accesses, one warp per token, each row read once.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kMaxK = 16;
+constexpr int kWarpsPerBlock = 8;
+
+// zero the pad rows [poff[e] + counts[e], poff[e+1]) of one expert group
+__device__ __forceinline__ void zero_pad_rows(const int32_t* offsets, const int32_t* poff, int e,
+                                              int d8, uint4* buf) {
+  const int r0 = poff[e] + (offsets[e + 1] - offsets[e]);
+  const int r1 = poff[e + 1];
+  const size_t n = (size_t)(r1 - r0) * d8;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  uint4* base = buf + (size_t)r0 * d8;
+  for (size_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = z;
+}
+
+// ------------------------------------------------------------------ permute
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+permute_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
+               const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
+               int k, int d8, int tok_blocks, uint4* __restrict__ Xp) {
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, Xp);
+    return;
+  }
+  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int r[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) r[j] = j < k ? dst[(size_t)t * k + j] : -1;
+  const uint4* xr = x + (size_t)t * d8;
+  for (int c0 = lane; c0 < d8; c0 += 32 * 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (c0 + 32 * u < d8) v[u] = ldg_stream(xr + c0 + 32 * u);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      uint4* o = Xp + (size_t)r[j] * d8;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + 32 * u < d8) o[c0 + 32 * u] = v[u];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ combine
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ gates,
+               const int32_t* __restrict__ dst, int T, int k, int d8, uint4* __restrict__ out) {
+  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int r[kMaxK];
+  float g[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    r[j] = j < k ? dst[(size_t)t * k + j] : -1;
+    g[j] = (j < k && gates) ? gates[(size_t)t * k + j] : 1.f;
+  }
+  for (int c = lane; c < d8; c += 32) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      float f[8];
+      unpack8(ldg_stream(Y + (size_t)r[j] * d8 + c), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+    }
+    out[(size_t)t * d8 + c] = pack8(acc);
+  }
+}
+
+// ------------------------------------------------------- combine backward
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
+                   const float* __restrict__ gates, const int32_t* __restrict__ dst,
+                   const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
+                   int k, int d8, int tok_blocks, uint4* __restrict__ dY, float* __restrict__ dg,
+                   float* __restrict__ dl, float* __restrict__ dl_rows) {
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY);
+    return;
+  }
+  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int r[kMaxK];
+  float g[kMaxK], dot[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    r[j] = j < k ? dst[(size_t)t * k + j] : -1;
+    g[j] = j < k ? gates[(size_t)t * k + j] : 0.f;
+    dot[j] = 0.f;
+  }
+  for (int c = lane; c < d8; c += 32) {
+    float fd[8];
+    unpack8(ldg_stream(dout + (size_t)t * d8 + c), fd);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      float fy[8], sc[8];
+      unpack8(ldg_stream(Y + (size_t)r[j] * d8 + c), fy);
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        s = fmaf(fd[i], fy[i], s);
+        sc[i] = g[j] * fd[i];
+      }
+      dot[j] += s;
+      dY[(size_t)r[j] * d8 + c] = pack8(sc);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j)
+    if (j < k) dot[j] = warp_sum(dot[j]);
+  if (lane == 0) {
+    float gs = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) gs = fmaf(g[j], dot[j], gs);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (j >= k) continue;
+      dg[(size_t)t * k + j] = dot[j];
+      if (dl) {
+        const float v = g[j] * (dot[j] - gs);
+        dl[(size_t)t * k + j] = v;
+        if (dl_rows && r[j] >= 0) dl_rows[r[j]] = v;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------- dispatch backward (dx)
+__global__ void transpose_f32_kernel(const float* __restrict__ in, int rows, int cols,
+                                     float* __restrict__ out) {
+  __shared__ float tile[32][33];
+  const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = by + i, c = bx + threadIdx.x;
+    if (r < rows && c < cols) tile[i][threadIdx.x] = in[(size_t)r * cols + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = bx + i, c = by + threadIdx.x;   // out is [cols, rows]
+    if (r < cols && c < rows) out[(size_t)r * rows + c] = tile[threadIdx.x][i];
+  }
+}
+
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+unpermute_sum_kernel(const uint4* __restrict__ dXp, const int32_t* __restrict__ dst,
+                     const int32_t* __restrict__ topk_idx, const float* __restrict__ dl,
+                     const float* __restrict__ WrT /* [E,d] or null */, int T, int k, int d8,
+                     int E, uint4* __restrict__ dx) {
+  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int r[kMaxK], e[kMaxK];
+  float w[kMaxK];
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    r[j] = j < k ? dst[(size_t)t * k + j] : -1;
+    e[j] = (j < k && WrT) ? topk_idx[(size_t)t * k + j] : -1;
+    w[j] = (j < k && WrT) ? dl[(size_t)t * k + j] : 0.f;
+  }
+  for (int c = lane; c < d8; c += 32) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      float f[8];
+      unpack8(ldg_stream(dXp + (size_t)r[j] * d8 + c), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += f[i];
+    }
+    if (WrT) {
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (r[j] < 0 || e[j] < 0 || e[j] >= E) continue;
+        const float4* wr = reinterpret_cast<const float4*>(WrT + (size_t)e[j] * d8 * 8) + 2 * c;
+        const float4 a = wr[0], b = wr[1];
+        acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
+        acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
+        acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
+        acc[6] = fmaf(w[j], b.z, acc[6]); acc[7] = fmaf(w[j], b.w, acc[7]);
+      }
+    }
+    dx[(size_t)t * d8 + c] = pack8(acc);
+  }
+}
+
+// --------------------------------------------------------- router wgrad
+// dWr[i, e] = sum over the real rows r of group e of x[src[r], i] * dl_rows[r]
+constexpr int kRwRowGroups = 8;
+__global__ void __launch_bounds__(256)
+router_wgrad_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ src,
+                    const float* __restrict__ dl_rows, const int32_t* __restrict__ offsets,
+                    const int32_t* __restrict__ poff, int d8, int E, float* __restrict__ dWr) {
+  __shared__ float red[kRwRowGroups][256 + 4];
+  const int e = blockIdx.x;
+  const int rg = threadIdx.x >> 5, cl = threadIdx.x & 31;
+  const int c = blockIdx.y * 32 + cl;       // 8-column chunk index
+  const int r0 = poff[e], n = offsets[e + 1] - offsets[e];
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (c < d8) {
+    for (int i = rg; i < n; i += kRwRowGroups) {
+      const int r = r0 + i;
+      const int t = src[r];
+      const float w = dl_rows[r];
+      float f[8];
+      unpack8(x[(size_t)t * d8 + c], f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = fmaf(f[q], w, acc[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) red[rg][cl * 8 + q] = acc[q];
+  __syncthreads();
+  const int col = blockIdx.y * 256 + threadIdx.x;
+  if (col < d8 * 8) {
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < kRwRowGroups; ++g) s += red[g][threadIdx.x];
+    dWr[(size_t)col * E + e] = s;
+  }
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" moe_status_t moe_permute(const void* x, const int32_t* dst, const int32_t* offsets,
+                                    const int32_t* poff, int T, int k, int d, int E,
+                                    int A_pad_max, void* Xp, uint8_t* Xq, uint8_t* Xs,
+                                    moe_stream_t stream);
+
+moe_status_t moe_permute_mx_launch(const void* x, const int32_t* dst, const int32_t* offsets,
+                                   const int32_t* poff, int T, int k, int d, int E, int A_pad_max,
+                                   void* Xp, uint8_t* Xq, uint8_t* Xs, cudaStream_t s);
+
+extern "C" moe_status_t moe_permute(const void* x, const int32_t* dst, const int32_t* offsets,
+                                    const int32_t* poff, int T, int k, int d, int E,
+                                    int A_pad_max, void* Xp, uint8_t* Xq, uint8_t* Xs,
+                                    moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && E > 0 && d > 0 && d % 8 == 0,
+                "moe_permute: bad T/k/E/d");
+  MOE_CHECK_ARG(x && dst && offsets && poff && Xp && aligned16(x) && aligned16(Xp),
+                "moe_permute: null or unaligned pointer");
+  MOE_CHECK_ARG((Xq == nullptr) == (Xs == nullptr), "moe_permute: Xq and Xs go together");
+  (void)A_pad_max;
+  if (Xq) return moe_permute_mx_launch(x, dst, offsets, poff, T, k, d, E, A_pad_max, Xp, Xq, Xs, s);
+  const int tok_blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  permute_kernel<<<tok_blocks + E, 32 * kWarpsPerBlock, 0, s>>>(
+      static_cast<const uint4*>(x), dst, offsets, poff, T, k, d / 8, tok_blocks,
+      static_cast<uint4*>(Xp));
+  MOE_CHECK_LAUNCH("permute");
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_unpermute_combine(const void* Y, const float* gates,
+                                              const int32_t* dst, int T, int k, int d, void* out,
+                                              moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && d > 0 && d % 8 == 0, "moe_unpermute_combine: bad sizes");
+  MOE_CHECK_ARG(Y && dst && out && aligned16(Y) && aligned16(out),
+                "moe_unpermute_combine: null or unaligned pointer");
+  const int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  combine_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(static_cast<const uint4*>(Y), gates, dst,
+                                                        T, k, d / 8, static_cast<uint4*>(out));
+  MOE_CHECK_LAUNCH("combine");
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_combine_bwd(const void* dout, const void* Y, const float* gates,
+                                        const int32_t* dst, const int32_t* offsets,
+                                        const int32_t* poff, int T, int k, int d, int E, void* dY,
+                                        float* dg, float* dl, float* dl_rows,
+                                        moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && E > 0 && d > 0 && d % 8 == 0,
+                "moe_combine_bwd: bad sizes");
+  MOE_CHECK_ARG(dout && Y && gates && dst && offsets && poff && dY && dg,
+                "moe_combine_bwd: null pointer");
+  MOE_CHECK_ARG(aligned16(dout) && aligned16(Y) && aligned16(dY), "moe_combine_bwd: unaligned");
+  const int tok_blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  combine_bwd_kernel<<<tok_blocks + E, 32 * kWarpsPerBlock, 0, s>>>(
+      static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff, T,
+      k, d / 8, tok_blocks, static_cast<uint4*>(dY), dg, dl, dl_rows);
+  MOE_CHECK_LAUNCH("combine_bwd");
+  return MOE_OK;
+}
+
+extern "C" size_t moe_unpermute_sum_workspace_size(int d, int E) {
+  if (d <= 0 || E <= 0) return 0;
+  return round_up((size_t)d * E * sizeof(float), 256);
+}
+
+extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
+                                          const int32_t* topk_idx, const float* dl,
+                                          const float* Wr, int T, int k, int d, int E, void* dx,
+                                          void* ws, size_t ws_bytes, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && d > 0 && d % 8 == 0 && E > 0,
+                "moe_unpermute_sum: bad sizes");
+  MOE_CHECK_ARG(dXp && dst && dx && aligned16(dXp) && aligned16(dx),
+                "moe_unpermute_sum: null or unaligned pointer");
+  float* WrT = nullptr;
+  if (Wr) {
+    MOE_CHECK_ARG(topk_idx && dl, "moe_unpermute_sum: router term needs topk_idx and dl");
+    const size_t need = moe_unpermute_sum_workspace_size(d, E);
+    if (!ws || ws_bytes < need) {
+      set_error("moe_unpermute_sum: workspace %zu < %zu bytes", ws_bytes, need);
+      return MOE_ERR_WORKSPACE;
+    }
+    MOE_CHECK_ARG(aligned16(ws), "moe_unpermute_sum: unaligned workspace");
+    WrT = static_cast<float*>(ws);
+    dim3 grid((E + 31) / 32, (d + 31) / 32), block(32, 8);
+    transpose_f32_kernel<<<grid, block, 0, s>>>(Wr, d, E, WrT);
+    MOE_CHECK_LAUNCH("transpose Wr");
+  }
+  const int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  unpermute_sum_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(
+      static_cast<const uint4*>(dXp), dst, topk_idx, dl, WrT, T, k, d / 8, E,
+      static_cast<uint4*>(dx));
+  MOE_CHECK_LAUNCH("unpermute_sum");
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const float* dl_rows,
+                                         const int32_t* offsets, const int32_t* poff, int T,
+                                         int d, int E, float* dWr, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && d > 0 && d % 8 == 0 && E > 0, "moe_router_wgrad: bad sizes");
+  MOE_CHECK_ARG(x && src && dl_rows && offsets && poff && dWr && aligned16(x),
+                "moe_router_wgrad: null or unaligned pointer");
+  dim3 grid(E, (d + 255) / 256);
+  router_wgrad_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), src, dl_rows, offsets,
+                                           poff, d / 8, E, dWr);
+  MOE_CHECK_LAUNCH("router_wgrad");
+  return MOE_OK;
+}

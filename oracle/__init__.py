@@ -29,7 +29,8 @@ brute-force nearest-code search.
 from .moe_oracle import (  # noqa: F401
     router_logits, topk_select, gates_from_logits, routing_metadata,
     permute_rows, expert_forward, combine, layer_forward, layer_backward,
-    silu, round_bf16,
+    silu, round_bf16, grouped_matmul, grouped_matmul_t, grouped_wgrad, swiglu_backward,
+    combine_backward, gate_logit_grad, unpermute_sum, router_backward,
 )
 from .mx import (  # noqa: F401
     e4m3_decode_table, e4m3_encode, mx_scale_exponent, mx_quantize_rows,

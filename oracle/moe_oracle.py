@@ -215,6 +215,85 @@ def layer_forward(x, W1, W3, W2, k, Wr=None, bias=None, topk_idx=None,
                 h=h, Y=Y, out=out, router=router, mx=mx, k=k)
 
 
+def grouped_matmul(A, B, poff):
+    """C[r] = A[r] @ B[e] for every row r of group e (rows poff[e]..poff[e+1])."""
+    A = np.asarray(A, np.float64)
+    C = np.zeros((A.shape[0], B.shape[2]))
+    for e in range(B.shape[0]):
+        a, b = int(poff[e]), int(poff[e + 1])
+        if a < b:
+            C[a:b] = A[a:b] @ np.asarray(B[e], np.float64)
+    return C
+
+
+def grouped_matmul_t(dC, B, poff):
+    """dA[r] = dC[r] @ B[e]^T for every row r of group e."""
+    dC = np.asarray(dC, np.float64)
+    dA = np.zeros((dC.shape[0], B.shape[1]))
+    for e in range(B.shape[0]):
+        a, b = int(poff[e]), int(poff[e + 1])
+        if a < b:
+            dA[a:b] = dC[a:b] @ np.asarray(B[e], np.float64).T
+    return dA
+
+
+def grouped_wgrad(A, dC, poff, E):
+    """dB[e] = A_e^T @ dC_e, summed over the rows of group e (zero if empty)."""
+    A = np.asarray(A, np.float64); dC = np.asarray(dC, np.float64)
+    dB = np.zeros((E, A.shape[1], dC.shape[1]))
+    for e in range(E):
+        a, b = int(poff[e]), int(poff[e + 1])
+        if a < b:
+            dB[e] = A[a:b].T @ dC[a:b]
+    return dB
+
+
+def swiglu_backward(dh, H1, H3):
+    """h = silu(H1) * H3:  dH1 = dh * H3 * s * (1 + H1 (1 - s)),
+    dH3 = dh * H1 * s, with s = sigmoid(H1)."""
+    s = _sigmoid(H1)
+    return dh * H3 * s * (1.0 + H1 * (1.0 - s)), dh * H1 * s
+
+
+def combine_backward(dout, Y, gates, dst):
+    """Backward of out[t] = sum_j g[t,j] Y[dst[t,j]]:
+    dY[dst[t,j]] = g[t,j] dout[t] (other rows zero), dg[t,j] = <dout[t], Y[dst[t,j]]>."""
+    dout = np.asarray(dout, np.float64)
+    T, k = dst.shape
+    dY = np.zeros((Y.shape[0], dout.shape[1]))
+    dg = np.zeros((T, k))
+    for j in range(k):
+        dY[dst[:, j]] = gates[:, j:j + 1] * dout
+        dg[:, j] = np.sum(dout * Y[dst[:, j]], axis=1)
+    return dY, dg
+
+
+def gate_logit_grad(gates, dg):
+    """Gates are a softmax over the chosen logits, so the chosen logits get
+    dl_j = g_j (dg_j - sum_i g_i dg_i)."""
+    return gates * (dg - np.sum(gates * dg, axis=1, keepdims=True))
+
+
+def unpermute_sum(dXp, dst):
+    """dx[t] = sum_j dXp[dst[t,j]]."""
+    T, k = dst.shape
+    dx = np.zeros((T, dXp.shape[1]))
+    for j in range(k):
+        dx += dXp[dst[:, j]]
+    return dx
+
+
+def router_backward(x, Wr, idx, dl):
+    """Logits L = x Wr (+ b): with dL[t, idx[t,j]] = dl[t,j] and zero
+    elsewhere, dWr = x^T dL and the input gradient dL Wr^T."""
+    T, k = idx.shape
+    E = Wr.shape[1]
+    dL = np.zeros((T, E))
+    for j in range(k):
+        dL[np.arange(T), idx[:, j].astype(np.int64)] += dl[:, j]
+    return np.asarray(x, np.float64).T @ dL, dL @ np.asarray(Wr, np.float64).T
+
+
 def layer_backward(ctx, dout):
     """Gradients of <dout, out> with respect to x, W1, W3, W2 and (router
     mode) Wr, plus the gate gradient dg.  The top-k choice is piecewise
@@ -222,19 +301,13 @@ def layer_backward(ctx, dout):
     constant."""
     dout = np.asarray(dout, np.float64)
     mx = ctx["mx"]
-    meta = ctx["meta"]; dst = meta["dst"]; src = meta["src"]; poff = meta["poff"]
+    meta = ctx["meta"]; dst = meta["dst"]; poff = meta["poff"]
     g = ctx["gates"]; Y = ctx["Y"]; Xp = ctx["Xp"]
     H1, H3, h = ctx["H1"], ctx["H3"], ctx["h"]
     W1, W3, W2 = ctx["W1"], ctx["W3"], ctx["W2"]
-    T, k = dst.shape
-    E, d, F = W1.shape
+    E = W1.shape[0]
 
-    # gate-weighted combine, backward: dY rows and the gate gradient
-    dY = np.zeros_like(Y)
-    dg = np.zeros((T, k))
-    for j in range(k):
-        dY[dst[:, j]] = g[:, j:j + 1] * dout
-        dg[:, j] = np.sum(dout * Y[dst[:, j]], axis=1)
+    dY, dg = combine_backward(dout, Y, g, dst)
     if mx:
         dY = round_bf16(dY)
 
@@ -249,10 +322,7 @@ def layer_backward(ctx, dout):
         # GEMM2 dgrad (K = d) and wgrad (K = rows of the group)
         dh = _gemm(dYe, W2[e].T, mx, "rows", "cols")
         dW2[e] = _gemm(he.T, dYe, mx, "rows", "cols")
-        # SwiGLU backward
-        s = _sigmoid(H1[a:b])
-        dA1 = dh * H3[a:b] * s * (1.0 + H1[a:b] * (1.0 - s))
-        dA3 = dh * H1[a:b] * s
+        dA1, dA3 = swiglu_backward(dh, H1[a:b], H3[a:b])
         if mx:
             dA1 = round_bf16(dA1); dA3 = round_bf16(dA3)
         # GEMM1 dgrad (K = 2F) and wgrad (K = rows of the group)
@@ -262,20 +332,12 @@ def layer_backward(ctx, dout):
         dW1[e] = _gemm(Xe.T, dA1, mx, "rows", "cols")
         dW3[e] = _gemm(Xe.T, dA3, mx, "rows", "cols")
 
-    # unpermute: every token sums the k rows it was copied to
-    dx = np.zeros((T, d))
-    for j in range(k):
-        dx += dXp[dst[:, j]]
-
+    dx = unpermute_sum(dXp, dst)
     out = dict(dx=dx, dW1=dW1, dW3=dW3, dW2=dW2, dg=dg, dY=dY, dXp=dXp)
     if ctx["router"]:
-        # softmax over the chosen logits: dL_j = g_j (dg_j - sum_i g_i dg_i)
-        dl = g * (dg - np.sum(g * dg, axis=1, keepdims=True))
-        dL = np.zeros((T, E))
-        idx = ctx["topk_idx"].astype(np.int64)
-        for j in range(k):
-            dL[np.arange(T), idx[:, j]] += dl[:, j]
-        out["dWr"] = ctx["x"].T @ dL
-        out["dx"] = dx + dL @ ctx["Wr"].T
+        dl = gate_logit_grad(g, dg)
+        dWr, dx_r = router_backward(ctx["x"], ctx["Wr"], ctx["topk_idx"], dl)
+        out["dWr"] = dWr
+        out["dx"] = dx + dx_r
         out["dl"] = dl
     return out

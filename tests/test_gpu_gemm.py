@@ -1,0 +1,200 @@
+"""GPU parity of the tcgen05 grouped GEMMs (fwd / dgrad / wgrad, BF16 and
+MXFP8) against the oracle's grouped products, on ragged groups with empty
+experts, several tiles and a partial last tile per group."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from gpu_util import f64, rel_err
+
+pytestmark = pytest.mark.gpu
+moe = pytest.importorskip("mixture_experts_layer_25_b200")
+
+
+def _groups(counts, extra_rows=256):
+    counts = np.asarray(counts)
+    padded = -(-counts // 128) * 128
+    poff = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    A = int(poff[-1]) + extra_rows
+    real = np.zeros(A, bool)
+    for e, c in enumerate(counts):
+        real[poff[e]:poff[e] + c] = True
+    return poff, A, real
+
+
+def _act(A, cols, real, seed, scale=1.0):
+    t = moe_inputs.random_bf16((A, cols), seed, std=scale, device="cuda")
+    t[torch.from_numpy(~real).cuda()] = 0     # pad rows are zero, as the library keeps them
+    return t
+
+
+def _w(E, r, c, seed):
+    return moe_inputs.random_bf16((E, r, c), seed, std=0.05, device="cuda")
+
+
+COUNTS = [0, 5, 300, 128, 1, 0, 513]
+
+
+@pytest.mark.parametrize("mx", [False, True])
+def test_fwd_plain(mx):
+    E, K, N = len(COUNTS), 512, 512
+    poff, A, real = _groups(COUNTS)
+    X = _act(A, K, real, 1)
+    B = _w(E, K, N, 2)
+    P = int(poff[-1])
+    tp = torch.from_numpy(poff).cuda()
+    if not mx:
+        C = moe.moe_grouped_gemm_fwd(X, B, tp, E)
+        ref = oracle.grouped_matmul(f64(X), f64(B), poff)
+    else:
+        Xq, Xs = moe.mx_quantize(X, 0)
+        Bq, Bs = moe.mx_quantize(B.view(E * K, N), 1)
+        C = moe.moe_grouped_gemm_fwd(Xq, Bq.view(E, K, N), tp, E, A_sc=Xs, B_sc=Bs)
+        Xd = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(f64(X)))
+        Bd = oracle.mx_dequantize_cols(*oracle.mx_quantize_cols_grouped(f64(B).reshape(E * K, N), [0, E * K]))
+        ref = oracle.grouped_matmul(Xd, Bd.reshape(E, K, N), poff)
+    torch.cuda.synchronize()
+    err = rel_err(f64(C[:P]), ref[:P])
+    assert err < (1e-2 if not mx else 3e-2), err
+
+
+@pytest.mark.parametrize("mx", [False, True])
+def test_fwd_swiglu(mx):
+    E, K, F = len(COUNTS), 256, 384
+    poff, A, real = _groups(COUNTS)
+    X = _act(A, K, real, 3)
+    W1, W3 = _w(E, K, F, 4), _w(E, K, F, 5)
+    P = int(poff[-1])
+    tp = torch.from_numpy(poff).cuda()
+    if not mx:
+        h, aux = moe.moe_grouped_gemm_fwd(X, W1, tp, E, epilogue=moe.MOE_EPI_SWIGLU, B3=W3)
+        Xd, W1d, W3d = f64(X), f64(W1), f64(W3)
+    else:
+        Xq, Xs = moe.mx_quantize(X, 0)
+        W1q, W1s = moe.mx_quantize(W1.view(E * K, F), 1)
+        W3q, W3s = moe.mx_quantize(W3.view(E * K, F), 1)
+        h, aux = moe.moe_grouped_gemm_fwd(Xq, W1q.view(E, K, F), tp, E, epilogue=moe.MOE_EPI_SWIGLU,
+                                          B3=W3q.view(E, K, F), A_sc=Xs, B_sc=W1s, B3_sc=W3s)
+        Xd = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(f64(X)))
+        q = lambda W: oracle.mx_dequantize_cols(*oracle.mx_quantize_cols_grouped(
+            f64(W).reshape(E * K, F), [0, E * K])).reshape(E, K, F)
+        W1d, W3d = q(W1), q(W3)
+    torch.cuda.synchronize()
+    H1 = oracle.grouped_matmul(Xd, W1d, poff)
+    H3 = oracle.grouped_matmul(Xd, W3d, poff)
+    tol = 1e-2 if not mx else 3e-2
+    assert rel_err(f64(aux[:P, :F]), H1[:P]) < tol
+    assert rel_err(f64(aux[:P, F:]), H3[:P]) < tol
+    assert rel_err(f64(h[:P]), (oracle.silu(H1) * H3)[:P]) < tol
+
+
+@pytest.mark.parametrize("mx", [False, True])
+@pytest.mark.parametrize("dual", [False, True])
+def test_dgrad(mx, dual):
+    E, K, N = len(COUNTS), 512, 256
+    poff, A, real = _groups(COUNTS)
+    dC = _act(A, 2 * N if dual else N, real, 6)
+    B, B3 = _w(E, K, N, 7), (_w(E, K, N, 8) if dual else None)
+    P = int(poff[-1])
+    tp = torch.from_numpy(poff).cuda()
+    if not mx:
+        dA = moe.moe_grouped_gemm_dgrad(dC, B, tp, E, B3=B3)
+        dCd, Bd = f64(dC), f64(B)
+        B3d = f64(B3) if dual else None
+    else:
+        dCq, dCs = moe.mx_quantize(dC, 0)
+        Bq, Bs = moe.mx_quantize(B.view(E * K, N), 0)
+        B3q, B3s = (moe.mx_quantize(B3.view(E * K, N), 0) if dual else (None, None))
+        dA = moe.moe_grouped_gemm_dgrad(dCq, Bq.view(E, K, N), tp, E,
+                                        B3=None if B3q is None else B3q.view(E, K, N),
+                                        dC_sc=dCs, B_sc=Bs, B3_sc=B3s)
+        dCd = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(f64(dC)))
+        q = lambda W: oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(
+            f64(W).reshape(E * K, N))).reshape(E, K, N)
+        Bd = q(B)
+        B3d = q(B3) if dual else None
+    torch.cuda.synchronize()
+    ref = oracle.grouped_matmul_t(dCd[:, :N], Bd, poff)
+    if dual:
+        ref += oracle.grouped_matmul_t(dCd[:, N:], B3d, poff)
+    assert rel_err(f64(dA[:P]), ref[:P]) < (1e-2 if not mx else 3e-2)
+
+
+@pytest.mark.parametrize("mx", [False, True])
+def test_dgrad_swiglu_bwd(mx):
+    E, F, d = len(COUNTS), 256, 512
+    poff, A, real = _groups(COUNTS)
+    dY = _act(A, d, real, 9)
+    W2 = _w(E, F, d, 10)
+    H13 = _act(A, 2 * F, real, 11, scale=2.0)
+    P = int(poff[-1])
+    tp = torch.from_numpy(poff).cuda()
+    if not mx:
+        dA = moe.moe_grouped_gemm_dgrad(dY, W2, tp, E, epilogue=moe.MOE_EPI_SWIGLU_BWD, aux=H13)
+        dYd, W2d = f64(dY), f64(W2)
+    else:
+        dYq, dYs = moe.mx_quantize(dY, 0)
+        Wq, Ws = moe.mx_quantize(W2.view(E * F, d), 0)
+        dA = moe.moe_grouped_gemm_dgrad(dYq, Wq.view(E, F, d), tp, E,
+                                        epilogue=moe.MOE_EPI_SWIGLU_BWD, aux=H13, dC_sc=dYs, B_sc=Ws)
+        dYd = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(f64(dY)))
+        W2d = oracle.mx_dequantize_rows(*oracle.mx_quantize_rows(f64(W2).reshape(E * F, d))).reshape(E, F, d)
+    torch.cuda.synchronize()
+    dh = oracle.grouped_matmul_t(dYd, W2d, poff)
+    H = f64(H13)
+    d1, d3 = oracle.swiglu_backward(dh, H[:, :F], H[:, F:])
+    tol = 1e-2 if not mx else 3e-2
+    assert rel_err(f64(dA[:P, :F]), d1[:P]) < tol
+    assert rel_err(f64(dA[:P, F:]), d3[:P]) < tol
+
+
+@pytest.mark.parametrize("mx", [False, True])
+@pytest.mark.parametrize("split", [False, True])
+def test_wgrad(mx, split):
+    E, K, N = len(COUNTS), 256, 256
+    poff, A, real = _groups(COUNTS)
+    X = _act(A, K, real, 12)
+    dC = _act(A, 2 * N if split else N, real, 13)
+    tp = torch.from_numpy(poff).cuda()
+    if not mx:
+        r = moe.moe_grouped_gemm_wgrad(X, dC, tp, E, split=split)
+        Xd, dCd = f64(X), f64(dC)
+    else:
+        Xq, Xs = moe.mx_quantize(X, 1)
+        dCq, dCs = moe.mx_quantize(dC, 1)
+        r = moe.moe_grouped_gemm_wgrad(Xq, dCq, tp, E, split=split, A_sc=Xs, dC_sc=dCs)
+        Xd = oracle.mx_dequantize_cols(*oracle.mx_quantize_cols_grouped(f64(X), [0, A]))
+        dCd = oracle.mx_dequantize_cols(*oracle.mx_quantize_cols_grouped(f64(dC), [0, A]))
+    torch.cuda.synchronize()
+    ref = oracle.grouped_wgrad(Xd, dCd, poff, E)
+    tol = 1e-2 if not mx else 3e-2
+    if split:
+        dB, dB3 = r
+        assert rel_err(f64(dB), ref[:, :, :N]) < tol
+        assert rel_err(f64(dB3), ref[:, :, N:]) < tol
+    else:
+        assert rel_err(f64(r), ref) < tol
+    got = f64(r[0] if split else r)
+    assert np.all(got[0] == 0) and np.all(got[5] == 0)      # empty experts
+
+
+def test_fwd_full_width_sampled_experts():
+    """The 128-expert layer's GEMM1 shape (K = 2048, N = 2F = 2048) with
+    ~512 rows per expert; checked on a sample of experts."""
+    E, K, F = 128, 2048, 1024
+    rng = np.random.default_rng(0)
+    counts = rng.multinomial(65536, np.ones(E) / E)
+    poff, A, real = _groups(counts, extra_rows=0)
+    X = _act(A, K, real, 14)
+    W1, W3 = _w(E, K, F, 15), _w(E, K, F, 16)
+    tp = torch.from_numpy(poff).cuda()
+    h, aux = moe.moe_grouped_gemm_fwd(X, W1, tp, E, epilogue=moe.MOE_EPI_SWIGLU, B3=W3)
+    torch.cuda.synchronize()
+    for e in (0, 37, 127):
+        a, b = int(poff[e]), int(poff[e]) + int(counts[e])
+        Xe = f64(X[a:b])
+        H1 = Xe @ f64(W1[e]); H3 = Xe @ f64(W3[e])
+        assert rel_err(f64(h[a:b]), oracle.silu(H1) * H3) < 1e-2
+        assert rel_err(f64(aux[a:b, :F]), H1) < 1e-2

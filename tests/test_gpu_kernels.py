@@ -1,0 +1,212 @@
+"""GPU parity of the routing, dispatch, combine, backward and MX kernels
+against the CPU oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from gpu_util import f64, np_i, rel_err, scales_to_plain
+
+pytestmark = pytest.mark.gpu
+
+moe = pytest.importorskip("mixture_experts_layer_25_b200")
+U = 2.0 ** -24
+
+
+def _router_inputs(T, d, E, seed, bias=False):
+    x = moe_inputs.random_bf16((T, d), seed, device="cuda")
+    g = torch.Generator(device="cuda"); g.manual_seed(seed + 1)
+    Wr = (torch.randn((d, E), generator=g, device="cuda") * 0.02).contiguous()
+    b = None
+    if bias:
+        rng = np.random.default_rng(seed + 2)
+        rank = rng.permutation(E) + 1
+        b = torch.tensor(3.0 * np.log(rank.astype(np.float64) ** -1.2), dtype=torch.float32).cuda()
+    return x, Wr, b
+
+
+def _check_metadata(meta, idx, E):
+    """GPU metadata bit-exact against the oracle's counting sort of idx."""
+    ref = oracle.routing_metadata(idx, E, 128)
+    assert np_i(meta["counts"]).tolist() == ref["counts"].tolist()
+    assert np_i(meta["offsets"]).tolist() == ref["offsets"].tolist()
+    assert np_i(meta["poff"]).tolist() == ref["poff"].tolist()
+    np.testing.assert_array_equal(np_i(meta["dst"]), ref["dst"])
+    src = np_i(meta["src"])
+    P = int(ref["poff"][E])
+    np.testing.assert_array_equal(src[:P], ref["src"])
+    assert np.all(src[P:] == -1)
+    return ref
+
+
+@pytest.mark.parametrize("T,d,E,k,bias", [
+    (1024, 256, 8, 2, False),     # the tiny layer
+    (37, 64, 5, 3, False),        # ragged: one partial routing block
+    (1000, 128, 16, 4, True),
+    (4096, 2048, 128, 4, True),   # skewed load, many empty experts
+    (16384, 2048, 128, 4, False), # the 128-expert layer at full size
+])
+def test_route_router_mode(T, d, E, k, bias):
+    x, Wr, b = _router_inputs(T, d, E, 11 + T, bias)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    meta = moe.moe_route(x, Wr, b, k, E, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    Lg = f64(meta["logits"])
+    idx_g = np_i(meta["topk_idx"])
+    # (i) strict: the oracle's selection and metadata on the device's logits
+    idx_o = oracle.topk_select(Lg, k)
+    np.testing.assert_array_equal(idx_g, idx_o)
+    assert rel_err(f64(meta["gates"]), oracle.gates_from_logits(Lg, idx_o)) < 1e-5
+    _check_metadata(meta, idx_o, E)
+    # (ii) end to end: fp32 logits within the fp32 dot-product bound of the
+    # fp64 logits; only near-tie tokens may choose differently
+    x64, W64 = f64(x), f64(Wr)
+    b64 = None if b is None else f64(b)
+    L64 = oracle.router_logits(x64, W64, b64)
+    bound = 4 * d * U * (np.abs(x64) @ np.abs(W64)) + 4 * U * np.abs(L64)
+    assert np.all(np.abs(Lg - L64) <= bound)
+    srt = -np.sort(-L64, axis=1)
+    near = (srt[:, k - 1] - srt[:, k]) < 2 * bound.max(axis=1) if k < E else np.zeros(T, bool)
+    differ = np.any(oracle.topk_select(L64, k) != idx_g, axis=1)
+    assert not np.any(differ & ~near)
+    if bias:
+        assert np.sum(np_i(meta["counts"]) == 0) >= 1
+
+
+@pytest.mark.parametrize("T,E,k", [(8192, 384, 8), (100, 7, 7), (1, 4, 2), (3000, 64, 1)])
+def test_route_given_mode(T, E, k):
+    idx, gates = moe_inputs.random_routing(T, E, k, 5 + T)
+    ti = torch.from_numpy(idx).cuda()
+    tg = torch.from_numpy(gates).cuda()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    meta = moe.moe_route(None, None, None, k, E, topk_idx=ti, gates=tg, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    _check_metadata(meta, idx, E)
+
+
+def test_route_given_mode_rejects_bad_experts():
+    idx, gates = moe_inputs.random_routing(64, 8, 3, 1)
+    idx[5, 1] = 8          # out of range
+    idx[9, 2] = idx[9, 0]  # repeated inside a token
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    meta = moe.moe_route(None, None, None, 3, 8, topk_idx=torch.from_numpy(idx).cuda(),
+                         gates=torch.from_numpy(gates).cuda(), status=st)
+    torch.cuda.synchronize()
+    assert st.item() == (moe.MOE_DEV_BAD_EXPERT | moe.MOE_DEV_DUP_EXPERT)
+    dst = np_i(meta["dst"])
+    assert dst[5, 1] == -1 and dst[9, 2] == -1
+    counts = np_i(meta["counts"])
+    assert counts.sum() == 64 * 3 - 2
+    src = np_i(meta["src"])
+    valid = dst[dst >= 0]
+    assert len(set(valid.tolist())) == len(valid) and np.all(src[valid] >= 0)
+
+
+def _meta_for(T, E, k, seed):
+    idx, gates = moe_inputs.random_routing(T, E, k, seed)
+    meta = moe.moe_route(None, None, None, k, E, topk_idx=torch.from_numpy(idx).cuda(),
+                         gates=torch.from_numpy(gates).cuda())
+    return idx, gates, meta
+
+
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (333, 2048, 64, 4), (50, 6144, 384, 8)])
+def test_permute_bit_exact_and_pad_rows_zero(T, d, E, k):
+    idx, gates, meta = _meta_for(T, E, k, 3)
+    x = moe_inputs.random_bf16((T, d), 7, device="cuda")
+    Xp = moe.moe_permute(x, meta, k, E)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    P = int(ref["poff"][E])
+    np.testing.assert_array_equal(f64(Xp[:P]), oracle.permute_rows(f64(x), ref))
+
+
+def test_permute_fused_mx_codes():
+    T, d, E, k = 700, 512, 16, 4
+    idx, gates, meta = _meta_for(T, E, k, 4)
+    x = moe_inputs.random_bf16((T, d), 8, device="cuda")
+    x[3, :64] = 0          # an all-zero block
+    x[4, :32] *= 1e-30     # tiny values
+    Xp, Xq, Xs = moe.moe_permute(x, meta, k, E, mx=True)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    P = int(ref["poff"][E])
+    Xp64 = oracle.permute_rows(f64(x), ref)
+    c, s = oracle.mx_quantize_rows(Xp64)
+    np.testing.assert_array_equal(Xq[:P].cpu().numpy(), c)
+    A = meta["A_pad_max"]
+    np.testing.assert_array_equal(scales_to_plain(Xs, A, d, 0)[:P], s)
+
+
+@pytest.mark.parametrize("R,C,axis", [(256, 512, 0), (512, 384, 1), (128, 128, 0), (384, 2048, 1)])
+def test_mx_quantize_bit_exact(R, C, axis):
+    g = torch.Generator(device="cuda"); g.manual_seed(R + C + axis)
+    v = torch.randn((R, C), generator=g, device="cuda") * torch.exp(
+        torch.randn((R, 1), generator=g, device="cuda") * 3)
+    v = v.to(torch.bfloat16)
+    v[0, :32] = 0
+    v[1, 5] = -0.0
+    v[2, :] = -v[2, :].abs() * 1e-6
+    v[5, 7] = 300.0
+    v[6, 0] = 400.0        # a negative value that rounds to zero keeps its sign
+    v[6, 1] = -1e-5
+    codes, scales = moe.mx_quantize(v, axis)
+    torch.cuda.synchronize()
+    v64 = f64(v)
+    if axis == 0:
+        c, s = oracle.mx_quantize_rows(v64)
+    else:
+        c, s = oracle.mx_quantize_cols_grouped(v64, np.array([0, R]))
+    np.testing.assert_array_equal(codes.cpu().numpy(), c)
+    np.testing.assert_array_equal(scales_to_plain(scales, R, C, axis), s)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (257, 2048, 32, 4), (64, 6144, 384, 8)])
+def test_combine_and_its_backward(T, d, E, k):
+    idx, gates, meta = _meta_for(T, E, k, 5)
+    A = meta["A_pad_max"]
+    Y = moe_inputs.random_bf16((A, d), 9, device="cuda")
+    dout = moe_inputs.random_bf16((T, d), 10, device="cuda")
+    tg = torch.from_numpy(gates).cuda()
+    out = moe.moe_unpermute_combine(Y, tg, meta["dst"])
+    dY, dg, dl, dl_rows = moe.moe_combine_bwd(dout, Y, tg, meta, E)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    dst = ref["dst"]
+    Y64, g64 = f64(Y), gates.astype(np.float64)
+    assert rel_err(f64(out), oracle.combine(Y64, g64, dst)) < 1e-2
+    dY_o, dg_o = oracle.combine_backward(f64(dout), Y64, g64, dst)
+    P = int(ref["poff"][E])
+    assert rel_err(f64(dY[:P]), dY_o[:P]) < 1e-2
+    pad = ref["src"] < 0
+    assert np.all(f64(dY[:P])[pad] == 0)
+    assert rel_err(dg.cpu().numpy(), dg_o) < 1e-4
+    dl_o = oracle.gate_logit_grad(g64, dg_o)
+    assert rel_err(dl.cpu().numpy(), dl_o) < 1e-4
+    np.testing.assert_allclose(dl_rows.cpu().numpy()[dst], dl.cpu().numpy(), rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (300, 2048, 128, 4)])
+def test_unpermute_sum_and_router_grads(T, d, E, k):
+    idx, gates, meta = _meta_for(T, E, k, 6)
+    A = meta["A_pad_max"]
+    dXp = moe_inputs.random_bf16((A, d), 12, device="cuda")
+    x = moe_inputs.random_bf16((T, d), 13, device="cuda")
+    g = torch.Generator(device="cuda"); g.manual_seed(14)
+    Wr = torch.randn((d, E), generator=g, device="cuda") * 0.02
+    dl = torch.randn((T, k), generator=g, device="cuda")
+    dl_rows = torch.zeros(A, dtype=torch.float32, device="cuda")
+    dst_t = meta["dst"].long()
+    dl_rows[dst_t.reshape(-1)] = dl.reshape(-1)
+    dx_plain = moe.moe_unpermute_sum(dXp, meta["dst"])
+    dx = moe.moe_unpermute_sum(dXp, meta["dst"], topk_idx=meta["topk_idx"], dl=dl, Wr=Wr, E=E)
+    dWr = moe.moe_router_wgrad(x, meta, dl_rows, E)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    dxs = oracle.unpermute_sum(f64(dXp), ref["dst"])
+    assert rel_err(f64(dx_plain), dxs) < 1e-2
+    dWr_o, dxr = oracle.router_backward(f64(x), f64(Wr), idx, dl.cpu().numpy().astype(np.float64))
+    assert rel_err(f64(dx), dxs + dxr) < 1e-2
+    assert rel_err(dWr.cpu().numpy(), dWr_o) < 1e-4

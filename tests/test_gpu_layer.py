@@ -1,0 +1,153 @@
+"""GPU parity of the whole layer (moe_layer_fwd + moe_layer_bwd through the C
+ABI) against the oracle: the tiny layer element by element; the full-size
+layers on sampled tokens and experts.
+
+Routing reading: the device computes logits in fp32.  The strict check runs
+the oracle's routing on the device's logits (bit-exact metadata); the
+full-size checks use the oracle's own fp64 routing and skip the rare
+near-tie tokens, whose choice may legitimately differ."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from gpu_util import f64, np_i, rel_err
+
+pytestmark = pytest.mark.gpu
+moe = pytest.importorskip("mixture_experts_layer_25_b200")
+
+
+def _layer(cfg, inp):
+    return moe.MoELayer(T=cfg.T, d=cfg.d, E=cfg.E, k=cfg.k, F=cfg.F, W1=inp["W1"], W3=inp["W3"],
+                        W2=inp["W2"], Wr=inp["Wr"] if cfg.routing == "router" else None,
+                        bias=inp["bias"], topk_idx=inp.get("topk_idx"), gates=inp.get("gates"),
+                        mx=cfg.mx)
+
+
+def _run(cfg, inp):
+    L = _layer(cfg, inp)
+    out = L.forward(inp["x"])
+    dx = L.backward(inp["x"], inp["dout"])
+    torch.cuda.synchronize()
+    assert L.status.item() == 0
+    return L, out, dx
+
+
+@pytest.mark.parametrize("variant", ["bf16", "mx", "given", "skewed"])
+def test_tiny_layer_element_by_element(variant):
+    cfg = moe_inputs.CONFIGS["tiny"]
+    if variant == "mx":
+        cfg = cfg.with_(mx=True)
+    if variant == "given":
+        cfg = cfg.with_(routing="random")
+    if variant == "skewed":
+        cfg = cfg.with_(bias="zipf", E=8)
+    inp = moe_inputs.make_layer_inputs(cfg, "cuda")
+    L, out, dx = _run(cfg, inp)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    W = [f64(inp[n]) for n in ("W1", "W3", "W2")]
+    if cfg.routing == "router":
+        logits = L.ctx_tensor("logits", (T, E), torch.float32)
+        ctx = oracle.layer_forward(f64(inp["x"]), *W, k, Wr=f64(inp["Wr"]),
+                                   bias=moe_inputs.to_f64(inp["bias"]), logits=f64(logits),
+                                   mx=cfg.mx)
+    else:
+        ctx = oracle.layer_forward(f64(inp["x"]), *W, k, topk_idx=np_i(inp["topk_idx"]),
+                                   gates=f64(inp["gates"]), mx=cfg.mx)
+    g = oracle.layer_backward(ctx, f64(inp["dout"]))
+    # routing metadata bit-exact
+    np.testing.assert_array_equal(np_i(L.ctx_tensor("topk_idx", (T, k), torch.int32)), ctx["topk_idx"])
+    np.testing.assert_array_equal(np_i(L.ctx_tensor("dst", (T, k), torch.int32)), ctx["meta"]["dst"])
+    np.testing.assert_array_equal(np_i(L.ctx_tensor("poff", (E + 1,), torch.int32)), ctx["meta"]["poff"])
+    tol = 3e-2 if cfg.mx else 1e-2
+    errs = {
+        "out": rel_err(f64(out), ctx["out"]),
+        "dx": rel_err(f64(dx), g["dx"]),
+        "dW1": rel_err(f64(L.dW1), g["dW1"]),
+        "dW3": rel_err(f64(L.dW3), g["dW3"]),
+        "dW2": rel_err(f64(L.dW2), g["dW2"]),
+    }
+    if cfg.routing == "router":
+        errs["dWr"] = rel_err(L.dWr.cpu().numpy(), g["dWr"])
+    bad = {n: e for n, e in errs.items() if not e < tol}
+    assert not bad, errs
+
+
+def _oracle_on_tokens(cfg, inp, cache, toks):
+    """Oracle fwd + bwd of the sub-batch `toks` (each token's result does not
+    depend on the other tokens), over the experts these tokens choose."""
+    x = f64(inp["x"][toks]); dout = f64(inp["dout"][toks])
+    if cfg.routing == "router":
+        Wr, b = cache["Wr"], cache["b"]
+        idx = oracle.topk_select(oracle.router_logits(x, Wr, b), cfg.k)
+    else:
+        idx = np_i(inp["topk_idx"][toks]); g = f64(inp["gates"][toks])
+    S = np.unique(idx)
+    pos = {int(e): i for i, e in enumerate(S)}
+    Ws = [cache["W"](n, S) for n in ("W1", "W3", "W2")]
+    if cfg.routing == "router":
+        ctx = oracle.layer_forward(x, *Ws, cfg.k, Wr=Wr[:, S], bias=None if b is None else b[S],
+                                   mx=cfg.mx)
+    else:
+        ci = np.vectorize(pos.get)(idx).astype(np.int32)
+        ctx = oracle.layer_forward(x, *Ws, cfg.k, topk_idx=ci, gates=g, mx=cfg.mx)
+    return ctx, oracle.layer_backward(ctx, dout), S, pos
+
+
+@pytest.mark.parametrize("name", ["olmo128", "olmo128_mx", "skewed", "trillion"])
+def test_full_size_layer_sampled(name):
+    cfg = moe_inputs.CONFIGS[name]
+    inp = moe_inputs.make_layer_inputs(cfg, "cuda")
+    L, out, dx = _run(cfg, inp)
+    T, E, k = cfg.T, cfg.E, cfg.k
+    cache = {"Wr": f64(inp["Wr"]), "b": moe_inputs.to_f64(inp["bias"])}
+    wcache = {}
+
+    def W(n, S):
+        key = (n, tuple(S.tolist()))
+        if key not in wcache:
+            wcache.clear()
+            wcache[key] = inp[n][torch.from_numpy(S).cuda()].to(torch.float64).cpu().numpy()
+        return wcache[key]
+    cache["W"] = W
+    tol = 3e-2 if cfg.mx else 1e-2
+    topk = np_i(L.ctx_tensor("topk_idx", (T, k), torch.int32))
+    # routing metadata bit-exact against the oracle's counting sort
+    meta = oracle.routing_metadata(topk, E, 128)
+    np.testing.assert_array_equal(np_i(L.ctx_tensor("dst", (T, k), torch.int32)), meta["dst"])
+    np.testing.assert_array_equal(np_i(L.ctx_tensor("counts", (E,), torch.int32)), meta["counts"])
+    # sampled tokens: out and dx rows
+    rng = np.random.default_rng(cfg.index)
+    toks = np.sort(rng.choice(T, 24, replace=False))
+    ctx, g, S, pos = _oracle_on_tokens(cfg, inp, cache, toks)
+    same = np.all(S[ctx["topk_idx"]] == topk[toks], axis=1)
+    assert same.sum() >= len(toks) - 1           # at most a near-tie
+    assert rel_err(f64(out[toks])[same], ctx["out"][same]) < tol
+    assert rel_err(f64(dx[toks])[same], g["dx"][same]) < tol
+    # sampled experts: every weight gradient of the expert (and its router column)
+    counts = meta["counts"]
+    cand = [e for e in np.argsort(-counts)[:3].tolist() + [int(rng.integers(E))] if counts[e] > 0]
+    for e in cand[:2]:
+        grp = meta["src"][meta["poff"][e]:meta["poff"][e] + counts[e]]
+        ctx, g, S, pos = _oracle_on_tokens(cfg, inp, cache, grp)
+        if not np.all(S[ctx["topk_idx"]] == topk[grp]):
+            continue                             # a near-tie token in the group
+        i = pos[e]
+        assert rel_err(f64(L.dW1[e]), g["dW1"][i]) < tol, ("dW1", e)
+        assert rel_err(f64(L.dW3[e]), g["dW3"][i]) < tol, ("dW3", e)
+        assert rel_err(f64(L.dW2[e]), g["dW2"][i]) < tol, ("dW2", e)
+        if cfg.routing == "router":
+            assert rel_err(L.dWr[:, e].cpu().numpy(), g["dWr"][:, i]) < tol, ("dWr", e)
+
+
+def test_host_buffer_step_matches_device_step():
+    cfg = moe_inputs.CONFIGS["tiny"]
+    inp = moe_inputs.make_layer_inputs(cfg, "cuda")
+    L, out, dx = _run(cfg, inp)
+    xh = inp["x"].cpu().pin_memory(); dh = inp["dout"].cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory(); dxh = torch.empty_like(xh).pin_memory()
+    bufs = [torch.empty_like(inp["x"]) for _ in range(4)]
+    L.step_host(xh, dh, oh, dxh, *bufs)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out.cpu()) and torch.equal(dxh, dx.cpu())

@@ -147,3 +147,39 @@ def test_round_bf16_against_torch():
     v = (rng.normal(size=10000) * np.exp(rng.normal(size=10000) * 5)).astype(np.float32).astype(np.float64)
     ref = torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(oracle.round_bf16(v), ref)
+
+
+def test_grouped_matmuls_equal_block_diagonal_dense_products():
+    """Grouped products equal one dense product with a block-diagonal
+    operand built from the groups (a plain library matmul)."""
+    rng = np.random.default_rng(7)
+    E, K, N = 3, 5, 4
+    poff = np.array([0, 2, 2, 6])           # group 1 empty
+    A = rng.normal(size=(6, K)); B = rng.normal(size=(E, K, N)); dC = rng.normal(size=(6, N))
+    # dense: rows of group e use columns block e of a [6, E*K] expanded A
+    Aexp = np.zeros((6, E * K))
+    for e in range(E):
+        Aexp[poff[e]:poff[e + 1], e * K:(e + 1) * K] = A[poff[e]:poff[e + 1]]
+    Bstack = B.reshape(E * K, N)
+    np.testing.assert_allclose(oracle.grouped_matmul(A, B, poff), Aexp @ Bstack, rtol=1e-13)
+    np.testing.assert_allclose(oracle.grouped_matmul_t(dC, B, poff) , (dC @ Bstack.T).reshape(6, E, K)[np.arange(6), [0, 0, 2, 2, 2, 2]], rtol=1e-13)
+    dB = oracle.grouped_wgrad(A, dC, poff, E)
+    np.testing.assert_allclose(dB.reshape(E * K, N), Aexp.T @ dC, rtol=1e-13, atol=1e-14)
+    assert np.all(dB[1] == 0)
+
+
+def test_backward_pieces_compose_to_layer_backward():
+    T, d, E, F, k = 9, 6, 4, 5, 2
+    x, W1, W3, W2, Wr, dout = _layer(T, d, E, F, 8)
+    ctx = oracle.layer_forward(x, W1, W3, W2, k, Wr=Wr, align=2)
+    g = oracle.layer_backward(ctx, dout)
+    # SwiGLU backward against the closed form of d(silu(a) b)
+    a = np.linspace(-4, 4, 17)
+    s = 1 / (1 + np.exp(-a))
+    d1, d3 = oracle.swiglu_backward(np.ones_like(a), a, np.full_like(a, 2.0))
+    np.testing.assert_allclose(d1, 2.0 * (s + a * s * (1 - s)), rtol=1e-14)
+    np.testing.assert_allclose(d3, a * s, rtol=1e-14)
+    # dY rows are gate-scaled dout rows
+    for t in range(T):
+        for j in range(k):
+            np.testing.assert_allclose(g["dY"][ctx["meta"]["dst"][t, j]], ctx["gates"][t, j] * dout[t])
