@@ -7,8 +7,11 @@ Notation: T tokens, d model width, E experts, k experts per token, F expert
 hidden width; A = T*k assignments.  Everything is float64 unless it is an
 index.  Rounding to bf16 is NOT emulated in the BF16 path (the tolerance
 covers it); the MXFP8 path quantises each GEMM operand along that GEMM's K
-with the MX rule in ``oracle.mx`` and rounds the tensors it quantises to bf16
-first, as the device stores them in bf16 before quantising.
+with the MX rule in ``oracle.mx``, rounds the tensors it quantises to bf16
+first (the device stores them in bf16 before quantising), and lets the saved
+H1/H3 enter the SwiGLU backward at their stored bf16 precision: quantisation
+turns a one-ulp bf16 difference into a one-ulp E4M3 difference, so the MX
+operands must be the same values on both sides.
 """
 from __future__ import annotations
 
@@ -322,7 +325,12 @@ def layer_backward(ctx, dout):
         # GEMM2 dgrad (K = d) and wgrad (K = rows of the group)
         dh = _gemm(dYe, W2[e].T, mx, "rows", "cols")
         dW2[e] = _gemm(he.T, dYe, mx, "rows", "cols")
-        dA1, dA3 = swiglu_backward(dh, H1[a:b], H3[a:b])
+        if mx:
+            # the saved activations enter the backward at their stored (bf16)
+            # precision, so the quantised dA operands are the device's
+            dA1, dA3 = swiglu_backward(dh, round_bf16(H1[a:b]), round_bf16(H3[a:b]))
+        else:
+            dA1, dA3 = swiglu_backward(dh, H1[a:b], H3[a:b])
         if mx:
             dA1 = round_bf16(dA1); dA3 = round_bf16(dA3)
         # GEMM1 dgrad (K = 2F) and wgrad (K = rows of the group)
