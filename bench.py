@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""MoE feed-forward layer, forward + backward, on B200s: throughput bench.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config olmo128]
+    python bench.py --impl reference ...     (the CPU oracle on the host cores)
+
+One step = moe_layer_fwd + moe_layer_bwd on one batch of seeded synthetic
+inputs already resident in HBM (router, routing metadata, dispatch, the two
+SwiGLU grouped GEMMs, combine, and the whole backward including all weight
+gradients).  The N GPUs run independent replicas (the single-GPU layer has
+no exchange step); `value` counts the tokens of all ranks over the slowest
+rank's device time.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import moe_inputs  # noqa: E402
+
+METRIC = "MoE layer fwd+bwd tokens/sec and grouped-GEMM TFLOP/s (% of peak) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="olmo128", choices=sorted(moe_inputs.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = str(index)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", self.index], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                "sw_power_cap"), f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ CPU baseline
+def _oracle_step(oracle, cfg, x, dout, W, Wr, b, topk=None, gates=None):
+    if topk is None:
+        ctx = oracle.layer_forward(x, *W, cfg.k, Wr=Wr, bias=b)
+    else:
+        ctx = oracle.layer_forward(x, *W, cfg.k, topk_idx=topk, gates=gates)
+    oracle.layer_backward(ctx, dout)
+
+
+class OracleRunner:
+    """The CPU oracle, as it stands, on a token sample of the workload."""
+
+    def __init__(self, cfg, inp, target_s):
+        import oracle
+        from threadpoolctl import threadpool_limits
+        self.oracle = oracle
+        self.cfg = cfg
+        self.cores = len(os.sched_getaffinity(0))
+        self._limit = threadpool_limits(self.cores)
+        f64 = moe_inputs.to_f64
+        self.W = [inp[n].to(torch.float64).cpu().numpy() if inp[n].is_cuda else f64(inp[n])
+                  for n in ("W1", "W3", "W2")]
+        self.x = f64(inp["x"]); self.dout = f64(inp["dout"])
+        self.Wr = f64(inp["Wr"]); self.b = f64(inp["bias"])
+        self.topk = None if cfg.routing == "router" else inp["topk_idx"].cpu().numpy()
+        self.gates = None if cfg.routing == "router" else f64(inp["gates"])
+        # grow the sample (doubling) until one step takes about target_s / 2
+        # or more; the groups are padded to 128 rows, so the cost is far from
+        # linear in the sample at small sizes
+        n = min(cfg.T, 256)
+        while True:
+            t = self._time(n)
+            if t >= target_s / 2 or n >= cfg.T:
+                break
+            n = min(cfg.T, 2 * n)
+        self.n, self.last_t = n, t
+
+    def _time(self, n):
+        sl = slice(0, n)
+        t0 = time.perf_counter()
+        _oracle_step(self.oracle, self.cfg, self.x[sl], self.dout[sl], self.W, self.Wr, self.b,
+                     None if self.topk is None else self.topk[sl],
+                     None if self.gates is None else self.gates[sl])
+        return time.perf_counter() - t0
+
+    def step(self):
+        return self._time(self.n)
+
+    def describe(self):
+        return (f"first {self.n} of {self.cfg.T} tokens of the workload, full fwd+bwd of the fp64 "
+                f"NumPy oracle (all {self.cfg.E} experts, groups padded to 128 rows)")
+
+
+# ----------------------------------------------------------------- helpers
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _maxreduce(v, world):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _traffic(kernel_file):
+    """dram bytes per launch of the grouped GEMM from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    src = open(os.path.join(ROOT, "mixture_experts_layer_25_b200", "csrc", kernel_file), "rb").read()
+    if d.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+def _cfg_dict(cfg, extra):
+    d = {"workload": f"{cfg.name}: one MoE SwiGLU FFN layer fwd+bwd, T={cfg.T} tokens, d_model={cfg.d}, "
+                     f"E={cfg.E} experts, top-{cfg.k}, d_ff={cfg.F}, "
+                     f"{'router softmax/top-k' if cfg.routing == 'router' else 'random routing'}"
+                     f"{' + Zipf bias' if cfg.bias else ''}, {'MXFP8' if cfg.mx else 'BF16'} grouped GEMMs",
+         "T": cfg.T, "d_model": cfg.d, "experts": cfg.E, "top_k": cfg.k, "d_ff": cfg.F,
+         "routing": cfg.routing, "grouped_gemm_dtype": "mxfp8" if cfg.mx else "bf16",
+         "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (3 * cfg.E * cfg.d * cfg.F * 2 / 1e9),
+         "parallelism": "replicas (no exchange step in the single-GPU layer)"}
+    d.update(extra)
+    return d
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    world, rank, local = _dist()
+    if rank != 0:
+        return
+    cfg = moe_inputs.CONFIGS[args.config]
+    inp = moe_inputs.make_layer_inputs(cfg, "cpu")
+    r = OracleRunner(cfg, inp, target_s=4.0)
+    for _ in range(args.warmup):
+        r.step()
+    t = 0.0
+    for _ in range(args.steps):
+        t += r.step()
+    value = r.n * args.steps / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _cfg_dict(cfg, {"sample_tokens_per_step": r.n}),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r.cores, "kind": "oracle",
+                             "sample": r.describe()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args):
+    import mixture_experts_layer_25_b200 as moe
+    from mixture_experts_layer_25_b200 import _lib
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    cfg = moe_inputs.CONFIGS[args.config]
+    peaks, peak_kind = _peaks()
+    inp = moe_inputs.make_layer_inputs(cfg, "cuda")
+    layer = moe.MoELayer(T=cfg.T, d=cfg.d, E=cfg.E, k=cfg.k, F=cfg.F, W1=inp["W1"], W3=inp["W3"],
+                         W2=inp["W2"], Wr=inp["Wr"] if cfg.routing == "router" else None,
+                         bias=inp["bias"], topk_idx=inp.get("topk_idx"), gates=inp.get("gates"),
+                         mx=cfg.mx)
+    x, dout = inp["x"], inp["dout"]
+    out = torch.empty_like(x)
+    dx = torch.empty_like(dout)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.forward(x, out)
+        layer.backward(x, dout, dx)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.status.item() != 0:
+        raise RuntimeError(f"device status {layer.status.item()} after warm-up")
+
+    nst = len(_lib.STAGES)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nst)] for _ in range(args.steps)]
+    arrs = [(ctypes.c_void_p * (2 * nst))(*[e.cuda_event for e in row]) for row in evs]
+    for row in evs:
+        for e in row:
+            e.record(stream)     # materialise the handles before use by the library
+    torch.cuda.synchronize()
+    lib = _lib.lib()
+    launches0 = lib.moe_launch_count()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_index = vis.split(",")[local] if vis else str(local)
+    clocks = ClockSampler(smi_index)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        lib.moe_set_stage_events(arrs[i], 2 * nst)
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(world)
+    lib.moe_set_stage_events(None, 0)
+    launches = lib.moe_launch_count() - launches0
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    ms = _maxreduce(ms, world)
+    if layer.status.item() != 0:
+        raise RuntimeError(f"device status {layer.status.item()} after timing")
+
+    # per-stage device time, from the stage events recorded inside the steps
+    recorded = set(range(nst))
+    if not cfg.mx:
+        recorded -= {2, 4, 8, 10, 12, 14}
+    if cfg.routing != "router":
+        recorded -= {17}
+    stage_ms = {}
+    for s in sorted(recorded):
+        v = [evs[i][2 * s].elapsed_time(evs[i][2 * s + 1]) for i in range(args.steps)]
+        stage_ms[_lib.STAGES[s]] = statistics.mean(v)
+
+    T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
+    A = T * k
+    gemm_flops = {"gemm1_swiglu": 4.0 * A * d * F, "gemm2": 2.0 * A * F * d,
+                  "gemm2_dgrad_swiglu_bwd": 2.0 * A * d * F, "gemm2_wgrad": 2.0 * A * F * d,
+                  "gemm1_dgrad": 4.0 * A * F * d, "gemm1_wgrad": 4.0 * A * d * F}
+    gemm_ms = sum(stage_ms[n] for n in gemm_flops)
+    flops = sum(gemm_flops.values())
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    per_gemm = {n: round(gemm_flops[n] / (stage_ms[n] * 1e-3) / 1e12, 1) for n in gemm_flops}
+    peak_key = "bf16_tflops_sustained"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    if cfg.mx:
+        peak *= 2.0   # fp8 dense = 2x bf16 dense (nominal 4.5 vs 2.25 PFLOP/s)
+    bpe = 2
+    mem_bytes = {
+        "route": T * d * bpe + d * E * 4 + T * E * 4 + T * k * 16,
+        "permute": T * d * bpe + A * d * bpe,
+        "combine": A * d * bpe + T * d * bpe,
+        "combine_bwd": T * d * bpe + 2 * A * d * bpe,
+        "unpermute_sum": A * d * bpe + T * d * bpe,
+    }
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    mem = {n: {"GB_s": round(b / (stage_ms[n] * 1e-3) / 1e9, 1),
+               "frac_of_hbm": round(b / (stage_ms[n] * 1e-3) / 1e9 / hbm, 3),
+               "ms": round(stage_ms[n], 4)} for n, b in mem_bytes.items() if n in stage_ms}
+
+    # end to end through the C ABI with host buffers (copies inside)
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory(); dh = dout.cpu().pin_memory()
+        oh = torch.empty_like(xh).pin_memory(); dxh = torch.empty_like(xh).pin_memory()
+        bufs = [torch.empty_like(x) for _ in range(4)]
+        for _ in range(2):
+            layer.step_host(xh, dh, oh, dxh, *bufs)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
+        _barrier(world)
+        a.record(stream)
+        for _ in range(args.steps):
+            layer.step_host(xh, dh, oh, dxh, *bufs)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = _maxreduce(a.elapsed_time(b), world)
+        nb = T * d * 2
+        e2e = {"value": world * T * args.steps / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": 2 * nb, "d2h_bytes_per_step": 2 * nb,
+               "ms_per_step": e_ms / args.steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            r = OracleRunner(cfg, inp, target_s=15.0)
+            t = r.last_t
+            cpu = {"value": r.n / t, "unit": "tokens/s", "cores": r.cores, "kind": "oracle",
+                   "sample": r.describe(), "seconds": round(t, 2)}
+        except MemoryError:
+            cpu = None
+
+    traffic = _traffic("grouped_gemm.cu")
+    line = {
+        "metric": METRIC,
+        "value": world * T * args.steps / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "mxfp8" if cfg.mx else "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 activations and upstream grads, N(0,0.02) random-init weights",
+        "config": _cfg_dict(cfg, {}),
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / peak, 4),
+                     "traffic": traffic,
+                     "kernel": "grouped_gemm_kernel (all 6 launches of a step; algorithmic FLOPs "
+                               "18*T*k*d*F over their summed event time)",
+                     "peak_source": f"{peak_key} of {peak_kind}" + (" x2 for fp8" if cfg.mx else "")},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "detail": {"stage_ms": {n: round(v, 4) for n, v in stage_ms.items()},
+                   "grouped_gemm_tflops": per_gemm, "memory_bound": mem,
+                   "gemm_ms_per_step": round(gemm_ms, 4)},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -112,6 +112,20 @@ typedef enum {
 MOE_API const char* moe_last_error(void);
 /* Library version string. */
 MOE_API const char* moe_version(void);
+/* Number of kernels this library has launched in this process. */
+MOE_API unsigned long long moe_launch_count(void);
+
+/* Benchmark hook: when set (per host thread), moe_layer_fwd / moe_layer_bwd
+ * record events[2*s] before and events[2*s+1] after stage s on the stream
+ * (cudaEvent_t handles; n = number of handles; NULL disables).  Stages:
+ *   0 route  1 permute  2 quantise fwd weights  3 GEMM1+SwiGLU  4 quantise h
+ *   5 GEMM2  6 combine  7 combine bwd  8 quantise for GEMM2 dgrad
+ *   9 GEMM2 dgrad+SwiGLU bwd  10 quantise for GEMM2 wgrad  11 GEMM2 wgrad
+ *   12 quantise for GEMM1 dgrad  13 GEMM1 dgrad  14 quantise for GEMM1 wgrad
+ *   15 GEMM1 wgrad  16 unpermute-sum  17 router weight grad
+ * (quantise stages run in MXFP8 mode only). */
+#define MOE_NUM_STAGES 18
+MOE_API void moe_set_stage_events(void* const* events, int n);
 
 /* ------------------------------------------------------------------ route
  * Router and GPU-resident routing metadata ([OC3-ja] "ルーティングと計算の最適化":

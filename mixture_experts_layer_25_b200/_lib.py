@@ -55,6 +55,8 @@ class CtxView(ctypes.Structure):
 _SIGS = {
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_version": (ctypes.c_char_p, []),
+    "moe_launch_count": (ctypes.c_ulonglong, []),
+    "moe_set_stage_events": (None, [ctypes.POINTER(P), I]),
     "moe_route_workspace_size": (Z, [I, I]),
     "moe_route": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, Z, P, P]),
     "moe_permute": (I, [P, P, P, P, I, I, I, I, I, P, P, P, P]),
@@ -100,6 +102,12 @@ def call(name: str, *args) -> None:
     code = getattr(lib(), name)(*args)
     if code != MOE_OK:
         raise MoeError(name, code, lib().moe_last_error().decode())
+
+
+STAGES = ["route", "permute", "quant_w_fwd", "gemm1_swiglu", "quant_h", "gemm2", "combine",
+          "combine_bwd", "quant_dgrad2", "gemm2_dgrad_swiglu_bwd", "quant_wgrad2", "gemm2_wgrad",
+          "quant_dgrad1", "gemm1_dgrad", "quant_wgrad1", "gemm1_wgrad", "unpermute_sum",
+          "router_wgrad"]
 
 
 def exported_names() -> list[str]:

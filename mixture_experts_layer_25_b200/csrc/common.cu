@@ -1,5 +1,7 @@
 // Host-side helpers: per-thread error message, SM count, version.
 #include <stdarg.h>
+
+#include <atomic>
 #include <stdio.h>
 
 #include "common.cuh"
@@ -15,6 +17,10 @@ void set_error(const char* fmt, ...) {
   va_end(ap);
 }
 
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -26,5 +32,7 @@ int num_sms() {
 }  // namespace moe
 
 extern "C" const char* moe_last_error(void) { return moe::g_err; }
+
+extern "C" unsigned long long moe_launch_count(void) { return moe::g_launches.load(); }
 
 extern "C" const char* moe_version(void) { return "libmoe 0.1 (sm_100a)"; }

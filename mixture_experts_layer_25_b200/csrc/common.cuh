@@ -15,6 +15,7 @@ namespace moe {
 
 // ---------------------------------------------------------------- host side
 void set_error(const char* fmt, ...);
+void count_launch();
 
 #define MOE_CHECK_ARG(cond, ...)                     \
   do {                                               \
@@ -26,6 +27,7 @@ void set_error(const char* fmt, ...);
 
 #define MOE_CHECK_LAUNCH(what)                                                   \
   do {                                                                           \
+    ::moe::count_launch();                                                       \
     cudaError_t e_ = cudaGetLastError();                                         \
     if (e_ != cudaSuccess) {                                                     \
       ::moe::set_error("%s: %s", what, cudaGetErrorString(e_));                  \

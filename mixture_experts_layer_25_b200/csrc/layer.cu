@@ -88,10 +88,26 @@ size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   return moe::round_up(l.off, 256);
 }
 
-template <class T>
-T* bf(void* p) { return static_cast<T*>(p); }
+thread_local void* const* g_events = nullptr;
+thread_local int g_nevents = 0;
+
+// record the start (end = false) or end of stage s, if a benchmark asked
+void mark(int s, bool end, cudaStream_t st) {
+  const int i = 2 * s + (end ? 1 : 0);
+  if (g_events && i < g_nevents && g_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(g_events[i]), st);
+}
+
+enum Stage { S_ROUTE, S_PERMUTE, S_QW, S_GEMM1, S_QH, S_GEMM2, S_COMBINE, S_COMBINE_BWD,
+             S_QD2, S_DGRAD2, S_QW2, S_WGRAD2, S_QD1, S_DGRAD1, S_QW1, S_WGRAD1, S_UNPERMUTE,
+             S_ROUTER_WGRAD };
 
 }  // namespace
+
+extern "C" void moe_set_stage_events(void* const* events, int n) {
+  g_events = events;
+  g_nevents = events ? n : 0;
+}
 
 using moe::set_error;
 
@@ -144,31 +160,52 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
       return MOE_ERR_CUDA;
     }
   }
+  mark(S_ROUTE, false, s);
   MOE_TRY(moe_route(x, w->Wr, w->bias, T, d, E, k, L->align, L->route_mode, c.topk_idx, c.gates,
                     c.counts, c.offsets, c.poff, c.dst, c.src, A, c.logits, c.ws, c.ws_bytes,
                     dev_status, stream));
+  mark(S_ROUTE, true, s);
   if (!mx) {
+    mark(S_PERMUTE, false, s);
     MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, nullptr, nullptr, stream));
+    mark(S_PERMUTE, true, s);
+    mark(S_GEMM1, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_BF16, c.Xp, nullptr, w->W1, nullptr, w->W3, nullptr, c.poff,
                                  E, A, F, d, MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
+    mark(S_GEMM1, true, s);
+    mark(S_GEMM2, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_BF16, c.h, nullptr, w->W2, nullptr, nullptr, nullptr, c.poff,
                                  E, A, d, F, MOE_EPI_NONE, c.Y, nullptr, dev_status, stream));
+    mark(S_GEMM2, true, s);
   } else {
     const int32_t* nrows = c.poff + E;
     uint8_t* W1q = c.W13_q; uint8_t* W3q = c.W13_q + (size_t)E * d * F;
     uint8_t* W1s = c.W13_s; uint8_t* W3s = c.W13_s + (size_t)E * d * F / 32;
+    mark(S_PERMUTE, false, s);
     MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, c.Xp_q, c.Xp_s, stream));
+    mark(S_PERMUTE, true, s);
     // weights along the fwd GEMMs' K: W1/W3 down d, W2 down F
+    mark(S_QW, false, s);
     MOE_TRY(mx_quantize(w->W1, E * d, F, 1, nullptr, E, nullptr, W1q, W1s, stream));
     MOE_TRY(mx_quantize(w->W3, E * d, F, 1, nullptr, E, nullptr, W3q, W3s, stream));
     MOE_TRY(mx_quantize(w->W2, E * F, d, 1, nullptr, E, nullptr, c.W2_q, c.W2_s, stream));
+    mark(S_QW, true, s);
+    mark(S_GEMM1, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.Xp_q, c.Xp_s, W1q, W1s, W3q, W3s, c.poff, E, A, F, d,
                                  MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
+    mark(S_GEMM1, true, s);
+    mark(S_QH, false, s);
     MOE_TRY(mx_quantize(c.h, A, F, 0, c.poff, E, nrows, c.h_q, c.h_s, stream));
+    mark(S_QH, true, s);
+    mark(S_GEMM2, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.h_q, c.h_s, c.W2_q, c.W2_s, nullptr, nullptr, c.poff,
                                  E, A, d, F, MOE_EPI_NONE, c.Y, nullptr, dev_status, stream));
+    mark(S_GEMM2, true, s);
   }
-  return moe_unpermute_combine(c.Y, c.gates, c.dst, T, k, d, out, stream);
+  mark(S_COMBINE, false, s);
+  MOE_TRY(moe_unpermute_combine(c.Y, c.gates, c.dst, T, k, d, out, stream));
+  mark(S_COMBINE, true, s);
+  return MOE_OK;
 }
 
 extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w,
@@ -183,50 +220,82 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   const int T = L->T, d = L->d, E = L->E, k = L->k, F = L->F, A = c.A_pad_max;
   const bool mx = L->dtype == MOE_MXFP8;
 
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  mark(S_COMBINE_BWD, false, s);
   MOE_TRY(moe_combine_bwd(dout, c.Y, c.gates, c.dst, c.offsets, c.poff, T, k, d, E, c.dY, c.dg,
                           router ? c.dl : nullptr, router ? c.dl_rows : nullptr, stream));
+  mark(S_COMBINE_BWD, true, s);
   if (!mx) {
+    mark(S_DGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_dgrad(MOE_BF16, c.dY, nullptr, w->W2, nullptr, nullptr, nullptr,
                                    c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
                                    dev_status, stream));
+    mark(S_DGRAD2, true, s);
+    mark(S_WGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, E, A, F, d,
                                    G->dW2, nullptr, dev_status, stream));
+    mark(S_WGRAD2, true, s);
+    mark(S_DGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_dgrad(MOE_BF16, c.dA13, nullptr, w->W1, nullptr, w->W3, nullptr,
                                    c.poff, E, A, F, d, MOE_EPI_NONE, nullptr, c.dXp, dev_status,
                                    stream));
+    mark(S_DGRAD1, true, s);
+    mark(S_WGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, E, A, d, F,
                                    G->dW1, G->dW3, dev_status, stream));
+    mark(S_WGRAD1, true, s);
   } else {
     const int32_t* nrows = c.poff + E;
     uint8_t* W1q = c.W13t_q; uint8_t* W3q = c.W13t_q + (size_t)E * d * F;
     uint8_t* W1s = c.W13t_s; uint8_t* W3s = c.W13t_s + (size_t)E * d * F / 32;
     // GEMM2 dgrad: K = d.  dY along d, W2 along d (rows of the [E*F, d] view)
+    mark(S_QD2, false, s);
     MOE_TRY(mx_quantize(c.dY, A, d, 0, c.poff, E, nrows, c.dY_q, c.dY_s, stream));
     MOE_TRY(mx_quantize(w->W2, E * F, d, 0, nullptr, E, nullptr, c.W2t_q, c.W2t_s, stream));
+    mark(S_QD2, true, s);
+    mark(S_DGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dY_q, c.dY_s, c.W2t_q, c.W2t_s, nullptr, nullptr,
                                    c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
                                    dev_status, stream));
+    mark(S_DGRAD2, true, s);
     // GEMM2 wgrad: K = rows of the group.  h and dY down their columns
+    mark(S_QW2, false, s);
     MOE_TRY(mx_quantize(c.h, A, F, 1, c.poff, E, nrows, c.hT_q, c.hT_s, stream));
     MOE_TRY(mx_quantize(c.dY, A, d, 1, c.poff, E, nrows, c.dYT_q, c.dYT_s, stream));
+    mark(S_QW2, true, s);
+    mark(S_WGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff, E, A, F,
                                    d, G->dW2, nullptr, dev_status, stream));
+    mark(S_WGRAD2, true, s);
     // GEMM1 dgrad: K = 2F.  dA13 along 2F, W1/W3 along F
+    mark(S_QD1, false, s);
     MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 0, c.poff, E, nrows, c.dA_q, c.dA_s, stream));
     MOE_TRY(mx_quantize(w->W1, E * d, F, 0, nullptr, E, nullptr, W1q, W1s, stream));
     MOE_TRY(mx_quantize(w->W3, E * d, F, 0, nullptr, E, nullptr, W3q, W3s, stream));
+    mark(S_QD1, true, s);
+    mark(S_DGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, W1q, W1s, W3q, W3s, c.poff, E, A, F,
                                    d, MOE_EPI_NONE, nullptr, c.dXp, dev_status, stream));
+    mark(S_DGRAD1, true, s);
     // GEMM1 wgrad: K = rows of the group.  Xp and dA13 down their columns
+    mark(S_QW1, false, s);
     MOE_TRY(mx_quantize(c.Xp, A, d, 1, c.poff, E, nrows, c.XpT_q, c.XpT_s, stream));
     MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 1, c.poff, E, nrows, c.dAT_q, c.dAT_s, stream));
+    mark(S_QW1, true, s);
+    mark(S_WGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff, E, A, d,
                                    F, G->dW1, G->dW3, dev_status, stream));
+    mark(S_WGRAD1, true, s);
   }
+  mark(S_UNPERMUTE, false, s);
   MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, c.topk_idx, router ? c.dl : nullptr,
                             router ? w->Wr : nullptr, T, k, d, E, dx, c.ws, c.ws_bytes, stream));
-  if (router && G->dWr)
+  mark(S_UNPERMUTE, true, s);
+  if (router && G->dWr) {
+    mark(S_ROUTER_WGRAD, false, s);
     MOE_TRY(moe_router_wgrad(x, c.src, c.dl_rows, c.offsets, c.poff, T, d, E, G->dWr, stream));
+    mark(S_ROUTER_WGRAD, true, s);
+  }
   return MOE_OK;
 }
 
