@@ -269,11 +269,12 @@ def run_ours(args):
 
     nst = len(_lib.STAGES)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nst)] for _ in range(args.steps)]
-    arrs = [(ctypes.c_void_p * (2 * nst))(*[e.cuda_event for e in row]) for row in evs]
     for row in evs:
         for e in row:
-            e.record(stream)     # materialise the handles before use by the library
+            e.record(stream)     # torch creates the event handles on first record
     torch.cuda.synchronize()
+    arrs = [(ctypes.c_void_p * (2 * nst))(*[e.cuda_event for e in row]) for row in evs]
+    assert all(a[i] for a in arrs for i in range(2 * nst))
     lib = _lib.lib()
     launches0 = lib.moe_launch_count()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
