@@ -152,6 +152,29 @@ MOE_API moe_status_t moe_route(const void* x, const float* Wr, const float* bias
                        int32_t* src, int A_pad_max, float* logits, void* ws, size_t ws_bytes,
                        int32_t* dev_status, moe_stream_t stream);
 
+/* moe_route_noalloc: moe_route with no workspace argument, for callers that
+ * cannot allocate device memory while they run (a host whose device memory
+ * is owned by a pooling allocator, or a latency-critical loop that must not
+ * call cudaMalloc, which can synchronise the device and take an unbounded
+ * time).  The pages have no counterpart to this call; it is a library
+ * convenience.  Its scratch is a fixed, library-owned array in device memory
+ * of MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES (4 MiB) on every device that loads
+ * the library, kept until the process exits; the caller still passes all
+ * inputs and outputs.  Limit: moe_route_workspace_size(T, E) =
+ * ceil(T/32)*E*4 bytes must fit (e.g. T <= 262144 with E = 128); larger
+ * sizes return MOE_ERR_INVALID_ARG.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress), so make that first call
+ * before any stream capture.  All calls share the one array: calls that
+ * overlap on the GPU (other streams, other host threads) race and must be
+ * serialised by the caller.  Arguments and results as moe_route. */
+#define MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES (4u << 20)
+MOE_API moe_status_t moe_route_noalloc(const void* x, const float* Wr, const float* bias, int T,
+                                       int d, int E, int k, int align, int mode,
+                                       int32_t* topk_idx, float* gates, int32_t* counts,
+                                       int32_t* offsets, int32_t* poff, int32_t* dst,
+                                       int32_t* src, int A_pad_max, float* logits,
+                                       int32_t* dev_status, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- permute
  * Rowwise dispatch ([OC3-ja] "ルーティングと計算の最適化": routed tokens are
  * written directly into the experts' input buffers): Xp[dst[t,j]] = x[t]

@@ -59,6 +59,7 @@ _SIGS = {
     "moe_set_stage_events": (None, [ctypes.POINTER(P), I]),
     "moe_route_workspace_size": (Z, [I, I]),
     "moe_route": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, Z, P, P]),
+    "moe_route_noalloc": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P]),
     "moe_permute": (I, [P, P, P, P, I, I, I, I, I, P, P, P, P]),
     "mx_quantize": (I, [P, I, I, I, P, I, P, P, P, P]),
     "moe_grouped_gemm_fwd": (I, [I, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P]),

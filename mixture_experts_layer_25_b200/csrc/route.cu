@@ -14,6 +14,8 @@
 //   3. route_scatter: dst = poff[e] + block offset + in-block rank, src, and
 //      -1 for every pad row.
 // The result is the stable counting sort of the assignments by expert.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -376,4 +378,71 @@ extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* b
                                                   A_pad_max, nA);
   MOE_CHECK_LAUNCH("route_scatter");
   return MOE_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Routing without any device allocation by the caller.
+//
+// Some callers cannot call cudaMalloc once they are running: a host whose
+// device memory is owned by a pooling allocator, or a latency-critical loop
+// that must not allocate (an allocation can synchronise the device and take
+// an unbounded time).  This entry point gives them the router and routing
+// metadata with the block-histogram scratch held in a fixed array that the
+// library owns in device memory.  Inputs and outputs still come from the
+// caller.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+// One copy per device that loads the library; held until the process exits.
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The array's
+// name is only a host-side stand-in, so the address is looked up once per
+// device with cudaGetSymbolAddress.
+moe_status_t scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    set_error("moe_route_noalloc: no usable current device");
+    return MOE_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || !p) {
+      set_error("moe_route_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+      return MOE_ERR_CUDA;
+    }
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_route_noalloc(const void* x, const float* Wr, const float* bias,
+                                          int T, int d, int E, int k, int align, int mode,
+                                          int32_t* topk_idx, float* gates, int32_t* counts,
+                                          int32_t* offsets, int32_t* poff, int32_t* dst,
+                                          int32_t* src, int A_pad_max, float* logits,
+                                          int32_t* dev_status, moe_stream_t stream) {
+  MOE_CHECK_ARG(T > 0 && E > 0, "moe_route_noalloc: bad T/E");
+  const size_t need = moe_route_workspace_size(T, E);
+  MOE_CHECK_ARG(need <= kNoAllocScratchBytes,
+                "moe_route_noalloc: needs %zu scratch bytes (ceil(T/32)*E*4) but the fixed "
+                "array holds %zu; use moe_route with a caller workspace",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  MOE_TRY(scratch_for_current_device(&scratch));
+  // the histogram rows are fully written by the first launch before they are
+  // read, so nothing in the shared array needs clearing between calls
+  return moe_route(x, Wr, bias, T, d, E, k, align, mode, topk_idx, gates, counts, offsets, poff,
+                   dst, src, A_pad_max, logits, scratch, kNoAllocScratchBytes, dev_status,
+                   stream);
 }
