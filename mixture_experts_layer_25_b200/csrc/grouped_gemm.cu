@@ -8,10 +8,12 @@
 // Design (sm_100a):
 //  * persistent CTAs (one per SM), 192 threads: warp 0 issues TMA loads,
 //    warp 1 issues tcgen05.mma (one thread) and owns TMEM, warps 2..5 are
-//    the epilogue (one accumulator row per thread, TMEM -> registers ->
-//    global).
+//    the epilogue: each owns 32 accumulator rows, moves 32-column chunks
+//    TMEM -> registers -> a 64-byte-swizzled shared-memory box -> TMA bulk
+//    store (the SwiGLU backward also TMA-loads its H1/H3 chunks), so global
+//    traffic is whole coalesced boxes.
 //  * tile 128 x 256, fp32 accumulators in TMEM (two buffers for BF16, so the
-//    epilogue of tile i overlaps the main loop of tile i+1), a 4-stage
+//    epilogue of tile i overlaps the main loop of tile i+1), a 3- or 4-stage
 //    shared-memory ring fed by TMA with 128-byte swizzle.
 //  * device-side tile schedule read from poff: "rows" mode walks the
 //    128-row tiles of the expert-contiguous buffer (every group starts on a
@@ -39,8 +41,9 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int STAGES = 4;
 constexpr int NUM_THREADS = 192;
+constexpr int CHUNK = 32;           // epilogue columns per staged box
+constexpr int BOX_BYTES = 32 * CHUNK * 2;   // 32 rows x 32 bf16
 constexpr int A_BYTES = BM * 128;   // 128-byte rows (64 bf16 or 128 fp8 of K)
 constexpr int B_BYTES = BN * 128;
 constexpr int SFA_BYTES = 512;      // 128 rows x 4 scale bytes
@@ -49,6 +52,22 @@ constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2 };
+
+// pipeline depth and per-warp staging (boxes of 2 KB) for each epilogue,
+// within the 227 KB of shared memory per CTA: STORE double-buffers one box,
+// SwiGLU stages h / H1 / H3, the SwiGLU backward double-buffers H1/H3 pairs
+template <bool MX, int EPI> struct EpiCfg {
+  static constexpr int STAGES = (EPI == EPI_SWIGLU_BWD || (MX && EPI == EPI_SWIGLU)) ? 3 : 4;
+  static constexpr int STG = (EPI == EPI_STORE ? 2 : EPI == EPI_SWIGLU ? 3 : 4) * BOX_BYTES;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES +
+                                 (MX ? SFA_BYTES + SFB_BYTES : 0)) + 4 * STG;
+};
+
+// byte offset of 16-byte chunk j of row r inside a [32 rows x 64 B] box
+// stored with the 64-byte swizzle (chunk index XOR row bits 1..2)
+__device__ __forceinline__ uint32_t sw64(int r, int j) {
+  return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
 enum BLoad { B_MN = 0, B_MN_DUAL_N = 1, B_K = 2, B_K_DUAL_K = 3 };
 
 struct Params {
@@ -68,6 +87,7 @@ struct Params {
   __nv_bfloat16* C2; int n_split;
   __nv_bfloat16* aux; long long ld_aux; int half;
   long long c_expert_stride;
+  int k_out;          // wgrad: output rows per expert (K of the weight)
   int32_t* status;
 };
 
@@ -132,7 +152,12 @@ template <bool MX, bool A_MN, int BLOAD, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmB3, const Params p) {
+                    const __grid_constant__ CUtensorMap tmB3,
+                    const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmC2,
+                    const __grid_constant__ CUtensorMap tmIn, const Params p) {
+  constexpr int STAGES = EpiCfg<MX, EPI>::STAGES;
+  constexpr int STG = EpiCfg<MX, EPI>::STG;
   constexpr int ELEM = MX ? 1 : 2;
   constexpr int BK = 128 / ELEM;                 // K per stage (128-byte rows)
   constexpr int MMA_K = MX ? 32 : 16;
@@ -147,7 +172,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar;
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar, in_bar[4][2];
   __shared__ uint32_t tmem_slot;
   __shared__ int poff_s[MAX_E + 1];
   __shared__ volatile int abort_flag;
@@ -157,6 +182,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* sA = smem;                                  // STAGES x A_BYTES
   uint8_t* sB = smem + STAGES * A_BYTES;               // STAGES x B_BYTES
   uint8_t* sSF = sB + STAGES * B_BYTES;                // STAGES x (SFA + SFB), MX only
+  uint8_t* sStg = sSF + (MX ? STAGES * (SFA_BYTES + SFB_BYTES) : 0);   // 4 x STG (epilogue)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -172,12 +198,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_init(&acc_empty[a], 4);
     }
     mbar_init(&drain_bar, 1);
+    for (int w = 0; w < 4; ++w) {
+      mbar_init(&in_bar[w][0], 1);
+      mbar_init(&in_bar[w][1], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch(&tmA);
     tma_prefetch(&tmB);
     if (BLOAD == B_MN_DUAL_N || BLOAD == B_K_DUAL_K) tma_prefetch(&tmB3);
+    tma_prefetch(&tmC);
+    if (EPI == EPI_SWIGLU || (EPI == EPI_STORE && p.wgrad)) tma_prefetch(&tmC2);
+    if (EPI == EPI_SWIGLU_BWD) tma_prefetch(&tmIn);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_slot, TMEM_COLS);
@@ -345,34 +378,43 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
-    const int r = q * 32 + lane;            // accumulator row of this thread
+    const int r = lane;                     // row inside the warp's 32-row box
+    uint8_t* stg = sStg + q * STG;          // this warp's staging boxes
+    uint32_t in_phase = 0;                  // bit i: parity of in_bar[q][i]
+    uint32_t in_pending = 0;                // bit i: a load into pair i not yet waited for (lane 0)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const Tile t = decode(p, poff_s, tile);
       const int nkb = group_kb(t);
       const int acc = ACC_BUFS == 2 ? (it & 1) : 0;
       const uint32_t acc_par = ACC_BUFS == 2 ? ((it >> 1) & 1) : (it & 1);
+      const bool empty = nkb <= 0;
+      const int y0 = (p.wgrad ? t.e * p.k_out + t.m0 : t.row0) + q * 32;
+
+      if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // H1/H3 chunk 0 does not depend on the accumulator: fetch it now
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          mbar_arrive_expect_tx(&in_bar[q][0], 2 * BOX_BYTES);
+          tma_load_2d(stg, &tmIn, &in_bar[q][0], t.nt * BN, y0);
+          tma_load_2d(stg + BOX_BYTES, &tmIn, &in_bar[q][0], p.half + t.nt * BN, y0);
+          in_pending |= 1u;
+        }
+      }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_par, &abort_flag, p.status, kWaitLimitNs);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256;
-      const bool empty = nkb <= 0;
 
       if constexpr (EPI == EPI_STORE) {
-        __nv_bfloat16* out;
         const int n0 = t.nt * BN;
-        if (!p.wgrad) {
-          out = p.C + (long long)(t.row0 + r) * p.ldc + n0;
-        } else if (p.C2 && n0 >= p.n_split) {
-          out = p.C2 + (long long)t.e * p.c_expert_stride + (long long)(t.m0 + r) * p.ldc +
-                (n0 - p.n_split);
-        } else {
-          out = p.C + (long long)t.e * p.c_expert_stride + (long long)(t.m0 + r) * p.ldc + n0;
-        }
+        const CUtensorMap* map = &tmC;
+        int x0 = n0;
+        if (p.wgrad && p.n_split > 0 && n0 >= p.n_split) { map = &tmC2; x0 = n0 - p.n_split; }
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = 0; c < BN; c += CHUNK) {
           uint32_t v[32];
           if (!empty) {
             tmem_ld32(tbase + c, v);
@@ -381,87 +423,137 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          uint4* o = reinterpret_cast<uint4*>(out + c);
+          uint8_t* buf = stg + ((c / CHUNK) & 1) * BOX_BYTES;
+          if (lane == 0) bulk_wait_read<1>();    // the store that used `buf` has read it
+          __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int j = 0; j < 4; ++j) {
             uint4 w;
-            w.x = bf16x2_bits(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-            w.y = bf16x2_bits(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-            w.z = bf16x2_bits(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-            w.w = bf16x2_bits(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-            o[i] = w;
+            w.x = bf16x2_bits(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
+            w.y = bf16x2_bits(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
+            w.z = bf16x2_bits(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
+            w.w = bf16x2_bits(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+            *reinterpret_cast<uint4*>(buf + sw64(r, j)) = w;
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(map, buf, x0 + c, y0);
+            bulk_commit();
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
         // accumulator columns [0,128) = A W1, [128,256) = A W3 for the output
         // columns [nt*128, nt*128 + 128)
-        const long long row = t.row0 + r;
         const int n0 = t.nt * (BN / 2);
-        __nv_bfloat16* hout = p.C + row * p.ldc + n0;
-        __nv_bfloat16* a1 = p.aux ? p.aux + row * p.ld_aux + n0 : nullptr;
-        __nv_bfloat16* a3 = p.aux ? p.aux + row * p.ld_aux + p.half + n0 : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
+        for (int c = 0; c < BN / 2; c += CHUNK) {
           uint32_t g[32], u[32];
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + BN / 2 + c, u);
           tmem_wait_ld();
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int j = 0; j < 4; ++j) {
             uint4 hw, gw, uw;
             uint32_t* hp = &hw.x;
             uint32_t* gp = &gw.x;
             uint32_t* up = &uw.x;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float g0 = __uint_as_float(g[8 * i + 2 * j]);
-              const float g1 = __uint_as_float(g[8 * i + 2 * j + 1]);
-              const float u0 = __uint_as_float(u[8 * i + 2 * j]);
-              const float u1 = __uint_as_float(u[8 * i + 2 * j + 1]);
-              hp[j] = bf16x2_bits(silu_f(g0) * u0, silu_f(g1) * u1);
-              gp[j] = bf16x2_bits(g0, g1);
-              up[j] = bf16x2_bits(u0, u1);
+            for (int i = 0; i < 4; ++i) {
+              const float g0 = __uint_as_float(g[8 * j + 2 * i]);
+              const float g1 = __uint_as_float(g[8 * j + 2 * i + 1]);
+              const float u0 = __uint_as_float(u[8 * j + 2 * i]);
+              const float u1 = __uint_as_float(u[8 * j + 2 * i + 1]);
+              hp[i] = bf16x2_bits(silu_f(g0) * u0, silu_f(g1) * u1);
+              gp[i] = bf16x2_bits(g0, g1);
+              up[i] = bf16x2_bits(u0, u1);
             }
-            reinterpret_cast<uint4*>(hout + c)[i] = hw;
-            if (a1) {
-              reinterpret_cast<uint4*>(a1 + c)[i] = gw;
-              reinterpret_cast<uint4*>(a3 + c)[i] = uw;
+            *reinterpret_cast<uint4*>(stg + sw64(r, j)) = hw;
+            *reinterpret_cast<uint4*>(stg + BOX_BYTES + sw64(r, j)) = gw;
+            *reinterpret_cast<uint4*>(stg + 2 * BOX_BYTES + sw64(r, j)) = uw;
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, stg, n0 + c, y0);
+            if (p.aux) {
+              tma_store_2d(&tmC2, stg + BOX_BYTES, n0 + c, y0);
+              tma_store_2d(&tmC2, stg + 2 * BOX_BYTES, p.half + n0 + c, y0);
             }
+            bulk_commit();
           }
         }
       } else {  // EPI_SWIGLU_BWD: accumulator = dh for columns [nt*256, +256)
-        const long long row = t.row0 + r;
         const int n0 = t.nt * BN;
-        const __nv_bfloat16* h1 = p.aux + row * p.ld_aux + n0;
-        const __nv_bfloat16* h3 = p.aux + row * p.ld_aux + p.half + n0;
-        __nv_bfloat16* d1 = p.C + row * p.ldc + n0;
-        __nv_bfloat16* d3 = p.C + row * p.ldc + p.half + n0;
+        constexpr int NCH = BN / CHUNK;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
+        for (int ci = 0; ci < NCH; ++ci) {
+          const int c = ci * CHUNK;
+          const int pr = ci & 1;                      // staging pair of this chunk
+          uint8_t* b1 = stg + pr * 2 * BOX_BYTES;
+          uint8_t* b3 = b1 + BOX_BYTES;
+          if (ci + 1 < NCH && lane == 0) {            // prefetch the next chunk's H1/H3
+            uint8_t* n1 = stg + (pr ^ 1) * 2 * BOX_BYTES;
+            bulk_wait_read<0>();                      // its pair's previous stores have read it
+            mbar_arrive_expect_tx(&in_bar[q][pr ^ 1], 2 * BOX_BYTES);
+            tma_load_2d(n1, &tmIn, &in_bar[q][pr ^ 1], n0 + c + CHUNK, y0);
+            tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[q][pr ^ 1], p.half + n0 + c + CHUNK, y0);
+            in_pending |= 1u << (pr ^ 1);
+          }
           uint32_t v[32];
           tmem_ld32(tbase + c, v);
           tmem_wait_ld();
+          int got = 1;
+          if (lane == 0)
+            got = mbar_wait(&in_bar[q][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
+                            kWaitLimitNs);
+          got = __shfl_sync(0xffffffffu, got, 0);
+          if (got) {
+            in_phase ^= 1u << pr;
+            in_pending &= ~(1u << pr);
+          }
+          if (!got) { ok = 0; break; }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int j = 0; j < 4; ++j) {
             float f1[8], f3[8], o1[8], o3[8];
-            unpack8(reinterpret_cast<const uint4*>(h1 + c)[i], f1);
-            unpack8(reinterpret_cast<const uint4*>(h3 + c)[i], f3);
+            unpack8(*reinterpret_cast<const uint4*>(b1 + sw64(r, j)), f1);
+            unpack8(*reinterpret_cast<const uint4*>(b3 + sw64(r, j)), f3);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float dh = __uint_as_float(v[8 * i + j]);
-              const float z = f1[j];
-              const float s = 1.0f / (1.0f + __expf(-z));
-              o1[j] = dh * f3[j] * s * (1.0f + z * (1.0f - s));
-              o3[j] = dh * z * s;
+            for (int i = 0; i < 8; ++i) {
+              const float dh = __uint_as_float(v[8 * j + i]);
+              const float z = f1[i];
+              const float sg = 1.0f / (1.0f + __expf(-z));
+              o1[i] = dh * f3[i] * sg * (1.0f + z * (1.0f - sg));
+              o3[i] = dh * z * sg;
             }
-            reinterpret_cast<uint4*>(d1 + c)[i] = pack8(o1);
-            reinterpret_cast<uint4*>(d3 + c)[i] = pack8(o3);
+            *reinterpret_cast<uint4*>(b1 + sw64(r, j)) = pack8(o1);
+            *reinterpret_cast<uint4*>(b3 + sw64(r, j)) = pack8(o3);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, b1, n0 + c, y0);
+            tma_store_2d(&tmC, b3, p.half + n0 + c, y0);
+            bulk_commit();
           }
         }
+        if (!ok) break;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+    if (lane == 0) bulk_wait_all();     // every store has landed before the CTA exits
+    if constexpr (EPI == EPI_SWIGLU_BWD) {
+      // a prefetch issued for a tile that was then abandoned must land too
+      if (lane == 0) {
+        volatile int no_abort = 0;
+        for (int i = 0; i < 2; ++i)
+          if (in_pending & (1u << i))
+            mbar_wait(&in_bar[q][i], (in_phase >> i) & 1, &no_abort, p.status, kWaitLimitNs);
+      }
     }
   }
 
@@ -491,7 +583,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D map over a row-major [outer, inner] array of 1- or 2-byte elements,
 // box {box_inner, box_outer}, 128-byte swizzle.
 moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner,
-                      uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+                      uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                      CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) {
     set_error("cuTensorMapEncodeTiled unavailable");
@@ -503,7 +596,7 @@ moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                   2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed (%d): inner %llu outer %llu box %u x %u", (int)r,
@@ -513,15 +606,19 @@ moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t
   return MOE_OK;
 }
 
-constexpr size_t smem_bytes(bool mx) {
-  return 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + (mx ? SFA_BYTES + SFB_BYTES : 0));
+// epilogue box map: [outer, inner] bf16, 32 x 32 box, 64-byte swizzle
+moe_status_t make_out_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
+  return make_map(m, base, 2, inner, outer, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+struct Maps {
+  CUtensorMap a, b, b3, c, c2, in;
+};
+
 template <bool MX, bool A_MN, int BLOAD, int EPI>
-moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3,
-                    const Params& p, int max_tiles, cudaStream_t s) {
+moe_status_t launch(const Maps& m, const Params& p, int max_tiles, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI>;
-  const size_t smem = smem_bytes(MX);
+  const size_t smem = EpiCfg<MX, EPI>::SMEM;
   static bool attr = false;   // one per instantiation
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -532,7 +629,7 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
     attr = true;
   }
   const int grid = max(1, min(num_sms(), max_tiles));
-  kern<<<grid, NUM_THREADS, smem, s>>>(a, b, b3, p);
+  kern<<<grid, NUM_THREADS, smem, s>>>(m.a, m.b, m.b3, m.c, m.c2, m.in, p);
   MOE_CHECK_LAUNCH("grouped_gemm");
   return MOE_OK;
 }
@@ -575,16 +672,18 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   p.b3_sc = B3_sc;
   p.b_sc_kchunks = (int)((long long)E * K / 128);
   p.C = static_cast<__nv_bfloat16*>(C);
-  CUtensorMap ma, mb, mb3;
-  MOE_TRY(make_map(&ma, A, eb, K, A_pad_max, 128 / eb, BM));
+  Maps m;
+  MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, BM));
   if (epilogue == MOE_EPI_NONE) {
     MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_fwd: N %% 256");
     p.n_tiles = N / BN;
     p.ldc = N;
-    MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    MOE_TRY(make_out_map(&m.c, C, N, A_pad_max));
+    m.b3 = m.c2 = m.in = m.a;
     const int max_tiles = (A_pad_max / BM) * p.n_tiles;
-    return mx ? launch<true, false, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
-              : launch<false, false, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
+    return mx ? launch<true, false, B_MN, EPI_STORE>(m, p, max_tiles, s)
+              : launch<false, false, B_MN, EPI_STORE>(m, p, max_tiles, s);
   }
   MOE_CHECK_ARG(epilogue == MOE_EPI_SWIGLU, "gemm_fwd: epilogue must be NONE or SWIGLU");
   MOE_CHECK_ARG(B3 && (!mx || B3_sc), "gemm_fwd: SWIGLU needs B3 (W3)");
@@ -594,11 +693,15 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   p.aux = static_cast<__nv_bfloat16*>(aux);
   p.ld_aux = 2LL * N;
   p.half = N;
-  MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
-  MOE_TRY(make_map(&mb3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  MOE_TRY(make_map(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  MOE_TRY(make_out_map(&m.c, C, N, A_pad_max));
+  if (aux) MOE_TRY(make_out_map(&m.c2, aux, 2ULL * N, A_pad_max));
+  else m.c2 = m.c;
+  m.in = m.a;
   const int max_tiles = (A_pad_max / BM) * p.n_tiles;
-  return mx ? launch<true, false, B_MN_DUAL_N, EPI_SWIGLU>(ma, mb, mb3, p, max_tiles, s)
-            : launch<false, false, B_MN_DUAL_N, EPI_SWIGLU>(ma, mb, mb3, p, max_tiles, s);
+  return mx ? launch<true, false, B_MN_DUAL_N, EPI_SWIGLU>(m, p, max_tiles, s)
+            : launch<false, false, B_MN_DUAL_N, EPI_SWIGLU>(m, p, max_tiles, s);
 }
 
 extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc,
@@ -632,9 +735,9 @@ extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uin
   p.b3_sc = B3_sc;
   p.b_sc_kchunks = N / 128;
   p.C = static_cast<__nv_bfloat16*>(dA);
-  CUtensorMap ma, mb, mb3;
-  MOE_TRY(make_map(&ma, dC, eb, Ktot, A_pad_max, 128 / eb, BM));
-  MOE_TRY(make_map(&mb, B, eb, N, (uint64_t)E * K, 128 / eb, BN));
+  Maps m;
+  MOE_TRY(make_map(&m.a, dC, eb, Ktot, A_pad_max, 128 / eb, BM));
+  MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, BN));
   const int max_tiles = (A_pad_max / BM) * p.n_tiles;
   if (epilogue == MOE_EPI_SWIGLU_BWD) {
     MOE_CHECK_ARG(aux != nullptr, "gemm_dgrad: SWIGLU_BWD needs aux = [H1|H3]");
@@ -642,17 +745,24 @@ extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uin
     p.ld_aux = 2LL * K;
     p.half = K;
     p.ldc = 2LL * K;
-    return mx ? launch<true, false, B_K, EPI_SWIGLU_BWD>(ma, mb, mb, p, max_tiles, s)
-              : launch<false, false, B_K, EPI_SWIGLU_BWD>(ma, mb, mb, p, max_tiles, s);
+    MOE_TRY(make_out_map(&m.c, dA, 2ULL * K, A_pad_max));
+    MOE_TRY(make_out_map(&m.in, aux, 2ULL * K, A_pad_max));
+    m.b3 = m.c2 = m.a;
+    return mx ? launch<true, false, B_K, EPI_SWIGLU_BWD>(m, p, max_tiles, s)
+              : launch<false, false, B_K, EPI_SWIGLU_BWD>(m, p, max_tiles, s);
   }
   MOE_CHECK_ARG(epilogue == MOE_EPI_NONE, "gemm_dgrad: epilogue must be NONE or SWIGLU_BWD");
   p.ldc = K;
-  if (!dual)
-    return mx ? launch<true, false, B_K, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
-              : launch<false, false, B_K, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
-  MOE_TRY(make_map(&mb3, B3, eb, N, (uint64_t)E * K, 128 / eb, BN));
-  return mx ? launch<true, false, B_K_DUAL_K, EPI_STORE>(ma, mb, mb3, p, max_tiles, s)
-            : launch<false, false, B_K_DUAL_K, EPI_STORE>(ma, mb, mb3, p, max_tiles, s);
+  MOE_TRY(make_out_map(&m.c, dA, K, A_pad_max));
+  m.c2 = m.in = m.a;
+  if (!dual) {
+    m.b3 = m.a;
+    return mx ? launch<true, false, B_K, EPI_STORE>(m, p, max_tiles, s)
+              : launch<false, false, B_K, EPI_STORE>(m, p, max_tiles, s);
+  }
+  MOE_TRY(make_map(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, BN));
+  return mx ? launch<true, false, B_K_DUAL_K, EPI_STORE>(m, p, max_tiles, s)
+            : launch<false, false, B_K_DUAL_K, EPI_STORE>(m, p, max_tiles, s);
 }
 
 extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc,
@@ -675,19 +785,24 @@ extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint
   p.wgrad = 1;
   p.m_tiles_w = K / BM;
   p.n_tiles = Ncols / BN;
+  p.k_out = K;
   p.a_sc = A_sc;
   p.a_sc_kchunks = A_pad_max / 128;
   p.b_sc = dC_sc;
   p.b_sc_kchunks = A_pad_max / 128;
   p.C = static_cast<__nv_bfloat16*>(dB);
   p.C2 = static_cast<__nv_bfloat16*>(dB3);
-  p.n_split = dB3 ? N : Ncols;
+  p.n_split = dB3 ? N : 0;
   p.ldc = N;
   p.c_expert_stride = (long long)K * N;
-  CUtensorMap ma, mb;
-  MOE_TRY(make_map(&ma, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
-  MOE_TRY(make_map(&mb, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  Maps m;
+  MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
+  MOE_TRY(make_map(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  MOE_TRY(make_out_map(&m.c, dB, N, (uint64_t)E * K));
+  if (dB3) MOE_TRY(make_out_map(&m.c2, dB3, N, (uint64_t)E * K));
+  else m.c2 = m.c;
+  m.b3 = m.in = m.a;
   const int max_tiles = E * p.m_tiles_w * p.n_tiles;
-  return mx ? launch<true, true, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s)
-            : launch<false, true, B_MN, EPI_STORE>(ma, mb, mb, p, max_tiles, s);
+  return mx ? launch<true, true, B_MN, EPI_STORE>(m, p, max_tiles, s)
+            : launch<false, true, B_MN, EPI_STORE>(m, p, max_tiles, s);
 }
