@@ -45,6 +45,8 @@ def _args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (a smaller case of the same layer, e.g. for ncu captures)")
     return ap.parse_args()
 
 
@@ -74,7 +76,7 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "20",
                  "-i", self.index], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -246,6 +248,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     cfg = moe_inputs.CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.with_(T=args.tokens)
     peaks, peak_kind = _peaks()
     inp = moe_inputs.make_layer_inputs(cfg, "cuda")
     layer = moe.MoELayer(T=cfg.T, d=cfg.d, E=cfg.E, k=cfg.k, F=cfg.F, W1=inp["W1"], W3=inp["W3"],

@@ -289,11 +289,16 @@ MOE_API moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst, cons
 
 /* Router weight gradient: dWr[i, e] = sum over the real rows r of group e
  * of x[src[r], i] * dl_rows[r]  (= x^T dL with dL nonzero only at the chosen
- * experts), fp32 [d, E].
+ * experts), fp32 [d, E].  Reduced per 128-row block of the permuted buffer,
+ * then per expert (fixed order, independent of the load skew).  ws: at
+ * least moe_router_wgrad_workspace_size(d, A_pad_max) bytes.  `offsets` is
+ * unused (kept for the call's symmetry with the other metadata users).
  */
+MOE_API size_t moe_router_wgrad_workspace_size(int d, int A_pad_max);
 MOE_API moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const float* dl_rows,
-                              const int32_t* offsets, const int32_t* poff, int T, int d, int E,
-                              float* dWr, moe_stream_t stream);
+                                      const int32_t* offsets, const int32_t* poff, int T, int d,
+                                      int E, int A_pad_max, float* dWr, void* ws,
+                                      size_t ws_bytes, moe_stream_t stream);
 
 /* --------------------------------------------------------------- layer
  * The whole layer: route -> permute -> GEMM1+SwiGLU -> GEMM2 -> combine, and

@@ -183,9 +183,12 @@ def moe_unpermute_sum(dXp, dst, *, topk_idx=None, dl=None, Wr=None, E: int = 0, 
 
 def moe_router_wgrad(x, meta: dict, dl_rows, E: int, *, stream=None):
     T, d = x.shape
+    A = meta["A_pad_max"]
     dWr = torch.empty((d, E), dtype=torch.float32, device=x.device)
+    ws_bytes = _lib.lib().moe_router_wgrad_workspace_size(d, A)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
     _lib.call("moe_router_wgrad", _p(x), _p(meta["src"]), _p(dl_rows), _p(meta["offsets"]),
-              _p(meta["poff"]), T, d, E, _p(dWr), _s(stream))
+              _p(meta["poff"]), T, d, E, A, _p(dWr), _p(ws), ws_bytes, _s(stream))
     return dWr
 
 

@@ -69,7 +69,8 @@ _SIGS = {
     "moe_combine_bwd": (I, [P, P, P, P, P, P, I, I, I, I, P, P, P, P, P]),
     "moe_unpermute_sum_workspace_size": (Z, [I, I]),
     "moe_unpermute_sum": (I, [P, P, P, P, P, I, I, I, I, P, P, Z, P]),
-    "moe_router_wgrad": (I, [P, P, P, P, P, I, I, I, P, P]),
+    "moe_router_wgrad_workspace_size": (Z, [I, I]),
+    "moe_router_wgrad": (I, [P, P, P, P, P, I, I, I, I, P, P, Z, P]),
     "moe_layer_ctx_bytes": (Z, [ctypes.POINTER(LayerDesc)]),
     "moe_layer_ctx_view": (I, [ctypes.POINTER(LayerDesc), P, ctypes.POINTER(CtxView)]),
     "moe_layer_fwd": (I, [ctypes.POINTER(LayerDesc), ctypes.POINTER(LayerWeights), P, P, P, Z, P, P]),

@@ -41,7 +41,8 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI_WARPS = 8;    // two per TMEM lane quarter, each half of the columns
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int CHUNK = 32;           // epilogue columns per staged box
 constexpr int BOX_BYTES = 32 * CHUNK * 2;   // 32 rows x 32 bf16
 constexpr int A_BYTES = BM * 128;   // 128-byte rows (64 bf16 or 128 fp8 of K)
@@ -54,13 +55,15 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2 };
 
 // pipeline depth and per-warp staging (boxes of 2 KB) for each epilogue,
-// within the 227 KB of shared memory per CTA: STORE double-buffers one box,
-// SwiGLU stages h / H1 / H3, the SwiGLU backward double-buffers H1/H3 pairs
+// within the 227 KB of shared memory per CTA: STORE uses one box per warp
+// with a 4-stage ring; SwiGLU stages h / H1 / H3; the SwiGLU backward
+// double-buffers H1/H3 pairs (both with a 3-stage ring)
 template <bool MX, int EPI> struct EpiCfg {
-  static constexpr int STAGES = (EPI == EPI_SWIGLU_BWD || (MX && EPI == EPI_SWIGLU)) ? 3 : 4;
-  static constexpr int STG = (EPI == EPI_STORE ? 2 : EPI == EPI_SWIGLU ? 3 : 4) * BOX_BYTES;
+  static constexpr int STAGES = EPI == EPI_STORE ? 4 : 3;
+  static constexpr int BOXES = EPI == EPI_STORE ? 1 : EPI == EPI_SWIGLU ? 3 : 4;
+  static constexpr int STG = BOXES * BOX_BYTES;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES +
-                                 (MX ? SFA_BYTES + SFB_BYTES : 0)) + 4 * STG;
+                                 (MX ? SFA_BYTES + SFB_BYTES : 0)) + NUM_EPI_WARPS * STG;
 };
 
 // byte offset of 16-byte chunk j of row r inside a [32 rows x 64 B] box
@@ -172,7 +175,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar, in_bar[4][2];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], drain_bar;
+  __shared__ __align__(8) uint64_t in_bar[NUM_EPI_WARPS][2];
   __shared__ uint32_t tmem_slot;
   __shared__ int poff_s[MAX_E + 1];
   __shared__ volatile int abort_flag;
@@ -182,7 +186,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* sA = smem;                                  // STAGES x A_BYTES
   uint8_t* sB = smem + STAGES * A_BYTES;               // STAGES x B_BYTES
   uint8_t* sSF = sB + STAGES * B_BYTES;                // STAGES x (SFA + SFB), MX only
-  uint8_t* sStg = sSF + (MX ? STAGES * (SFA_BYTES + SFB_BYTES) : 0);   // 4 x STG (epilogue)
+  uint8_t* sStg = sSF + (MX ? STAGES * (SFA_BYTES + SFB_BYTES) : 0);   // per-warp staging
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -195,10 +199,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], NUM_EPI_WARPS);
     }
     mbar_init(&drain_bar, 1);
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < NUM_EPI_WARPS; ++w) {
       mbar_init(&in_bar[w][0], 1);
       mbar_init(&in_bar[w][1], 1);
     }
@@ -378,9 +382,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int ew = warp - 2;                // epilogue warp 0..7
+    const int hc = ew >> 2;                 // which half of the tile's columns
     const int r = lane;                     // row inside the warp's 32-row box
-    uint8_t* stg = sStg + q * STG;          // this warp's staging boxes
-    uint32_t in_phase = 0;                  // bit i: parity of in_bar[q][i]
+    uint8_t* stg = sStg + ew * STG;         // this warp's staging boxes
+    uint32_t in_phase = 0;                  // bit i: parity of in_bar[ew][i]
     uint32_t in_pending = 0;                // bit i: a load into pair i not yet waited for (lane 0)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
@@ -394,10 +400,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       if constexpr (EPI == EPI_SWIGLU_BWD) {
         // H1/H3 chunk 0 does not depend on the accumulator: fetch it now
         if (lane == 0) {
+          const int c0 = t.nt * BN + hc * (BN / 2);
           bulk_wait_read<0>();
-          mbar_arrive_expect_tx(&in_bar[q][0], 2 * BOX_BYTES);
-          tma_load_2d(stg, &tmIn, &in_bar[q][0], t.nt * BN, y0);
-          tma_load_2d(stg + BOX_BYTES, &tmIn, &in_bar[q][0], p.half + t.nt * BN, y0);
+          mbar_arrive_expect_tx(&in_bar[ew][0], 2 * BOX_BYTES);
+          tma_load_2d(stg, &tmIn, &in_bar[ew][0], c0, y0);
+          tma_load_2d(stg + BOX_BYTES, &tmIn, &in_bar[ew][0], p.half + c0, y0);
           in_pending |= 1u;
         }
       }
@@ -414,7 +421,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         int x0 = n0;
         if (p.wgrad && p.n_split > 0 && n0 >= p.n_split) { map = &tmC2; x0 = n0 - p.n_split; }
 #pragma unroll 1
-        for (int c = 0; c < BN; c += CHUNK) {
+        for (int c = hc * (BN / 2); c < (hc + 1) * (BN / 2); c += CHUNK) {
           uint32_t v[32];
           if (!empty) {
             tmem_ld32(tbase + c, v);
@@ -423,8 +430,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          uint8_t* buf = stg + ((c / CHUNK) & 1) * BOX_BYTES;
-          if (lane == 0) bulk_wait_read<1>();    // the store that used `buf` has read it
+          uint8_t* buf = stg;
+          if (lane == 0) bulk_wait_read<0>();    // the previous store has read the box
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -447,7 +454,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         // columns [nt*128, nt*128 + 128)
         const int n0 = t.nt * (BN / 2);
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += CHUNK) {
+        for (int c = hc * (BN / 4); c < (hc + 1) * (BN / 4); c += CHUNK) {
           uint32_t g[32], u[32];
           tmem_ld32(tbase + c, g);
           tmem_ld32(tbase + BN / 2 + c, u);
@@ -486,8 +493,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       } else {  // EPI_SWIGLU_BWD: accumulator = dh for columns [nt*256, +256)
-        const int n0 = t.nt * BN;
-        constexpr int NCH = BN / CHUNK;
+        const int n0 = t.nt * BN + hc * (BN / 2);
+        constexpr int NCH = BN / 2 / CHUNK;
 #pragma unroll 1
         for (int ci = 0; ci < NCH; ++ci) {
           const int c = ci * CHUNK;
@@ -497,17 +504,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (ci + 1 < NCH && lane == 0) {            // prefetch the next chunk's H1/H3
             uint8_t* n1 = stg + (pr ^ 1) * 2 * BOX_BYTES;
             bulk_wait_read<0>();                      // its pair's previous stores have read it
-            mbar_arrive_expect_tx(&in_bar[q][pr ^ 1], 2 * BOX_BYTES);
-            tma_load_2d(n1, &tmIn, &in_bar[q][pr ^ 1], n0 + c + CHUNK, y0);
-            tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[q][pr ^ 1], p.half + n0 + c + CHUNK, y0);
+            mbar_arrive_expect_tx(&in_bar[ew][pr ^ 1], 2 * BOX_BYTES);
+            tma_load_2d(n1, &tmIn, &in_bar[ew][pr ^ 1], n0 + c + CHUNK, y0);
+            tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[ew][pr ^ 1], p.half + n0 + c + CHUNK, y0);
             in_pending |= 1u << (pr ^ 1);
           }
           uint32_t v[32];
-          tmem_ld32(tbase + c, v);
+          tmem_ld32(tbase + hc * (BN / 2) + c, v);
           tmem_wait_ld();
           int got = 1;
           if (lane == 0)
-            got = mbar_wait(&in_bar[q][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
+            got = mbar_wait(&in_bar[ew][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
                             kWaitLimitNs);
           got = __shfl_sync(0xffffffffu, got, 0);
           if (got) {
@@ -552,7 +559,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         volatile int no_abort = 0;
         for (int i = 0; i < 2; ++i)
           if (in_pending & (1u << i))
-            mbar_wait(&in_bar[q][i], (in_phase >> i) & 1, &no_abort, p.status, kWaitLimitNs);
+            mbar_wait(&in_bar[ew][i], (in_phase >> i) & 1, &no_abort, p.status, kWaitLimitNs);
       }
     }
   }

@@ -82,7 +82,9 @@ size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   }
   const size_t ws_route = moe_route_workspace_size(L->T, L->E);
   const size_t ws_unperm = moe_unpermute_sum_workspace_size(L->d, L->E);
+  const size_t ws_rw = moe_router_wgrad_workspace_size(L->d, (int)A);
   x.ws_bytes = ws_route > ws_unperm ? ws_route : ws_unperm;
+  if (ws_rw > x.ws_bytes) x.ws_bytes = ws_rw;
   x.ws = l.take<uint8_t>(x.ws_bytes);
   if (v) *v = x;
   return moe::round_up(l.off, 256);
@@ -293,7 +295,8 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   mark(S_UNPERMUTE, true, s);
   if (router && G->dWr) {
     mark(S_ROUTER_WGRAD, false, s);
-    MOE_TRY(moe_router_wgrad(x, c.src, c.dl_rows, c.offsets, c.poff, T, d, E, G->dWr, stream));
+    MOE_TRY(moe_router_wgrad(x, c.src, c.dl_rows, c.offsets, c.poff, T, d, E, A, G->dWr, c.ws,
+                             c.ws_bytes, stream));
     mark(S_ROUTER_WGRAD, true, s);
   }
   return MOE_OK;

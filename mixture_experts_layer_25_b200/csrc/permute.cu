@@ -4,13 +4,24 @@
 // Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ, section
 // "ルーティングと計算の最適化": routed tokens are written straight into the
 // experts' input buffers.  Every kernel moves whole token rows with 16-byte
-// vector accesses, one warp per token, each row read once.
+// vector accesses, each row read once.
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int kMaxK = 16;
-constexpr int kWarpsPerBlock = 8;
+constexpr int kTopKLimit = 16;
+
+// call f(std::integral_constant<int, KM>) with the smallest KM in
+// {2, 4, 8, 16} >= k: the kernels keep k rows' state in register arrays
+template <class F>
+void dispatch_k(int k, F&& f) {
+  if (k <= 2) f(std::integral_constant<int, 2>{});
+  else if (k <= 4) f(std::integral_constant<int, 4>{});
+  else if (k <= 8) f(std::integral_constant<int, 8>{});
+  else f(std::integral_constant<int, 16>{});
+}
 
 // zero the pad rows [poff[e] + counts[e], poff[e+1]) of one expert group
 __device__ __forceinline__ void zero_pad_rows(const int32_t* offsets, const int32_t* poff, int e,
@@ -23,8 +34,19 @@ __device__ __forceinline__ void zero_pad_rows(const int32_t* offsets, const int3
   for (size_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = z;
 }
 
+// Row teams: `tpt` threads (a multiple of 32, at most 256) share one token
+// row, each moving 16-byte chunks lt, lt + tpt, ...; a 256-thread block holds
+// 256 / tpt tokens.  With d = 2048 a whole block works on one row, so every
+// load of the row is in flight at once.
+constexpr int kBlock = 256;
+
+__host__ __device__ __forceinline__ int team_threads(int d8) {
+  return d8 >= kBlock ? kBlock : ((d8 + 31) / 32) * 32;
+}
+
 // ------------------------------------------------------------------ permute
-__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock)
 permute_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
                const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
                int k, int d8, int tok_blocks, uint4* __restrict__ Xp) {
@@ -32,35 +54,31 @@ permute_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
     zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, Xp);
     return;
   }
-  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int tpt = team_threads(d8);
+  const int t = blockIdx.x * (kBlock / tpt) + threadIdx.x / tpt;
+  const int lt = threadIdx.x % tpt;
   if (t >= T) return;
   int r[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) r[j] = j < k ? dst[(size_t)t * k + j] : -1;
   const uint4* xr = x + (size_t)t * d8;
-  for (int c0 = lane; c0 < d8; c0 += 32 * 4) {
-    uint4 v[4];
+#pragma unroll 2
+  for (int c = lt; c < d8; c += tpt) {
+    const uint4 v = ldg_stream(xr + c);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (c0 + 32 * u < d8) v[u] = ldg_stream(xr + c0 + 32 * u);
-#pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (r[j] < 0) continue;
-      uint4* o = Xp + (size_t)r[j] * d8;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (c0 + 32 * u < d8) o[c0 + 32 * u] = v[u];
-    }
+    for (int j = 0; j < kMaxK; ++j)
+      if (r[j] >= 0) Xp[(size_t)r[j] * d8 + c] = v;
   }
 }
 
 // ------------------------------------------------------------------ combine
-__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock)
 combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ gates,
                const int32_t* __restrict__ dst, int T, int k, int d8, uint4* __restrict__ out) {
-  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int tpt = team_threads(d8);
+  const int t = blockIdx.x * (kBlock / tpt) + threadIdx.x / tpt;
+  const int lt = threadIdx.x % tpt;
   if (t >= T) return;
   int r[kMaxK];
   float g[kMaxK];
@@ -69,13 +87,18 @@ combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ gates,
     r[j] = j < k ? dst[(size_t)t * k + j] : -1;
     g[j] = (j < k && gates) ? gates[(size_t)t * k + j] : 1.f;
   }
-  for (int c = lane; c < d8; c += 32) {
+#pragma unroll 2
+  for (int c = lt; c < d8; c += tpt) {
+    uint4 v[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (r[j] >= 0) v[j] = ldg_stream(Y + (size_t)r[j] * d8 + c);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (r[j] < 0) continue;
       float f[8];
-      unpack8(ldg_stream(Y + (size_t)r[j] * d8 + c), f);
+      unpack8(v[j], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
     }
@@ -84,7 +107,8 @@ combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ gates,
 }
 
 // ------------------------------------------------------- combine backward
-__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock)
 combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
                    const float* __restrict__ gates, const int32_t* __restrict__ dst,
                    const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
@@ -94,52 +118,74 @@ combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
     zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY);
     return;
   }
-  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
+  __shared__ float red[kBlock / 32][kMaxK];
+  const int tpt = team_threads(d8);
+  const int t = blockIdx.x * (kBlock / tpt) + threadIdx.x / tpt;
+  const int lt = threadIdx.x % tpt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool live = t < T;
   int r[kMaxK];
   float g[kMaxK], dot[kMaxK];
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j) {
-    r[j] = j < k ? dst[(size_t)t * k + j] : -1;
-    g[j] = j < k ? gates[(size_t)t * k + j] : 0.f;
+    r[j] = (live && j < k) ? dst[(size_t)t * k + j] : -1;
+    g[j] = (live && j < k) ? gates[(size_t)t * k + j] : 0.f;
     dot[j] = 0.f;
   }
-  for (int c = lane; c < d8; c += 32) {
-    float fd[8];
-    unpack8(ldg_stream(dout + (size_t)t * d8 + c), fd);
+  if (live) {
+#pragma unroll 2
+    for (int c = lt; c < d8; c += tpt) {
+      const uint4 dv = ldg_stream(dout + (size_t)t * d8 + c);
+      uint4 yv[kMaxK];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (r[j] < 0) continue;
-      float fy[8], sc[8];
-      unpack8(ldg_stream(Y + (size_t)r[j] * d8 + c), fy);
-      float s = 0.f;
+      for (int j = 0; j < kMaxK; ++j)
+        if (r[j] >= 0) yv[j] = ldg_stream(Y + (size_t)r[j] * d8 + c);
+      float fd[8];
+      unpack8(dv, fd);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        s = fmaf(fd[i], fy[i], s);
-        sc[i] = g[j] * fd[i];
+      for (int j = 0; j < kMaxK; ++j) {
+        if (r[j] < 0) continue;
+        float fy[8], sc[8];
+        unpack8(yv[j], fy);
+        float sdot = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          sdot = fmaf(fd[i], fy[i], sdot);
+          sc[i] = g[j] * fd[i];
+        }
+        dot[j] += sdot;
+        dY[(size_t)r[j] * d8 + c] = pack8(sc);
       }
-      dot[j] += s;
-      dY[(size_t)r[j] * d8 + c] = pack8(sc);
     }
   }
+  // team reduction of the k dot products: warps, then the team's warps
 #pragma unroll
   for (int j = 0; j < kMaxK; ++j)
     if (j < k) dot[j] = warp_sum(dot[j]);
-  if (lane == 0) {
-    float gs = 0.f;
+  if (lane == 0)
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j)
-      if (j < k) gs = fmaf(g[j], dot[j], gs);
+      if (j < k) red[warp][j] = dot[j];
+  __syncthreads();
+  if (!live || lt != 0) return;
+  const int w0 = warp, nw = tpt / 32;
+  float gs = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      if (j >= k) continue;
-      dg[(size_t)t * k + j] = dot[j];
-      if (dl) {
-        const float v = g[j] * (dot[j] - gs);
-        dl[(size_t)t * k + j] = v;
-        if (dl_rows && r[j] >= 0) dl_rows[r[j]] = v;
-      }
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j >= k) continue;
+    float s = 0.f;
+    for (int w = 0; w < nw; ++w) s += red[w0 + w][j];
+    dot[j] = s;
+    gs = fmaf(g[j], s, gs);
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxK; ++j) {
+    if (j >= k) continue;
+    dg[(size_t)t * k + j] = dot[j];
+    if (dl) {
+      const float v = g[j] * (dot[j] - gs);
+      dl[(size_t)t * k + j] = v;
+      if (dl_rows && r[j] >= 0) dl_rows[r[j]] = v;
     }
   }
 }
@@ -160,13 +206,15 @@ __global__ void transpose_f32_kernel(const float* __restrict__ in, int rows, int
   }
 }
 
-__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock)
 unpermute_sum_kernel(const uint4* __restrict__ dXp, const int32_t* __restrict__ dst,
                      const int32_t* __restrict__ topk_idx, const float* __restrict__ dl,
                      const float* __restrict__ WrT /* [E,d] or null */, int T, int k, int d8,
                      int E, uint4* __restrict__ dx) {
-  const int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  const int tpt = team_threads(d8);
+  const int t = blockIdx.x * (kBlock / tpt) + threadIdx.x / tpt;
+  const int lt = threadIdx.x % tpt;
   if (t >= T) return;
   int r[kMaxK], e[kMaxK];
   float w[kMaxK];
@@ -175,23 +223,29 @@ unpermute_sum_kernel(const uint4* __restrict__ dXp, const int32_t* __restrict__ 
     r[j] = j < k ? dst[(size_t)t * k + j] : -1;
     e[j] = (j < k && WrT) ? topk_idx[(size_t)t * k + j] : -1;
     w[j] = (j < k && WrT) ? dl[(size_t)t * k + j] : 0.f;
+    if (e[j] >= E) e[j] = -1;
   }
-  for (int c = lane; c < d8; c += 32) {
+#pragma unroll 2
+  for (int c = lt; c < d8; c += tpt) {
+    uint4 v[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (r[j] >= 0) v[j] = ldg_stream(dXp + (size_t)r[j] * d8 + c);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) {
       if (r[j] < 0) continue;
       float f[8];
-      unpack8(ldg_stream(dXp + (size_t)r[j] * d8 + c), f);
+      unpack8(v[j], f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += f[i];
     }
     if (WrT) {
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
-        if (r[j] < 0 || e[j] < 0 || e[j] >= E) continue;
+        if (r[j] < 0 || e[j] < 0) continue;
         const float4* wr = reinterpret_cast<const float4*>(WrT + (size_t)e[j] * d8 * 8) + 2 * c;
-        const float4 a = wr[0], b = wr[1];
+        const float4 a = __ldg(wr), b = __ldg(wr + 1);
         acc[0] = fmaf(w[j], a.x, acc[0]); acc[1] = fmaf(w[j], a.y, acc[1]);
         acc[2] = fmaf(w[j], a.z, acc[2]); acc[3] = fmaf(w[j], a.w, acc[3]);
         acc[4] = fmaf(w[j], b.x, acc[4]); acc[5] = fmaf(w[j], b.y, acc[5]);
@@ -203,22 +257,28 @@ unpermute_sum_kernel(const uint4* __restrict__ dXp, const int32_t* __restrict__ 
 }
 
 // --------------------------------------------------------- router wgrad
-// dWr[i, e] = sum over the real rows r of group e of x[src[r], i] * dl_rows[r]
+// dWr[i, e] = sum over the real rows r of group e of x[src[r], i] * dl_rows[r].
+// Pass 1: every 128-row block of the permuted buffer (one expert's rows, as
+// groups start on multiples of 128) sums its rows into P[block][:]; pass 2
+// adds the blocks of each expert.  Work spreads evenly however skewed the
+// load, and the summation order is fixed.
 constexpr int kRwRowGroups = 8;
 __global__ void __launch_bounds__(256)
-router_wgrad_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ src,
-                    const float* __restrict__ dl_rows, const int32_t* __restrict__ offsets,
-                    const int32_t* __restrict__ poff, int d8, int E, float* __restrict__ dWr) {
+router_wgrad_blocks_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ src,
+                           const float* __restrict__ dl_rows, const int32_t* __restrict__ poff,
+                           int E, int d8, float* __restrict__ P) {
   __shared__ float red[kRwRowGroups][256 + 4];
-  const int e = blockIdx.x;
+  const int blk = blockIdx.x;
+  if (blk * 128 >= poff[E]) return;
   const int rg = threadIdx.x >> 5, cl = threadIdx.x & 31;
   const int c = blockIdx.y * 32 + cl;       // 8-column chunk index
-  const int r0 = poff[e], n = offsets[e + 1] - offsets[e];
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (c < d8) {
-    for (int i = rg; i < n; i += kRwRowGroups) {
-      const int r = r0 + i;
+#pragma unroll 4
+    for (int i = rg; i < 128; i += kRwRowGroups) {
+      const int r = blk * 128 + i;
       const int t = src[r];
+      if (t < 0) continue;                  // pad row
       const float w = dl_rows[r];
       float f[8];
       unpack8(x[(size_t)t * d8 + c], f);
@@ -231,11 +291,22 @@ router_wgrad_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ src
   __syncthreads();
   const int col = blockIdx.y * 256 + threadIdx.x;
   if (col < d8 * 8) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int g = 0; g < kRwRowGroups; ++g) s += red[g][threadIdx.x];
-    dWr[(size_t)col * E + e] = s;
+    for (int g = 0; g < kRwRowGroups; ++g) sum += red[g][threadIdx.x];
+    P[(size_t)blk * d8 * 8 + col] = sum;
   }
+}
+
+__global__ void __launch_bounds__(256)
+router_wgrad_reduce_kernel(const float* __restrict__ P, const int32_t* __restrict__ poff, int E,
+                           int d, float* __restrict__ dWr) {
+  const int e = blockIdx.x;
+  const int col = blockIdx.y * 256 + threadIdx.x;
+  if (col >= d) return;
+  float sum = 0.f;
+  for (int b = poff[e] / 128; b < poff[e + 1] / 128; ++b) sum += P[(size_t)b * d + col];
+  dWr[(size_t)col * E + e] = sum;
 }
 
 }  // namespace moe
@@ -256,17 +327,19 @@ extern "C" moe_status_t moe_permute(const void* x, const int32_t* dst, const int
                                     int A_pad_max, void* Xp, uint8_t* Xq, uint8_t* Xs,
                                     moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && E > 0 && d > 0 && d % 8 == 0,
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kTopKLimit && E > 0 && d > 0 && d % 8 == 0,
                 "moe_permute: bad T/k/E/d");
   MOE_CHECK_ARG(x && dst && offsets && poff && Xp && aligned16(x) && aligned16(Xp),
                 "moe_permute: null or unaligned pointer");
   MOE_CHECK_ARG((Xq == nullptr) == (Xs == nullptr), "moe_permute: Xq and Xs go together");
   (void)A_pad_max;
   if (Xq) return moe_permute_mx_launch(x, dst, offsets, poff, T, k, d, E, A_pad_max, Xp, Xq, Xs, s);
-  const int tok_blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  permute_kernel<<<tok_blocks + E, 32 * kWarpsPerBlock, 0, s>>>(
-      static_cast<const uint4*>(x), dst, offsets, poff, T, k, d / 8, tok_blocks,
+  const int tpb = kBlock / team_threads(d / 8);
+  const int tok_blocks = (T + tpb - 1) / tpb;
+  dispatch_k(k, [&](auto KM) {
+    permute_kernel<decltype(KM)::value><<<tok_blocks + E, kBlock, 0, s>>>(static_cast<const uint4*>(x), dst, offsets, poff, T, k, d / 8, tok_blocks,
       static_cast<uint4*>(Xp));
+  });
   MOE_CHECK_LAUNCH("permute");
   return MOE_OK;
 }
@@ -275,12 +348,15 @@ extern "C" moe_status_t moe_unpermute_combine(const void* Y, const float* gates,
                                               const int32_t* dst, int T, int k, int d, void* out,
                                               moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && d > 0 && d % 8 == 0, "moe_unpermute_combine: bad sizes");
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kTopKLimit && d > 0 && d % 8 == 0, "moe_unpermute_combine: bad sizes");
   MOE_CHECK_ARG(Y && dst && out && aligned16(Y) && aligned16(out),
                 "moe_unpermute_combine: null or unaligned pointer");
-  const int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  combine_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(static_cast<const uint4*>(Y), gates, dst,
+  const int tpb = kBlock / team_threads(d / 8);
+  const int blocks = (T + tpb - 1) / tpb;
+  dispatch_k(k, [&](auto KM) {
+    combine_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(Y), gates, dst,
                                                         T, k, d / 8, static_cast<uint4*>(out));
+  });
   MOE_CHECK_LAUNCH("combine");
   return MOE_OK;
 }
@@ -291,15 +367,17 @@ extern "C" moe_status_t moe_combine_bwd(const void* dout, const void* Y, const f
                                         float* dg, float* dl, float* dl_rows,
                                         moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && E > 0 && d > 0 && d % 8 == 0,
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kTopKLimit && E > 0 && d > 0 && d % 8 == 0,
                 "moe_combine_bwd: bad sizes");
   MOE_CHECK_ARG(dout && Y && gates && dst && offsets && poff && dY && dg,
                 "moe_combine_bwd: null pointer");
   MOE_CHECK_ARG(aligned16(dout) && aligned16(Y) && aligned16(dY), "moe_combine_bwd: unaligned");
-  const int tok_blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  combine_bwd_kernel<<<tok_blocks + E, 32 * kWarpsPerBlock, 0, s>>>(
-      static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff, T,
+  const int tpb = kBlock / team_threads(d / 8);
+  const int tok_blocks = (T + tpb - 1) / tpb;
+  dispatch_k(k, [&](auto KM) {
+    combine_bwd_kernel<decltype(KM)::value><<<tok_blocks + E, kBlock, 0, s>>>(static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff, T,
       k, d / 8, tok_blocks, static_cast<uint4*>(dY), dg, dl, dl_rows);
+  });
   MOE_CHECK_LAUNCH("combine_bwd");
   return MOE_OK;
 }
@@ -314,7 +392,7 @@ extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
                                           const float* Wr, int T, int k, int d, int E, void* dx,
                                           void* ws, size_t ws_bytes, moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kMaxK && d > 0 && d % 8 == 0 && E > 0,
+  MOE_CHECK_ARG(T > 0 && k > 0 && k <= kTopKLimit && d > 0 && d % 8 == 0 && E > 0,
                 "moe_unpermute_sum: bad sizes");
   MOE_CHECK_ARG(dXp && dst && dx && aligned16(dXp) && aligned16(dx),
                 "moe_unpermute_sum: null or unaligned pointer");
@@ -332,24 +410,43 @@ extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
     transpose_f32_kernel<<<grid, block, 0, s>>>(Wr, d, E, WrT);
     MOE_CHECK_LAUNCH("transpose Wr");
   }
-  const int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  unpermute_sum_kernel<<<blocks, 32 * kWarpsPerBlock, 0, s>>>(
-      static_cast<const uint4*>(dXp), dst, topk_idx, dl, WrT, T, k, d / 8, E,
+  const int tpb = kBlock / team_threads(d / 8);
+  const int blocks = (T + tpb - 1) / tpb;
+  dispatch_k(k, [&](auto KM) {
+    unpermute_sum_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(dXp), dst, topk_idx, dl, WrT, T, k, d / 8, E,
       static_cast<uint4*>(dx));
+  });
   MOE_CHECK_LAUNCH("unpermute_sum");
   return MOE_OK;
 }
 
+extern "C" size_t moe_router_wgrad_workspace_size(int d, int A_pad_max) {
+  if (d <= 0 || A_pad_max <= 0) return 0;
+  return round_up((size_t)((A_pad_max + 127) / 128) * d * sizeof(float), 256);
+}
+
 extern "C" moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const float* dl_rows,
                                          const int32_t* offsets, const int32_t* poff, int T,
-                                         int d, int E, float* dWr, moe_stream_t stream) {
+                                         int d, int E, int A_pad_max, float* dWr, void* ws,
+                                         size_t ws_bytes, moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && d > 0 && d % 8 == 0 && E > 0, "moe_router_wgrad: bad sizes");
-  MOE_CHECK_ARG(x && src && dl_rows && offsets && poff && dWr && aligned16(x),
+  (void)offsets;
+  MOE_CHECK_ARG(T > 0 && d > 0 && d % 8 == 0 && E > 0 && A_pad_max > 0,
+                "moe_router_wgrad: bad sizes");
+  MOE_CHECK_ARG(x && src && dl_rows && poff && dWr && aligned16(x),
                 "moe_router_wgrad: null or unaligned pointer");
-  dim3 grid(E, (d + 255) / 256);
-  router_wgrad_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), src, dl_rows, offsets,
-                                           poff, d / 8, E, dWr);
-  MOE_CHECK_LAUNCH("router_wgrad");
+  const size_t need = moe_router_wgrad_workspace_size(d, A_pad_max);
+  if (!ws || ws_bytes < need) {
+    set_error("moe_router_wgrad: workspace %zu < %zu bytes", ws_bytes, need);
+    return MOE_ERR_WORKSPACE;
+  }
+  float* P = static_cast<float*>(ws);
+  dim3 g1((A_pad_max + 127) / 128, (d + 255) / 256);
+  router_wgrad_blocks_kernel<<<g1, 256, 0, s>>>(static_cast<const uint4*>(x), src, dl_rows, poff,
+                                                E, d / 8, P);
+  MOE_CHECK_LAUNCH("router_wgrad_blocks");
+  dim3 g2(E, (d + 255) / 256);
+  router_wgrad_reduce_kernel<<<g2, 256, 0, s>>>(P, poff, E, d, dWr);
+  MOE_CHECK_LAUNCH("router_wgrad_reduce");
   return MOE_OK;
 }
