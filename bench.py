@@ -39,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="olmo128", choices=sorted(moe_inputs.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -285,6 +285,7 @@ def run_ours(args):
     smi_index = vis.split(",")[local] if vis else str(local)
     clocks = ClockSampler(smi_index)
     clocks.start()
+    time.sleep(0.5)          # let the sampler take its first readings before the timed region
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     _barrier(world)

@@ -134,7 +134,10 @@ MOE_API void moe_set_stage_events(void* const* events, int n);
  *
  * mode MOE_ROUTE_ROUTER: logits = x W_r (+ bias) in fp32, top-k (ties to the
  *   lower index, slot j = j-th largest), gates = softmax of the k chosen
- *   logits (fp32); writes topk_idx [T,k] and gates [T,k].
+ *   logits (fp32); writes topk_idx [T,k] and gates [T,k].  With E <= 256,
+ *   E % 8 == 0, k <= 8 and d % 64 == 0 the logits run on the tensor cores:
+ *   W_r is split exactly into three bf16 parts (w0 + w1 + w2 = W_r, each
+ *   product exact) accumulated in fp32; otherwise fp32 FMA on CUDA cores.
  * mode MOE_ROUTE_GIVEN: topk_idx and gates are INPUTS (random-routing stress
  *   workload, [OC3-ja] "実証されたスケール"); x and W_r are not read.  An index
  *   outside [0,E) or a repeat inside a token sets MOE_DEV_BAD_EXPERT /
@@ -143,9 +146,10 @@ MOE_API void moe_set_stage_events(void* const* events, int n);
  *   logits: optional [T,E] fp32 copy of the router logits (ROUTER mode).
  *   align must be 128.  Router mode needs E <= 512, k <= min(E, 16),
  *   d % 8 == 0; given mode E <= 4096.
- *   ws: device workspace of at least moe_route_workspace_size(T, E) bytes.
+ *   ws: 256-byte aligned device workspace of at least
+ *   moe_route_workspace_size(T, d, E) bytes (pass d = 0 for given mode).
  */
-MOE_API size_t moe_route_workspace_size(int T, int E);
+MOE_API size_t moe_route_workspace_size(int T, int d, int E);
 MOE_API moe_status_t moe_route(const void* x, const float* Wr, const float* bias, int T, int d,
                        int E, int k, int align, int mode, int32_t* topk_idx, float* gates,
                        int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* dst,
@@ -160,9 +164,10 @@ MOE_API moe_status_t moe_route(const void* x, const float* Wr, const float* bias
  * convenience.  Its scratch is a fixed, library-owned array in device memory
  * of MOE_ROUTE_NOALLOC_MAX_SCRATCH_BYTES (4 MiB) on every device that loads
  * the library, kept until the process exits; the caller still passes all
- * inputs and outputs.  Limit: moe_route_workspace_size(T, E) =
- * ceil(T/32)*E*4 bytes must fit (e.g. T <= 262144 with E = 128); larger
- * sizes return MOE_ERR_INVALID_ARG.  The first call on a device looks up the
+ * inputs and outputs.  Limit: moe_route_workspace_size(T, d, E) (d = 0 in
+ * given mode) must fit, e.g. T = 65536, d = 2048, E = 128 in router mode or
+ * T <= 262144 with E = 128 in given mode; larger sizes return
+ * MOE_ERR_INVALID_ARG.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress), so make that first call
  * before any stream capture.  All calls share the one array: calls that
  * overlap on the GPU (other streams, other host threads) race and must be

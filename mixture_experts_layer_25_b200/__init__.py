@@ -69,7 +69,7 @@ def moe_route(x, Wr, bias, k: int, E: int, *, topk_idx=None, gates=None, align: 
         "src": torch.empty(A, **i32), "A_pad_max": A,
         "logits": torch.empty((T, E), **f32) if (want_logits and not given) else None,
     }
-    ws_bytes = _lib.lib().moe_route_workspace_size(T, E)
+    ws_bytes = _lib.lib().moe_route_workspace_size(T, 0 if given else d, E)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     _lib.call("moe_route", _p(x), _p(Wr), _p(bias), T, d, E, k, align,
               _lib.MOE_ROUTE_GIVEN if given else _lib.MOE_ROUTE_ROUTER,

@@ -57,7 +57,7 @@ _SIGS = {
     "moe_version": (ctypes.c_char_p, []),
     "moe_launch_count": (ctypes.c_ulonglong, []),
     "moe_set_stage_events": (None, [ctypes.POINTER(P), I]),
-    "moe_route_workspace_size": (Z, [I, I]),
+    "moe_route_workspace_size": (Z, [I, I, I]),
     "moe_route": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, Z, P, P]),
     "moe_route_noalloc": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P]),
     "moe_permute": (I, [P, P, P, P, I, I, I, I, I, P, P, P, P]),

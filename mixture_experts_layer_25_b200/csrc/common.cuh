@@ -41,6 +41,12 @@ void count_launch();
     if (s_ != MOE_OK) return s_;              \
   } while (0)
 
+// tensor-core router (grouped_gemm.cu): logits, top-k (k <= 8), gates,
+// in-block ranks and per-128-token-block histograms
+moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int T, int d, int E,
+                       int k, float* logits, int32_t* topk, float* gates, int32_t* rank,
+                       int32_t* hist, int32_t* status, cudaStream_t s);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int num_sms();

@@ -52,15 +52,15 @@ constexpr int SFB_BYTES = 1024;     // 256 rows x 4 scale bytes
 constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
-enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2 };
+enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3 };
 
 // pipeline depth and per-warp staging (boxes of 2 KB) for each epilogue,
 // within the 227 KB of shared memory per CTA: STORE uses one box per warp
 // with a 4-stage ring; SwiGLU stages h / H1 / H3; the SwiGLU backward
 // double-buffers H1/H3 pairs (both with a 3-stage ring)
 template <bool MX, int EPI> struct EpiCfg {
-  static constexpr int STAGES = EPI == EPI_STORE ? 4 : 3;
-  static constexpr int BOXES = EPI == EPI_STORE ? 1 : EPI == EPI_SWIGLU ? 3 : 4;
+  static constexpr int STAGES = (EPI == EPI_STORE || EPI == EPI_ROUTER) ? 4 : 3;
+  static constexpr int BOXES = (EPI == EPI_STORE || EPI == EPI_ROUTER) ? 1 : EPI == EPI_SWIGLU ? 3 : 4;
   static constexpr int STG = BOXES * BOX_BYTES;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES +
                                  (MX ? SFA_BYTES + SFB_BYTES : 0)) + NUM_EPI_WARPS * STG;
@@ -91,6 +91,14 @@ struct Params {
   __nv_bfloat16* aux; long long ld_aux; int half;
   long long c_expert_stride;
   int k_out;          // wgrad: output rows per expert (K of the weight)
+  // dense single-group mode (router): rows [0, dense_rows), no poff
+  int dense_rows;
+  int a_k_wrap;       // > 0: A's K coordinate wraps modulo a_k_wrap
+  int mma_n;          // > 0: MMA N (multiple of 16, <= 256) instead of BN
+  int b_boxes;        // > 0: MN-major B boxes loaded per stage (<= BN / chunk)
+  // router epilogue
+  const float* r_bias; float* r_logits; int32_t* r_topk; float* r_gates;
+  int32_t* r_rank; int32_t* r_hist; int r_k; int r_E;
   int32_t* status;
 };
 
@@ -113,7 +121,7 @@ __device__ __forceinline__ Tile decode(const Params& p, const int* poff_s, int t
     const int mt = tile / p.n_tiles;
     t.nt = tile - mt * p.n_tiles;
     t.row0 = mt * BM;
-    t.e = find_expert(poff_s, p.E, t.row0);
+    t.e = p.dense_rows ? 0 : find_expert(poff_s, p.E, t.row0);
     t.m0 = t.row0;
     t.nkb = p.num_kb;
     t.krow0 = 0;
@@ -132,6 +140,11 @@ __device__ __forceinline__ Tile decode(const Params& p, const int* poff_s, int t
 }
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) { return pack2(a, b); }
+
+// barrier over a subset of the CTA's warps (id 0 is __syncthreads')
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
@@ -190,7 +203,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) poff_s[i] = p.poff[i];
+  if (!p.dense_rows)
+    for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) poff_s[i] = p.poff[i];
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
@@ -225,7 +239,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
 
-  const int total = p.wgrad ? p.E * p.m_tiles_w * p.n_tiles : (poff_s[p.E] / BM) * p.n_tiles;
+  const int total = p.wgrad ? p.E * p.m_tiles_w * p.n_tiles
+                  : p.dense_rows ? ((p.dense_rows + BM - 1) / BM) * p.n_tiles
+                                 : (poff_s[p.E] / BM) * p.n_tiles;
   auto group_kb = [&](const Tile& t) {
     return p.wgrad ? (poff_s[t.e + 1] - poff_s[t.e]) / BK : t.nkb;
   };
@@ -243,12 +259,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
           uint64_t* fb = &full_bar[stage];
-          mbar_arrive_expect_tx(fb, STAGE_TX);
+          const int nbox = p.b_boxes ? p.b_boxes : BN / MN_CHUNK;
+          mbar_arrive_expect_tx(fb, B_MNMAJOR ? STAGE_TX - (BN / MN_CHUNK - nbox) * MN_CHUNK_BYTES
+                                              : STAGE_TX);
           uint8_t* a_dst = sA + stage * A_BYTES;
           uint8_t* b_dst = sB + stage * B_BYTES;
           // A operand
           if constexpr (!A_MN) {
-            tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
+            tma_load_2d(a_dst, &tmA, fb, p.a_k_wrap ? (kb * BK) % p.a_k_wrap : kb * BK, t.row0);
           } else {
 #pragma unroll
             for (int i = 0; i < BM / MN_CHUNK; ++i)
@@ -259,7 +277,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
           if constexpr (BLOAD == B_MN) {
 #pragma unroll
-            for (int i = 0; i < BN / MN_CHUNK; ++i)
+            for (int i = 0; i < nbox; ++i)
               tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * BN + i * MN_CHUNK,
                           brow + kb * BK);
           } else if constexpr (BLOAD == B_MN_DUAL_N) {
@@ -323,6 +341,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // ------------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t IDESC = make_idesc<MX>(A_MN, B_MNMAJOR);
+      const uint32_t idesc =
+          p.mma_n ? (IDESC & ~(0x3Fu << 17)) | ((uint32_t)(p.mma_n >> 3) << 17) : IDESC;
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -361,9 +381,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             else bd = smem_desc(sb + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
             const uint32_t accum = (kb > 0 || ks > 0) ? 1u : 0u;
             if constexpr (!MX) {
-              mma_bf16(d_tmem, ad, bd, IDESC, accum);
+              mma_bf16(d_tmem, ad, bd, idesc, accum);
             } else {
-              const uint32_t id = IDESC | ((uint32_t)ks << 4) | ((uint32_t)ks << 29);
+              const uint32_t id = idesc | ((uint32_t)ks << 4) | ((uint32_t)ks << 29);
               mma_mxf8(d_tmem, ad, bd, id, accum, sfa_t, sfb_t);
             }
           }
@@ -492,7 +512,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             bulk_commit();
           }
         }
-      } else {  // EPI_SWIGLU_BWD: accumulator = dh for columns [nt*256, +256)
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {  // accumulator = dh, columns [nt*256, +256)
         const int n0 = t.nt * BN + hc * (BN / 2);
         constexpr int NCH = BN / 2 / CHUNK;
 #pragma unroll 1
@@ -547,6 +567,85 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
         if (!ok) break;
+      } else {  // EPI_ROUTER: accumulator = fp32 logits, 128 tokens x E experts
+        constexpr int KT = 8;                          // running top-8 list (k <= 8)
+        int* sel_s = reinterpret_cast<int*>(sStg);     // [128][k] chosen experts
+        int* cnt_s = sel_s + BM * KT;                  // [E] per-expert counters
+        const int rloc = q * 32 + lane;
+        const int row = t.row0 + rloc;
+        const bool valid = row < p.dense_rows;
+        const int k = p.r_k, E = p.r_E;
+        if (hc == 0) {
+          float bv[KT];
+          int be[KT];
+#pragma unroll
+          for (int i = 0; i < KT; ++i) { bv[i] = -INFINITY; be[i] = 0x7fffffff; }
+#pragma unroll 1
+          for (int c = 0; c < E; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tbase + c, v);
+            tmem_wait_ld();
+            float L[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              L[i] = __uint_as_float(v[i]) + ((p.r_bias && c + i < E) ? __ldg(p.r_bias + c + i) : 0.f);
+            if (valid && p.r_logits) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                if (c + i < E)
+                  *reinterpret_cast<float4*>(p.r_logits + (size_t)row * E + c + i) =
+                      make_float4(L[i], L[i + 1], L[i + 2], L[i + 3]);
+            }
+            // experts arrive in increasing order, so a strict '>' keeps the
+            // lower index first among equal logits
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (c + i >= E) break;
+              float cv = L[i];
+              int ce = c + i;
+              if (cv != cv) { cv = -INFINITY; if (valid) report(p.status, MOE_DEV_NONFINITE); }
+#pragma unroll
+              for (int s2 = 0; s2 < KT; ++s2) {
+                if (cv > bv[s2]) {
+                  const float tv = bv[s2]; bv[s2] = cv; cv = tv;
+                  const int te = be[s2]; be[s2] = ce; ce = te;
+                }
+              }
+            }
+          }
+          float ssum = 0.f;
+#pragma unroll
+          for (int j = 0; j < KT; ++j)
+            if (j < k) ssum += expf(bv[j] - bv[0]);
+#pragma unroll
+          for (int j = 0; j < KT; ++j) {
+            if (j >= k) continue;
+            if (valid) {
+              p.r_topk[(size_t)row * k + j] = be[j];
+              p.r_gates[(size_t)row * k + j] = expf(bv[j] - bv[0]) / ssum;
+            }
+            sel_s[rloc * k + j] = valid ? be[j] : -1;
+          }
+          // rank of each assignment among this tile's assignments to the same
+          // expert, in token order, and the tile's per-expert histogram
+          named_bar_sync(1, 128);
+          for (int e = rloc; e < E; e += 128) cnt_s[e] = 0;
+          named_bar_sync(1, 128);
+          if (ew == 0) {
+            for (int tt = 0; tt < BM; ++tt) {
+              if (lane < k) {
+                const int e = sel_s[tt * k + lane];
+                int rk = -1;
+                if (e >= 0) { rk = cnt_s[e]; cnt_s[e] = rk + 1; }
+                if (t.row0 + tt < p.dense_rows) p.r_rank[(size_t)(t.row0 + tt) * k + lane] = rk;
+              }
+              __syncwarp();
+            }
+          }
+          named_bar_sync(1, 128);
+          for (int e = rloc; e < E; e += 128) p.r_hist[(size_t)(t.row0 / BM) * E + e] = cnt_s[e];
+          named_bar_sync(1, 128);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -654,6 +753,38 @@ static Params base_params(const int32_t* poff, int E, int32_t* status) {
   p.status = status;
   return p;
 }
+
+// Router logits on the tensor cores: x [T, d] (bf16) times W_r split exactly
+// into three bf16 parts stacked as wsplit [3d, E] (w0 + w1 + w2 = W_r), as one
+// K = 3d GEMM whose A operand repeats x; fp32 accumulation in TMEM; top-k,
+// gates, per-128-token-block ranks and histogram in the epilogue.
+namespace moe {
+moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int T, int d, int E,
+                       int k, float* logits, int32_t* topk, float* gates, int32_t* rank,
+                       int32_t* hist, int32_t* status, cudaStream_t s) {
+  Params p = base_params(nullptr, 1, status);
+  p.dense_rows = T;
+  p.a_k_wrap = d;
+  p.num_kb = 3 * d / 64;
+  p.b_rows_per_e = 0;
+  p.n_tiles = 1;
+  p.mma_n = (E + 15) / 16 * 16;
+  p.b_boxes = (p.mma_n + 63) / 64;
+  p.r_bias = bias;
+  p.r_logits = logits;
+  p.r_topk = topk;
+  p.r_gates = gates;
+  p.r_rank = rank;
+  p.r_hist = hist;
+  p.r_k = k;
+  p.r_E = E;
+  Maps m;
+  MOE_TRY(make_map(&m.a, x, 2, d, T, 64, BM));
+  MOE_TRY(make_map(&m.b, wsplit, 2, E, 3ULL * d, 64, 64));
+  m.b3 = m.c = m.c2 = m.in = m.a;
+  return launch<false, false, B_MN, EPI_ROUTER>(m, p, (T + BM - 1) / BM, s);
+}
+}  // namespace moe
 
 extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc,
                                              const void* B, const uint8_t* B_sc, const void* B3,

@@ -80,7 +80,8 @@ size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
     x.XpT_q = l.take<uint8_t>(A * d);      x.XpT_s = l.take<uint8_t>(A * d / 32);
     x.dAT_q = l.take<uint8_t>(A * 2 * F);  x.dAT_s = l.take<uint8_t>(A * 2 * F / 32);
   }
-  const size_t ws_route = moe_route_workspace_size(L->T, L->E);
+  const size_t ws_route =
+      moe_route_workspace_size(L->T, L->route_mode == MOE_ROUTE_ROUTER ? L->d : 0, L->E);
   const size_t ws_unperm = moe_unpermute_sum_workspace_size(L->d, L->E);
   const size_t ws_rw = moe_router_wgrad_workspace_size(L->d, (int)A);
   x.ws_bytes = ws_route > ws_unperm ? ws_route : ws_unperm;

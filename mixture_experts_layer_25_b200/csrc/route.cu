@@ -5,10 +5,15 @@
 // never waits for it.  Nothing here copies to the host or synchronises.
 //
 // Three launches, all stream-ordered:
-//   1. route_topk / route_given: per block of 32 tokens, the k experts of
-//      each token (router: fp32 logits, top-k, gates), each assignment's rank
-//      among the block's assignments to the same expert (token order), and
-//      the block's per-expert histogram.
+//   1. per block of tokens, the k experts of each token (router: fp32
+//      logits, top-k, gates), each assignment's rank among the block's
+//      assignments to the same expert (token order), and the block's
+//      per-expert histogram.  Router mode runs on the tensor cores when it
+//      can (E <= 256, E % 8 == 0, k <= 8, d % 64 == 0; blocks of 128 tokens):
+//      W_r is split exactly into three bf16 parts w0 + w1 + w2 and the logits
+//      are one K = 3d product [x|x|x] [w0;w1;w2] accumulated in fp32.  The
+//      fallback (and given-mode) kernels use blocks of 32 tokens and fp32
+//      FMA.
 //   2. route_scan (one CTA): per-expert exclusive scan of the block
 //      histograms -> block offsets, counts, offsets, padded offsets poff.
 //   3. route_scatter: dst = poff[e] + block offset + in-block rank, src, and
@@ -203,6 +208,24 @@ route_given_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
 }
 
 // ---------------------------------------------------------------------------
+// W_r [d, E] fp32 -> wsplit [3d, E] bf16 with w0 = bf16(W), w1 = bf16(W - w0),
+// w2 = bf16(W - w0 - w1): each difference is exact in fp32 and the last part
+// holds at most 8 significant bits, so w0 + w1 + w2 == W (normal range).
+__global__ void router_split_kernel(const float* __restrict__ Wr, int n,
+                                    __nv_bfloat16* __restrict__ ws) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float w = Wr[i];
+  const __nv_bfloat16 w0 = __float2bfloat16_rn(w);
+  const float r1 = w - __bfloat162float(w0);
+  const __nv_bfloat16 w1 = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(w1);
+  ws[i] = w0;
+  ws[n + i] = w1;
+  ws[2 * n + i] = __float2bfloat16_rn(r2);
+}
+
+// ---------------------------------------------------------------------------
 // One CTA: hist[b][e] -> exclusive offset of block b inside expert e;
 // counts, offsets, poff.
 constexpr int kScanThreads = 1024;
@@ -289,6 +312,7 @@ route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
 // pad rows of one expert each; the last block marks [poff[E], A_pad_max).
 __global__ void route_scatter_kernel(const int32_t* __restrict__ topk_idx,
                                      const int32_t* __restrict__ hist, int T, int E, int k,
+                                     int btok,
                                      const int32_t* __restrict__ counts,
                                      const int32_t* __restrict__ poff,
                                      int32_t* __restrict__ dst, int32_t* __restrict__ src,
@@ -304,7 +328,7 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk_idx,
       dst[a] = -1;
       return;
     }
-    const int r = poff[e] + hist[(size_t)(t / kTok) * E + e] + rank;
+    const int r = poff[e] + hist[(size_t)(t / btok) * E + e] + rank;
     dst[a] = r;
     src[r] = t;
   } else if (b < nA_blocks + E) {
@@ -319,10 +343,18 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk_idx,
 
 using namespace moe;
 
-extern "C" size_t moe_route_workspace_size(int T, int E) {
-  if (T <= 0 || E <= 0) return 0;
-  const size_t nblk = (T + kTok - 1) / kTok;
-  return round_up(nblk * (size_t)E * sizeof(int32_t), 256);
+static bool use_tensor_router(int d, int E, int k) {
+  return E <= 256 && E % 8 == 0 && k <= 8 && d % 64 == 0;
+}
+
+extern "C" size_t moe_route_workspace_size(int T, int d, int E) {
+  if (T <= 0 || E <= 0 || d < 0) return 0;
+  // fallback / given mode: histograms of 32-token blocks
+  const size_t simt = round_up((size_t)((T + kTok - 1) / kTok) * E * sizeof(int32_t), 256);
+  // tensor-core router: histograms of 128-token blocks + the split W_r
+  const size_t tc = round_up((size_t)((T + 127) / 128) * E * sizeof(int32_t), 256) +
+                    round_up((size_t)3 * d * E * sizeof(__nv_bfloat16), 256);
+  return simt > tc ? simt : tc;
 }
 
 extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* bias, int T,
@@ -338,14 +370,26 @@ extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* b
   MOE_CHECK_ARG(topk_idx && gates && counts && offsets && poff && dst && src,
                 "moe_route: null output");
   MOE_CHECK_ARG(mode == MOE_ROUTE_ROUTER || mode == MOE_ROUTE_GIVEN, "moe_route: bad mode");
-  const size_t need = moe_route_workspace_size(T, E);
+  const size_t need = moe_route_workspace_size(T, mode == MOE_ROUTE_ROUTER ? d : 0, E);
   if (!ws || ws_bytes < need) {
     set_error("moe_route: workspace %zu < %zu bytes", ws_bytes, need);
     return MOE_ERR_WORKSPACE;
   }
-  const int nblk = (T + kTok - 1) / kTok;
+  MOE_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255) == 0, "moe_route: workspace must be 256-byte aligned");
+  int btok = kTok;
   int32_t* hist = static_cast<int32_t*>(ws);
-  if (mode == MOE_ROUTE_ROUTER) {
+  if (mode == MOE_ROUTE_ROUTER && use_tensor_router(d, E, k)) {
+    MOE_CHECK_ARG(x && Wr && aligned16(x), "moe_route: router mode needs 16B-aligned x and Wr");
+    btok = 128;
+    const size_t hist_bytes = round_up((size_t)((T + 127) / 128) * E * sizeof(int32_t), 256);
+    __nv_bfloat16* wsplit =
+        reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + hist_bytes);
+    const int n = d * E;
+    router_split_kernel<<<(n + 255) / 256, 256, 0, s>>>(Wr, n, wsplit);
+    MOE_CHECK_LAUNCH("router_split");
+    MOE_TRY(router_tc(x, wsplit, bias, T, d, E, k, logits, topk_idx, gates, dst, hist,
+                      dev_status, s));
+  } else if (mode == MOE_ROUTE_ROUTER) {
     MOE_CHECK_ARG(x && Wr, "moe_route: router mode needs x and Wr");
     MOE_CHECK_ARG(E <= kMaxRouterE, "moe_route: router mode supports E <= %d", kMaxRouterE);
     MOE_CHECK_ARG(d > 0 && d % 8 == 0 && aligned16(x), "moe_route: d %% 8 and 16B-aligned x");
@@ -356,6 +400,7 @@ extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* b
                            (int)((size_t)kTok * (kMaxRouterE + 1) * sizeof(float)));
       attr_set = true;
     }
+    const int nblk = (T + kTok - 1) / kTok;
     route_topk_kernel<<<nblk, kRouteThreads, smem, s>>>(
         static_cast<const __nv_bfloat16*>(x), Wr, bias, T, d, E, k, topk_idx, gates, logits, dst,
         hist, dev_status);
@@ -363,19 +408,21 @@ extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* b
   } else {
     MOE_CHECK_ARG(E <= 4096, "moe_route: given mode supports E <= 4096");
     const size_t smem = (E + kTok * k) * sizeof(int);
+    const int nblk = (T + kTok - 1) / kTok;
     route_given_kernel<<<nblk, kRouteThreads, smem, s>>>(topk_idx, T, E, k, dst, hist,
                                                          dev_status);
     MOE_CHECK_LAUNCH("route_given");
   }
   {
+    const int nblk = (T + btok - 1) / btok;
     const int G = E <= kScanThreads ? max(1, kScanThreads / E) : 1;
     const size_t smem = ((size_t)G * E + E) * sizeof(int);
     route_scan_kernel<<<1, kScanThreads, smem, s>>>(hist, nblk, E, align, counts, offsets, poff);
     MOE_CHECK_LAUNCH("route_scan");
   }
   const int nA = (T * k + 255) / 256;
-  route_scatter_kernel<<<nA + E + 1, 256, 0, s>>>(topk_idx, hist, T, E, k, counts, poff, dst, src,
-                                                  A_pad_max, nA);
+  route_scatter_kernel<<<nA + E + 1, 256, 0, s>>>(topk_idx, hist, T, E, k, btok, counts, poff,
+                                                  dst, src, A_pad_max, nA);
   MOE_CHECK_LAUNCH("route_scatter");
   return MOE_OK;
 }
@@ -433,10 +480,10 @@ extern "C" moe_status_t moe_route_noalloc(const void* x, const float* Wr, const 
                                           int32_t* src, int A_pad_max, float* logits,
                                           int32_t* dev_status, moe_stream_t stream) {
   MOE_CHECK_ARG(T > 0 && E > 0, "moe_route_noalloc: bad T/E");
-  const size_t need = moe_route_workspace_size(T, E);
+  const size_t need = moe_route_workspace_size(T, mode == MOE_ROUTE_ROUTER ? d : 0, E);
   MOE_CHECK_ARG(need <= kNoAllocScratchBytes,
-                "moe_route_noalloc: needs %zu scratch bytes (ceil(T/32)*E*4) but the fixed "
-                "array holds %zu; use moe_route with a caller workspace",
+                "moe_route_noalloc: needs %zu scratch bytes (moe_route_workspace_size) but the "
+                "fixed array holds %zu; use moe_route with a caller workspace",
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
   MOE_TRY(scratch_for_current_device(&scratch));

@@ -39,8 +39,11 @@ def test_library_exports_every_declared_symbol():
 
 def test_host_size_queries():
     lib = _lib.lib()
-    assert lib.moe_route_workspace_size(16384, 128) == 512 * 128 * 4
-    assert lib.moe_route_workspace_size(0, 128) == 0
+    # given routing (d = 0): 32-token block histograms
+    assert lib.moe_route_workspace_size(16384, 0, 128) == 512 * 128 * 4
+    # tensor-core router: 128-token block histograms + W_r split in 3 bf16 parts
+    assert lib.moe_route_workspace_size(16384, 2048, 128) == 128 * 128 * 4 + 3 * 2048 * 128 * 2
+    assert lib.moe_route_workspace_size(0, 2048, 128) == 0
     assert lib.moe_unpermute_sum_workspace_size(2048, 128) == 2048 * 128 * 4
     d = _lib.LayerDesc(16384, 2048, 128, 4, 1024, 128, 0, 0)
     n = lib.moe_layer_ctx_bytes(ctypes.byref(d))

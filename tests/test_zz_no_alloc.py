@@ -75,9 +75,9 @@ def test_noalloc_route_matches_route_on_two_calls(mode):
 
 def test_noalloc_route_rejects_problems_beyond_its_fixed_scratch():
     E = 128
-    T = (_lib.lib().moe_route_workspace_size(1, E) and
-         (4 << 20) // (E * 4) * 32 + 32)          # one routing block too many
-    code = _lib.lib().moe_route_noalloc(None, None, None, T, 2048, E, 4, 128, 0, None, None,
+    T = (4 << 20) // (E * 4) * 32 + 32         # given routing: one 32-token block too many
+    assert _lib.lib().moe_route_workspace_size(T, 0, E) > (4 << 20)
+    code = _lib.lib().moe_route_noalloc(None, None, None, T, 0, E, 4, 128, 1, None, None,
                                         None, None, None, None, None, 0, None, None, None)
     assert code == _lib.MOE_ERR_INVALID_ARG
     assert b"fixed array" in _lib.lib().moe_last_error()
