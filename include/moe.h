@@ -207,6 +207,16 @@ MOE_API moe_status_t mx_quantize(const void* in, int rows, int cols, int axis, c
                          int E, const int32_t* nrows_dev, uint8_t* codes, uint8_t* scales,
                          moe_stream_t stream);
 
+/* mx_quantize_dual: both quantisations of one bf16 [rows, cols] tensor from
+ * a single pass -- codes_rows / scales_rows as mx_quantize axis 0 (blocks
+ * along a row) and codes_cols / scales_cols as axis 1 (blocks down a
+ * column), bit-identical to the two separate calls.  Every operand that
+ * feeds two GEMMs with different K axes (weights, h, dY, dA13) needs both. */
+MOE_API moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
+                                      const int32_t* nrows_dev, uint8_t* codes_rows,
+                                      uint8_t* scales_rows, uint8_t* codes_cols,
+                                      uint8_t* scales_cols, moe_stream_t stream);
+
 /* ------------------------------------------------------- grouped GEMMs
  * Grouped GEMM over the expert groups of the routing metadata ([OC3-ja]
  * "ルーティングと計算の最適化": many small per-expert matmuls as one grouped

@@ -18,7 +18,7 @@ from ._lib import (MOE_BF16, MOE_MXFP8, MOE_EPI_NONE, MOE_EPI_SWIGLU, MOE_EPI_SW
                    MOE_DEV_TIMEOUT, MOE_DEV_NONFINITE, MoeError, LayerDesc, LayerWeights,
                    LayerGrads, CtxView)
 
-__all__ = ["moe_route", "moe_permute", "mx_quantize", "moe_grouped_gemm_fwd",
+__all__ = ["moe_route", "moe_permute", "mx_quantize", "mx_quantize_dual", "moe_grouped_gemm_fwd",
            "moe_grouped_gemm_dgrad", "moe_grouped_gemm_wgrad", "moe_unpermute_combine",
            "moe_combine_bwd", "moe_unpermute_sum", "moe_router_wgrad", "MoELayer",
            "a_pad_max", "MoeError"]
@@ -101,6 +101,17 @@ def mx_quantize(t, axis: int, *, nrows=None, codes=None, scales=None, stream=Non
     _lib.call("mx_quantize", _p(t), R, C, axis, None, 0, _p(nrows), _p(codes), _p(scales),
               _s(stream))
     return codes, scales
+
+
+def mx_quantize_dual(t, *, nrows=None, stream=None):
+    """Both MX quantisations of a bf16 [R, C] tensor in one pass:
+    (codes, scales) along rows (axis 0) and (codes, scales) down columns."""
+    R, C = t.shape
+    mk = lambda *s: torch.empty(s, dtype=torch.uint8, device=t.device)
+    cr, sr, cc, sc = mk(R, C), mk(R * C // 32), mk(R, C), mk(R * C // 32)
+    _lib.call("mx_quantize_dual", _p(t), R, C, _p(nrows), _p(cr), _p(sr), _p(cc), _p(sc),
+              _s(stream))
+    return (cr, sr), (cc, sc)
 
 
 # ------------------------------------------------------------ grouped GEMM

@@ -62,6 +62,7 @@ _SIGS = {
     "moe_route_noalloc": (I, [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P]),
     "moe_permute": (I, [P, P, P, P, I, I, I, I, I, P, P, P, P]),
     "mx_quantize": (I, [P, I, I, I, P, I, P, P, P, P]),
+    "mx_quantize_dual": (I, [P, I, I, P, P, P, P, P, P]),
     "moe_grouped_gemm_fwd": (I, [I, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P]),
     "moe_grouped_gemm_dgrad": (I, [I, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P]),
     "moe_grouped_gemm_wgrad": (I, [I, P, P, P, P, P, I, I, I, I, P, P, P, P]),

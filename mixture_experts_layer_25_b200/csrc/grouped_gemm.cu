@@ -435,20 +435,52 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256;
 
+      // EARLY: this thread's accumulator slice goes to registers at once and
+      // the accumulator is handed back to the MMA warp before any store is
+      // made.  Used where TMEM holds a single accumulator (MXFP8) and the
+      // epilogue keeps no other large state; otherwise each 32-column chunk
+      // is read from TMEM when it is stored and the accumulator is released
+      // at the end of the tile (BF16 double-buffers its accumulators).
+      constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU);
+      constexpr int NV = EARLY ? 128 : 32;
+      uint32_t av[NV];
+      if constexpr (EARLY) {
+        if (!empty) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // STORE / SwiGLU-bwd: columns hc*128 + [0,128); SwiGLU: W1 part
+            // hc*64 + [0,64) then W3 part 128 + hc*64 + [0,64)
+            const uint32_t col = EPI == EPI_SWIGLU ? (i >> 1) * (BN / 2) + hc * 64 + (i & 1) * 32
+                                                   : hc * (BN / 2) + i * 32;
+            tmem_ld32(tbase + col, av + 32 * i);
+          }
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < NV; ++i) av[i] = 0u;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
+
       if constexpr (EPI == EPI_STORE) {
         const int n0 = t.nt * BN;
         const CUtensorMap* map = &tmC;
         int x0 = n0;
         if (p.wgrad && p.n_split > 0 && n0 >= p.n_split) { map = &tmC2; x0 = n0 - p.n_split; }
-#pragma unroll 1
-        for (int c = hc * (BN / 2); c < (hc + 1) * (BN / 2); c += CHUNK) {
-          uint32_t v[32];
-          if (!empty) {
-            tmem_ld32(tbase + c, v);
-            tmem_wait_ld();
-          } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
+        for (int ci = 0; ci < 4; ++ci) {
+          const int c = hc * (BN / 2) + ci * CHUNK;
+          const uint32_t* v = av + (EARLY ? 32 * ci : 0);
+          if constexpr (!EARLY) {
+            if (!empty) {
+              tmem_ld32(tbase + c, av);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) av[i] = 0u;
+            }
           }
           uint8_t* buf = stg;
           if (lane == 0) bulk_wait_read<0>();    // the previous store has read the box
@@ -473,12 +505,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         // accumulator columns [0,128) = A W1, [128,256) = A W3 for the output
         // columns [nt*128, nt*128 + 128)
         const int n0 = t.nt * (BN / 2);
-#pragma unroll 1
-        for (int c = hc * (BN / 4); c < (hc + 1) * (BN / 4); c += CHUNK) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tbase + c, g);
-          tmem_ld32(tbase + BN / 2 + c, u);
-          tmem_wait_ld();
+#pragma unroll
+        for (int ci = 0; ci < 2; ++ci) {
+          const int c = hc * (BN / 4) + ci * CHUNK;
+          uint32_t gl[EARLY ? 1 : 32], ul[EARLY ? 1 : 32];
+          if constexpr (!EARLY) {
+            tmem_ld32(tbase + c, gl);
+            tmem_ld32(tbase + BN / 2 + c, ul);
+            tmem_wait_ld();
+          }
+          const uint32_t* g = EARLY ? av + 32 * ci : gl;        // A W1
+          const uint32_t* u = EARLY ? av + 64 + 32 * ci : ul;   // A W3
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
 #pragma unroll
@@ -529,7 +566,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[ew][pr ^ 1], p.half + n0 + c + CHUNK, y0);
             in_pending |= 1u << (pr ^ 1);
           }
-          uint32_t v[32];
+          uint32_t* v = av;
           tmem_ld32(tbase + hc * (BN / 2) + c, v);
           tmem_wait_ld();
           int got = 1;
@@ -647,9 +684,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           named_bar_sync(1, 128);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if constexpr (!EARLY) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
     }
     if (lane == 0) bulk_wait_all();     // every store has landed before the CTA exits
     if constexpr (EPI == EPI_SWIGLU_BWD) {

@@ -7,7 +7,8 @@
 //           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad -> GEMM1 wgrad ->
 //           unpermute-sum (+ router input grad) -> router weight grad.
 // In MXFP8 mode every GEMM operand is quantised along that GEMM's K first
-// (weights included, inside the step).
+// (weights included, inside the step); operands used by two GEMMs with
+// different K axes are quantised along both in one pass.
 #include "common.cuh"
 
 namespace {
@@ -182,23 +183,28 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
     mark(S_GEMM2, true, s);
   } else {
     const int32_t* nrows = c.poff + E;
-    uint8_t* W1q = c.W13_q; uint8_t* W3q = c.W13_q + (size_t)E * d * F;
-    uint8_t* W1s = c.W13_s; uint8_t* W3s = c.W13_s + (size_t)E * d * F / 32;
+    const size_t wq = (size_t)E * d * F;
+    uint8_t* W1q = c.W13_q; uint8_t* W3q = c.W13_q + wq;
+    uint8_t* W1s = c.W13_s; uint8_t* W3s = c.W13_s + wq / 32;
     mark(S_PERMUTE, false, s);
     MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, c.Xp_q, c.Xp_s, stream));
     mark(S_PERMUTE, true, s);
-    // weights along the fwd GEMMs' K: W1/W3 down d, W2 down F
+    // every weight along both K axes it is used with, in one pass each:
+    // W1/W3 [E*d, F] down d (fwd GEMM1) and along F (GEMM1 dgrad); W2
+    // [E*F, d] down F (fwd GEMM2) and along d (GEMM2 dgrad)
     mark(S_QW, false, s);
-    MOE_TRY(mx_quantize(w->W1, E * d, F, 1, nullptr, E, nullptr, W1q, W1s, stream));
-    MOE_TRY(mx_quantize(w->W3, E * d, F, 1, nullptr, E, nullptr, W3q, W3s, stream));
-    MOE_TRY(mx_quantize(w->W2, E * F, d, 1, nullptr, E, nullptr, c.W2_q, c.W2_s, stream));
+    MOE_TRY(mx_quantize_dual(w->W1, E * d, F, nullptr, c.W13t_q, c.W13t_s, W1q, W1s, stream));
+    MOE_TRY(mx_quantize_dual(w->W3, E * d, F, nullptr, c.W13t_q + wq, c.W13t_s + wq / 32, W3q,
+                             W3s, stream));
+    MOE_TRY(mx_quantize_dual(w->W2, E * F, d, nullptr, c.W2t_q, c.W2t_s, c.W2_q, c.W2_s, stream));
     mark(S_QW, true, s);
     mark(S_GEMM1, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.Xp_q, c.Xp_s, W1q, W1s, W3q, W3s, c.poff, E, A, F, d,
                                  MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
     mark(S_GEMM1, true, s);
+    // h along F (fwd GEMM2) and down its rows (GEMM2 wgrad)
     mark(S_QH, false, s);
-    MOE_TRY(mx_quantize(c.h, A, F, 0, c.poff, E, nrows, c.h_q, c.h_s, stream));
+    MOE_TRY(mx_quantize_dual(c.h, A, F, nrows, c.h_q, c.h_s, c.hT_q, c.hT_s, stream));
     mark(S_QH, true, s);
     mark(S_GEMM2, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.h_q, c.h_s, c.W2_q, c.W2_s, nullptr, nullptr, c.poff,
@@ -249,41 +255,33 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
     mark(S_WGRAD1, true, s);
   } else {
     const int32_t* nrows = c.poff + E;
-    uint8_t* W1q = c.W13t_q; uint8_t* W3q = c.W13t_q + (size_t)E * d * F;
-    uint8_t* W1s = c.W13t_s; uint8_t* W3s = c.W13t_s + (size_t)E * d * F / 32;
-    // GEMM2 dgrad: K = d.  dY along d, W2 along d (rows of the [E*F, d] view)
+    const size_t wq = (size_t)E * d * F;
+    // (weights were quantised along both axes in the forward)
+    // dY along d (GEMM2 dgrad) and down its rows (GEMM2 wgrad)
     mark(S_QD2, false, s);
-    MOE_TRY(mx_quantize(c.dY, A, d, 0, c.poff, E, nrows, c.dY_q, c.dY_s, stream));
-    MOE_TRY(mx_quantize(w->W2, E * F, d, 0, nullptr, E, nullptr, c.W2t_q, c.W2t_s, stream));
+    MOE_TRY(mx_quantize_dual(c.dY, A, d, nrows, c.dY_q, c.dY_s, c.dYT_q, c.dYT_s, stream));
     mark(S_QD2, true, s);
     mark(S_DGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dY_q, c.dY_s, c.W2t_q, c.W2t_s, nullptr, nullptr,
                                    c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
                                    dev_status, stream));
     mark(S_DGRAD2, true, s);
-    // GEMM2 wgrad: K = rows of the group.  h and dY down their columns
-    mark(S_QW2, false, s);
-    MOE_TRY(mx_quantize(c.h, A, F, 1, c.poff, E, nrows, c.hT_q, c.hT_s, stream));
-    MOE_TRY(mx_quantize(c.dY, A, d, 1, c.poff, E, nrows, c.dYT_q, c.dYT_s, stream));
-    mark(S_QW2, true, s);
     mark(S_WGRAD2, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff, E, A, F,
                                    d, G->dW2, nullptr, dev_status, stream));
     mark(S_WGRAD2, true, s);
-    // GEMM1 dgrad: K = 2F.  dA13 along 2F, W1/W3 along F
+    // dA13 along 2F (GEMM1 dgrad) and down its rows (GEMM1 wgrad)
     mark(S_QD1, false, s);
-    MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 0, c.poff, E, nrows, c.dA_q, c.dA_s, stream));
-    MOE_TRY(mx_quantize(w->W1, E * d, F, 0, nullptr, E, nullptr, W1q, W1s, stream));
-    MOE_TRY(mx_quantize(w->W3, E * d, F, 0, nullptr, E, nullptr, W3q, W3s, stream));
+    MOE_TRY(mx_quantize_dual(c.dA13, A, 2 * F, nrows, c.dA_q, c.dA_s, c.dAT_q, c.dAT_s, stream));
     mark(S_QD1, true, s);
     mark(S_DGRAD1, false, s);
-    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, W1q, W1s, W3q, W3s, c.poff, E, A, F,
-                                   d, MOE_EPI_NONE, nullptr, c.dXp, dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, c.W13t_q, c.W13t_s, c.W13t_q + wq,
+                                   c.W13t_s + wq / 32, c.poff, E, A, F, d, MOE_EPI_NONE, nullptr,
+                                   c.dXp, dev_status, stream));
     mark(S_DGRAD1, true, s);
-    // GEMM1 wgrad: K = rows of the group.  Xp and dA13 down their columns
+    // Xp down its rows (GEMM1 wgrad)
     mark(S_QW1, false, s);
     MOE_TRY(mx_quantize(c.Xp, A, d, 1, c.poff, E, nrows, c.XpT_q, c.XpT_s, stream));
-    MOE_TRY(mx_quantize(c.dA13, A, 2 * F, 1, c.poff, E, nrows, c.dAT_q, c.dAT_s, stream));
     mark(S_QW1, true, s);
     mark(S_WGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff, E, A, d,

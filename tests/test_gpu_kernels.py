@@ -163,6 +163,24 @@ def test_mx_quantize_bit_exact(R, C, axis):
     np.testing.assert_array_equal(scales_to_plain(scales, R, C, axis), s)
 
 
+@pytest.mark.parametrize("R,C", [(256, 512), (384, 384), (128, 2048)])
+def test_mx_quantize_dual_equals_both_axes(R, C):
+    g = torch.Generator(device="cuda"); g.manual_seed(R * 7 + C)
+    v = (torch.randn((R, C), generator=g, device="cuda") *
+         torch.exp(torch.randn((R, 1), generator=g, device="cuda") * 3)).to(torch.bfloat16)
+    v[3, :40] = 0
+    v[7, 9] = -1e-30
+    (cr, sr), (cc, sc) = moe.mx_quantize_dual(v)
+    torch.cuda.synchronize()
+    v64 = f64(v)
+    c0, s0 = oracle.mx_quantize_rows(v64)
+    c1, s1 = oracle.mx_quantize_cols_grouped(v64, np.array([0, R]))
+    np.testing.assert_array_equal(cr.cpu().numpy(), c0)
+    np.testing.assert_array_equal(scales_to_plain(sr, R, C, 0), s0)
+    np.testing.assert_array_equal(cc.cpu().numpy(), c1)
+    np.testing.assert_array_equal(scales_to_plain(sc, R, C, 1), s1)
+
+
 @pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (257, 2048, 32, 4), (64, 6144, 384, 8)])
 def test_combine_and_its_backward(T, d, E, k):
     idx, gates, meta = _meta_for(T, E, k, 5)
