@@ -186,16 +186,25 @@ def _barrier(world):
 
 
 def _traffic(kernel_file):
-    """dram bytes per launch of the grouped GEMM from the committed ncu
-    summary, if it was taken on the current source of that kernel."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu
+    summary (profiles/traffic_grouped_gemm.md: lines `source_sha256: <hex>`
+    and `dram_bytes_per_launch: <int>`), or None unless that capture was
+    taken on the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic_grouped_gemm.md")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
+    fields = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip().strip("`- ")] = v.strip().strip("`")
     src = open(os.path.join(ROOT, "mixture_experts_layer_25_b200", "csrc", kernel_file), "rb").read()
-    if d.get("source_sha256") != hashlib.sha256(src).hexdigest():
+    if fields.get("source_sha256") != hashlib.sha256(src).hexdigest():
         return None
-    return d.get("dram_bytes_per_launch")
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def _cfg_dict(cfg, extra):

@@ -134,7 +134,7 @@ MOE_API void moe_set_stage_events(void* const* events, int n);
  *
  * mode MOE_ROUTE_ROUTER: logits = x W_r (+ bias) in fp32, top-k (ties to the
  *   lower index, slot j = j-th largest), gates = softmax of the k chosen
- *   logits (fp32); writes topk_idx [T,k] and gates [T,k].  With E <= 256,
+ *   logits (fp32); writes topk_idx [T,k] and gates [T,k].  With E <= 128,
  *   E % 8 == 0, k <= 8 and d % 64 == 0 the logits run on the tensor cores:
  *   W_r is split exactly into three bf16 parts (w0 + w1 + w2 = W_r, each
  *   product exact) accumulated in fp32; otherwise fp32 FMA on CUDA cores.

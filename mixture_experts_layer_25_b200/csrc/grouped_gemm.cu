@@ -59,10 +59,12 @@ enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3 };
 // with a 4-stage ring; SwiGLU stages h / H1 / H3; the SwiGLU backward
 // double-buffers H1/H3 pairs (both with a 3-stage ring)
 template <bool MX, int EPI> struct EpiCfg {
-  static constexpr int STAGES = (EPI == EPI_STORE || EPI == EPI_ROUTER) ? 4 : 3;
+  static constexpr int STAGES = EPI == EPI_STORE ? 4 : 3;
   static constexpr int BOXES = (EPI == EPI_STORE || EPI == EPI_ROUTER) ? 1 : EPI == EPI_SWIGLU ? 3 : 4;
   static constexpr int STG = BOXES * BOX_BYTES;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES +
+  // the router stage holds three B tiles (one per weight split) of <= 128 columns
+  static constexpr int B_STAGE = EPI == EPI_ROUTER ? 3 * 128 * 128 : B_BYTES;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_STAGE +
                                  (MX ? SFA_BYTES + SFB_BYTES : 0)) + NUM_EPI_WARPS * STG;
 };
 
@@ -93,7 +95,7 @@ struct Params {
   int k_out;          // wgrad: output rows per expert (K of the weight)
   // dense single-group mode (router): rows [0, dense_rows), no poff
   int dense_rows;
-  int a_k_wrap;       // > 0: A's K coordinate wraps modulo a_k_wrap
+  int split_rows;     // router: rows per weight split in the B map (= d)
   int mma_n;          // > 0: MMA N (multiple of 16, <= 256) instead of BN
   int b_boxes;        // > 0: MN-major B boxes loaded per stage (<= BN / chunk)
   // router epilogue
@@ -174,6 +176,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmIn, const Params p) {
   constexpr int STAGES = EpiCfg<MX, EPI>::STAGES;
   constexpr int STG = EpiCfg<MX, EPI>::STG;
+  constexpr int B_STAGE = EpiCfg<MX, EPI>::B_STAGE;
+  constexpr int SPLIT_BYTES = 128 * 128;   // router: one split's B tile (2 boxes)
   constexpr int ELEM = MX ? 1 : 2;
   constexpr int BK = 128 / ELEM;                 // K per stage (128-byte rows)
   constexpr int MMA_K = MX ? 32 : 16;
@@ -197,8 +201,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;                                  // STAGES x A_BYTES
-  uint8_t* sB = smem + STAGES * A_BYTES;               // STAGES x B_BYTES
-  uint8_t* sSF = sB + STAGES * B_BYTES;                // STAGES x (SFA + SFB), MX only
+  uint8_t* sB = smem + STAGES * A_BYTES;               // STAGES x B_STAGE
+  uint8_t* sSF = sB + STAGES * B_STAGE;                // STAGES x (SFA + SFB), MX only
   uint8_t* sStg = sSF + (MX ? STAGES * (SFA_BYTES + SFB_BYTES) : 0);   // per-warp staging
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -260,13 +264,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
           uint64_t* fb = &full_bar[stage];
           const int nbox = p.b_boxes ? p.b_boxes : BN / MN_CHUNK;
-          mbar_arrive_expect_tx(fb, B_MNMAJOR ? STAGE_TX - (BN / MN_CHUNK - nbox) * MN_CHUNK_BYTES
-                                              : STAGE_TX);
+          if constexpr (EPI == EPI_ROUTER)
+            mbar_arrive_expect_tx(fb, A_BYTES + 3 * nbox * MN_CHUNK_BYTES);
+          else
+            mbar_arrive_expect_tx(fb, B_MNMAJOR ? STAGE_TX - (BN / MN_CHUNK - nbox) * MN_CHUNK_BYTES
+                                                : STAGE_TX);
           uint8_t* a_dst = sA + stage * A_BYTES;
-          uint8_t* b_dst = sB + stage * B_BYTES;
+          uint8_t* b_dst = sB + stage * B_STAGE;
           // A operand
           if constexpr (!A_MN) {
-            tma_load_2d(a_dst, &tmA, fb, p.a_k_wrap ? (kb * BK) % p.a_k_wrap : kb * BK, t.row0);
+            tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
           } else {
 #pragma unroll
             for (int i = 0; i < BM / MN_CHUNK; ++i)
@@ -275,7 +282,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           // B operand
           const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
-          if constexpr (BLOAD == B_MN) {
+          if constexpr (EPI == EPI_ROUTER) {
+            // rows kb*BK.. of each weight split (split s starts at row s * d)
+            for (int sp = 0; sp < 3; ++sp)
+              for (int i = 0; i < nbox; ++i)
+                tma_load_2d(b_dst + sp * SPLIT_BYTES + i * MN_CHUNK_BYTES, &tmB, fb, i * MN_CHUNK,
+                            sp * p.split_rows + kb * BK);
+          } else if constexpr (BLOAD == B_MN) {
 #pragma unroll
             for (int i = 0; i < nbox; ++i)
               tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * BN + i * MN_CHUNK,
@@ -362,7 +375,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           tc_fence_after();
-          const uint32_t sa = a_base + stage * A_BYTES, sb = b_base + stage * B_BYTES;
+          const uint32_t sa = a_base + stage * A_BYTES, sb = b_base + stage * B_STAGE;
           uint32_t sfa_t = 0, sfb_t = 0;
           if constexpr (MX) {
             const uint32_t sf = smem_u32(sSF + stage * (SFA_BYTES + SFB_BYTES));
@@ -372,6 +385,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tmem_cp_32x128b_warpx4(sfb_t, smem_desc(sf + SFA_BYTES, 0, 128, 0));
             tmem_cp_32x128b_warpx4(sfb_t + 4, smem_desc(sf + SFA_BYTES + 512, 0, 128, 0));
           }
+          if constexpr (EPI == EPI_ROUTER) {
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+              const uint64_t ad = smem_desc(sa + ks * 32, 16, 1024, 2);
+#pragma unroll
+              for (int sp = 0; sp < 3; ++sp) {
+                const uint64_t bd =
+                    smem_desc(sb + sp * SPLIT_BYTES + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
+                mma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || ks > 0 || sp > 0) ? 1u : 0u);
+              }
+            }
+          } else
 #pragma unroll
           for (int ks = 0; ks < KSTEPS; ++ks) {
             uint64_t ad, bd;
@@ -794,8 +819,9 @@ static Params base_params(const int32_t* poff, int E, int32_t* status) {
 }
 
 // Router logits on the tensor cores: x [T, d] (bf16) times W_r split exactly
-// into three bf16 parts stacked as wsplit [3d, E] (w0 + w1 + w2 = W_r), as one
-// K = 3d GEMM whose A operand repeats x; fp32 accumulation in TMEM; top-k,
+// into three bf16 parts stacked as wsplit [3d, E] (w0 + w1 + w2 = W_r): each
+// stage holds one x tile and the three split tiles of the same K rows, and
+// all three products accumulate into one fp32 TMEM accumulator; top-k,
 // gates, per-128-token-block ranks and histogram in the epilogue.
 namespace moe {
 moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int T, int d, int E,
@@ -803,8 +829,8 @@ moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int
                        int32_t* hist, int32_t* status, cudaStream_t s) {
   Params p = base_params(nullptr, 1, status);
   p.dense_rows = T;
-  p.a_k_wrap = d;
-  p.num_kb = 3 * d / 64;
+  p.split_rows = d;        // split s of W_r starts at row s * d of wsplit
+  p.num_kb = d / 64;
   p.b_rows_per_e = 0;
   p.n_tiles = 1;
   p.mma_n = (E + 15) / 16 * 16;

@@ -9,7 +9,7 @@
 //      logits, top-k, gates), each assignment's rank among the block's
 //      assignments to the same expert (token order), and the block's
 //      per-expert histogram.  Router mode runs on the tensor cores when it
-//      can (E <= 256, E % 8 == 0, k <= 8, d % 64 == 0; blocks of 128 tokens):
+//      can (E <= 128, E % 8 == 0, k <= 8, d % 64 == 0; blocks of 128 tokens):
 //      W_r is split exactly into three bf16 parts w0 + w1 + w2 and the logits
 //      are one K = 3d product [x|x|x] [w0;w1;w2] accumulated in fp32.  The
 //      fallback (and given-mode) kernels use blocks of 32 tokens and fp32
@@ -344,7 +344,7 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ topk_idx,
 using namespace moe;
 
 static bool use_tensor_router(int d, int E, int k) {
-  return E <= 256 && E % 8 == 0 && k <= 8 && d % 64 == 0;
+  return E <= 128 && E % 8 == 0 && k <= 8 && d % 64 == 0;
 }
 
 extern "C" size_t moe_route_workspace_size(int T, int d, int E) {

@@ -42,7 +42,10 @@ def _check_metadata(meta, idx, E):
 
 @pytest.mark.parametrize("T,d,E,k,bias", [
     (1024, 256, 8, 2, False),     # the tiny layer
-    (37, 64, 5, 3, False),        # ragged: one partial routing block
+    (37, 64, 5, 3, False),        # ragged: one partial routing block (CUDA-core path)
+    (37, 128, 8, 2, False),       # ragged, tensor-core path
+    (300, 256, 64, 8, True),      # k = 8 on the tensor-core path
+    (200, 64, 136, 3, False),     # E > 128: CUDA-core path
     (1000, 128, 16, 4, True),
     (4096, 2048, 128, 4, True),   # skewed load, many empty experts
     (16384, 2048, 128, 4, False), # the 128-expert layer at full size
