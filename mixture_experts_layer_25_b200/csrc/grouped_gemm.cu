@@ -58,9 +58,20 @@ enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3 };
 // within the 227 KB of shared memory per CTA: STORE uses one box per warp
 // with a 4-stage ring; SwiGLU stages h / H1 / H3; the SwiGLU backward
 // double-buffers H1/H3 pairs (both with a 3-stage ring)
+#ifndef MOE_GG_SWIGLU_STAGES
+#define MOE_GG_SWIGLU_STAGES 4    // 4: one box, stores in turn; 3: h/H1/H3 boxes per warp
+#endif
+#ifndef MOE_GG_STORE_BOXES
+#define MOE_GG_STORE_BOXES 1      // 1: 4-stage ring; 2: double-buffered boxes, 3 stages
+#endif
 template <bool MX, int EPI> struct EpiCfg {
-  static constexpr int STAGES = EPI == EPI_STORE ? 4 : 3;
-  static constexpr int BOXES = (EPI == EPI_STORE || EPI == EPI_ROUTER) ? 1 : EPI == EPI_SWIGLU ? 3 : 4;
+  static constexpr int SWIGLU_STAGES = MX ? 3 : MOE_GG_SWIGLU_STAGES;
+  static constexpr int STORE_BOXES = MOE_GG_STORE_BOXES;
+  static constexpr int STAGES = EPI == EPI_STORE ? (STORE_BOXES == 1 ? 4 : 3)
+                              : EPI == EPI_SWIGLU ? SWIGLU_STAGES : 3;
+  static constexpr int BOXES = EPI == EPI_STORE ? STORE_BOXES
+                             : EPI == EPI_ROUTER ? 1
+                             : EPI == EPI_SWIGLU ? (SWIGLU_STAGES == 4 ? 1 : 3) : 4;
   static constexpr int STG = BOXES * BOX_BYTES;
   // the router stage holds three B tiles (one per weight split) of <= 128 columns
   static constexpr int B_STAGE = EPI == EPI_ROUTER ? 3 * 128 * 128 : B_BYTES;
@@ -494,7 +505,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const CUtensorMap* map = &tmC;
         int x0 = n0;
         if (p.wgrad && p.n_split > 0 && n0 >= p.n_split) { map = &tmC2; x0 = n0 - p.n_split; }
-#pragma unroll
+#pragma unroll(EARLY ? 4 : 1)
         for (int ci = 0; ci < 4; ++ci) {
           const int c = hc * (BN / 2) + ci * CHUNK;
           const uint32_t* v = av + (EARLY ? 32 * ci : 0);
@@ -507,8 +518,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               for (int i = 0; i < 32; ++i) av[i] = 0u;
             }
           }
-          uint8_t* buf = stg;
-          if (lane == 0) bulk_wait_read<0>();    // the previous store has read the box
+          constexpr int NB = EpiCfg<MX, EPI>::BOXES;
+          uint8_t* buf = stg + (NB > 1 ? (ci & 1) * BOX_BYTES : 0);
+          if (lane == 0) {                       // the store that last used `buf` has read it
+            if constexpr (NB > 1) bulk_wait_read<1>();
+            else bulk_wait_read<0>();
+          }
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -530,7 +545,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         // accumulator columns [0,128) = A W1, [128,256) = A W3 for the output
         // columns [nt*128, nt*128 + 128)
         const int n0 = t.nt * (BN / 2);
-#pragma unroll
+#pragma unroll(EARLY ? 2 : 1)
         for (int ci = 0; ci < 2; ++ci) {
           const int c = hc * (BN / 4) + ci * CHUNK;
           uint32_t gl[EARLY ? 1 : 32], ul[EARLY ? 1 : 32];
@@ -541,8 +556,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           const uint32_t* g = EARLY ? av + 32 * ci : gl;        // A W1
           const uint32_t* u = EARLY ? av + 64 + 32 * ci : ul;   // A W3
+          constexpr bool ONE_BOX = EpiCfg<MX, EPI>::BOXES == 1;
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
+          uint4 hkeep[ONE_BOX ? 4 : 1], gkeep[ONE_BOX ? 4 : 1], ukeep[ONE_BOX ? 4 : 1];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint4 hw, gw, uw;
@@ -559,19 +576,45 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               gp[i] = bf16x2_bits(g0, g1);
               up[i] = bf16x2_bits(u0, u1);
             }
-            *reinterpret_cast<uint4*>(stg + sw64(r, j)) = hw;
-            *reinterpret_cast<uint4*>(stg + BOX_BYTES + sw64(r, j)) = gw;
-            *reinterpret_cast<uint4*>(stg + 2 * BOX_BYTES + sw64(r, j)) = uw;
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmC, stg, n0 + c, y0);
-            if (p.aux) {
-              tma_store_2d(&tmC2, stg + BOX_BYTES, n0 + c, y0);
-              tma_store_2d(&tmC2, stg + 2 * BOX_BYTES, p.half + n0 + c, y0);
+            if constexpr (ONE_BOX) {
+              hkeep[j] = hw; gkeep[j] = gw; ukeep[j] = uw;
+            } else {
+              *reinterpret_cast<uint4*>(stg + sw64(r, j)) = hw;
+              *reinterpret_cast<uint4*>(stg + BOX_BYTES + sw64(r, j)) = gw;
+              *reinterpret_cast<uint4*>(stg + 2 * BOX_BYTES + sw64(r, j)) = uw;
             }
-            bulk_commit();
+          }
+          if constexpr (ONE_BOX) {
+            // one staging box: h, then H1, then H3, each stored before the next
+            const uint4* outs[3] = {hkeep, gkeep, ukeep};
+#pragma unroll
+            for (int o = 0; o < 3; ++o) {
+              if (o > 0 && !p.aux) break;
+              if (o > 0) {
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+              }
+#pragma unroll
+              for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(stg + sw64(r, j)) = outs[o][j];
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                if (o == 0) tma_store_2d(&tmC, stg, n0 + c, y0);
+                else tma_store_2d(&tmC2, stg, (o == 2 ? p.half : 0) + n0 + c, y0);
+                bulk_commit();
+              }
+            }
+          } else {
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmC, stg, n0 + c, y0);
+              if (p.aux) {
+                tma_store_2d(&tmC2, stg + BOX_BYTES, n0 + c, y0);
+                tma_store_2d(&tmC2, stg + 2 * BOX_BYTES, p.half + n0 + c, y0);
+              }
+              bulk_commit();
+            }
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {  // accumulator = dh, columns [nt*256, +256)

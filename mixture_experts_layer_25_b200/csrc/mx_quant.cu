@@ -10,8 +10,12 @@
 // number with exponent field 254 - byte (exact power-of-two scaling).
 // Scales go to the tensor-core layout (see the library header).
 #include <cuda_fp8.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace moe {
 
@@ -212,6 +216,127 @@ mx_quant_dual_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols,
   }
 }
 
+// ------------------------------ both axes, TMA-fed persistent variant
+// Persistent CTAs of 8 warps walk 128 x 128 tiles; each tile arrives in
+// shared memory by TMA (two 64-column boxes, no swizzle) while the previous
+// tile is quantised, so the bytes in flight do not depend on registers.
+// Warp w takes rows 16w..16w+15 of the tile (half of one 32-row MX column
+// block; warps 2b and 2b+1 combine their column maxima through shared
+// memory), lane L columns 4L..4L+3; both passes read shared memory.
+constexpr int kDualTile = 128;
+constexpr int kDualTileBytes = kDualTile * kDualTile * 2;
+constexpr int kDualWarps = 8;
+
+#ifndef MOE_QDUAL_MIN_BLOCKS
+#define MOE_QDUAL_MIN_BLOCKS 3     // resident CTAs per SM the register budget aims for
+#endif
+__global__ void __launch_bounds__(32 * kDualWarps, MOE_QDUAL_MIN_BLOCKS)
+mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int cols,
+                         const int32_t* __restrict__ nrows_dev, uint8_t* __restrict__ codes_r,
+                         uint8_t* __restrict__ scales_r, uint8_t* __restrict__ codes_c,
+                         uint8_t* __restrict__ scales_c) {
+  using namespace sm100;
+  extern __shared__ __align__(128) uint8_t qsm[];
+  __shared__ __align__(8) uint64_t full[2];
+  __shared__ volatile int abort_flag;
+  __shared__ float camax[kDualWarps][kDualTile];   // per-warp column maxima
+  __shared__ uint32_t cbyte[4][kDualTile];         // column scale byte per 32-row block
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nrows = nrows_dev ? min(*nrows_dev, rows) : rows;
+  const int tiles_r = (nrows + kDualTile - 1) / kDualTile, tiles_c = cols / kDualTile;
+  const int ntiles = tiles_r * tiles_c;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int tile, int buf) {
+    const int tr = tile / tiles_c, tc = tile % tiles_c;
+    uint8_t* dst = qsm + buf * kDualTileBytes;
+    mbar_arrive_expect_tx(&full[buf], kDualTileBytes);
+    tma_load_2d(dst, &tin, &full[buf], tc * kDualTile, tr * kDualTile);
+    tma_load_2d(dst + kDualTileBytes / 2, &tin, &full[buf], tc * kDualTile + 64, tr * kDualTile);
+  };
+  if (threadIdx.x == 0 && (int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+  uint32_t phase = 0;   // bit b: parity of full[b]
+  int it = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    if (threadIdx.x == 0 && tile + (int)gridDim.x < ntiles) issue(tile + gridDim.x, buf ^ 1);
+    if (!mbar_wait(&full[buf], (phase >> buf) & 1, &abort_flag, nullptr, 2000000000ull)) break;
+    phase ^= 1u << buf;
+    const int tr = tile / tiles_c, tc = tile % tiles_c;
+    const uint8_t* t = qsm + buf * kDualTileBytes;
+    // lane L: columns 4L..4L+3 of the tile: box L/16, 8-byte slot L%16 of a 128-byte row
+    const uint8_t* base = t + (lane >> 4) * (kDualTileBytes / 2) + (lane & 15) * 8;
+    const int rl0 = warp * 16;                         // first tile row of this warp
+    const int r0 = tr * kDualTile + rl0;
+    const int col = tc * kDualTile + lane * 4;
+    float amax[4] = {0, 0, 0, 0};
+    uint32_t rs[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float f[4];
+      unpack4(*reinterpret_cast<const uint2*>(base + (rl0 + r) * 128), f);
+      float ra = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        amax[i] = fmaxf(amax[i], fabsf(f[i]));
+        ra = fmaxf(ra, fabsf(f[i]));
+      }
+      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 1));
+      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 2));
+      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 4));
+      rs[r] = scale_byte(ra);
+      // the word of row r0+r for this tile's 4 column blocks: lanes 0, 8, 16, 24
+      const uint32_t b1 = __shfl_down_sync(0xffffffffu, rs[r], 8);
+      const uint32_t b2 = __shfl_down_sync(0xffffffffu, rs[r], 16);
+      const uint32_t b3 = __shfl_down_sync(0xffffffffu, rs[r], 24);
+      if (lane == 0 && r0 + r < nrows) {
+        const int mn = r0 + r;
+        const size_t off = ((size_t)(mn >> 7) * (cols / 128) + tc) * 512 + (mn & 31) * 16 +
+                           ((mn >> 5) & 3) * 4;
+        *reinterpret_cast<uint32_t*>(scales_r + off) = rs[r] | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) camax[warp][lane * 4 + i] = amax[i];
+    __syncthreads();
+    float inv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = fmaxf(amax[i], camax[warp ^ 1][lane * 4 + i]);
+      const uint32_t b = scale_byte(a);
+      inv[i] = inv_scale(b);
+      if ((warp & 1) == 0) cbyte[warp >> 1][lane * 4 + i] = (r0 < nrows) ? b : 0u;
+    }
+    if (r0 < nrows) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        float f[4];
+        unpack4(*reinterpret_cast<const uint2*>(base + (rl0 + r) * 128), f);
+        const float ir = inv_scale(rs[r]);
+        const float irr[4] = {ir, ir, ir, ir};
+        *reinterpret_cast<uint32_t*>(codes_c + (size_t)(r0 + r) * cols + col) = encode4(f, inv);
+        *reinterpret_cast<uint32_t*>(codes_r + (size_t)(r0 + r) * cols + col) = encode4(f, irr);
+      }
+    }
+    __syncthreads();
+    // column scales: the tile's four 32-row blocks of one column form one word
+    if (threadIdx.x < kDualTile) {
+      const int c = threadIdx.x;
+      const uint32_t word = cbyte[0][c] | (cbyte[1][c] << 8) | (cbyte[2][c] << 16) | (cbyte[3][c] << 24);
+      const int mn = tc * kDualTile + c;
+      const size_t off = ((size_t)(mn >> 7) * (rows / 128) + tr) * 512 + (mn & 31) * 16 +
+                         ((mn >> 5) & 3) * 4;
+      *reinterpret_cast<uint32_t*>(scales_c + off) = word;
+    }
+    __syncthreads();   // buffer `buf`, camax and cbyte are free for the next round
+  }
+}
+
 // -------------------------------------------- permute fused with MX codes
 constexpr int kMaxK = 16;
 constexpr int kWarps = 8;
@@ -315,6 +440,22 @@ extern "C" moe_status_t mx_quantize(const void* in, int rows, int cols, int axis
   return MOE_OK;
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_q() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+}  // namespace
+
 extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
                                          const int32_t* nrows_dev, uint8_t* codes_rows,
                                          uint8_t* scales_rows, uint8_t* codes_cols,
@@ -325,13 +466,33 @@ extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
   MOE_CHECK_ARG(in && codes_rows && scales_rows && codes_cols && scales_cols && aligned16(in) &&
                     aligned16(codes_rows) && aligned16(codes_cols),
                 "mx_quantize_dual: null or unaligned pointer");
-  const int segs = cols / 128;
-  const int warps_per_block = 4;
-  const long long warps = (long long)(rows / 128) * segs;
-  const long long blocks = (warps + warps_per_block - 1) / warps_per_block;
-  mx_quant_dual_kernel<<<(unsigned)blocks, 32 * warps_per_block, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(in), rows, cols, nrows_dev, codes_rows, scales_rows,
-      codes_cols, scales_cols);
+  auto fn = encode_fn_q();
+  if (!fn) {
+    set_error("mx_quantize_dual: cuTensorMapEncodeTiled unavailable");
+    return MOE_ERR_CUDA;
+  }
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(in), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+    set_error("mx_quantize_dual: tensor map encoding failed");
+    return MOE_ERR_CUDA;
+  }
+  const size_t smem = 2 * (size_t)kDualTileBytes;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(mx_quant_dual_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    attr = true;
+  }
+  const long long ntiles = (long long)(rows / 128) * (cols / 128);
+  const int grid = (int)std::min<long long>(ntiles, (long long)MOE_QDUAL_MIN_BLOCKS * num_sms());
+  mx_quant_dual_tma_kernel<<<grid, 32 * kDualWarps, smem, s>>>(m, rows, cols, nrows_dev, codes_rows,
+                                                   scales_rows, codes_cols, scales_cols);
   MOE_CHECK_LAUNCH("mx_quantize_dual");
   return MOE_OK;
 }
