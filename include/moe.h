@@ -271,6 +271,15 @@ MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t
                                     int A_pad_max, int K, int N, void* dB, void* dB3,
                                     int32_t* dev_status, moe_stream_t stream);
 
+/* Self-test of the failure detection the grouped GEMM relies on: a kernel
+ * waits on an mbarrier that nothing arrives at, gives up after limit_ns
+ * (at most 2 s), ORs MOE_DEV_TIMEOUT into *dev_status and returns, leaving
+ * the context usable.  The GEMM's own waits use the same bounded wait (2 s):
+ * a time-out there makes every role of the CTA drain its copies in flight,
+ * release TMEM and exit, with MOE_DEV_TIMEOUT set. */
+MOE_API moe_status_t moe_selftest_wait_timeout(int32_t* dev_status, uint64_t limit_ns,
+                                               moe_stream_t stream);
+
 /* -------------------------------------------------- unpermute / combine
  * Gate-weighted combine (the unpermute half of the rowwise dispatch of
  * [OC3-ja]): out[t] = sum_{j<k} gates[t,j] * Y[dst[t,j]], fp32 sum in slot

@@ -64,9 +64,12 @@ enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3 };
 #ifndef MOE_GG_STORE_BOXES
 #define MOE_GG_STORE_BOXES 1      // 1: 4-stage ring; 2: double-buffered boxes, 3 stages
 #endif
-template <bool MX, int EPI> struct EpiCfg {
+#ifndef MOE_GG_WGRAD_BOXES
+#define MOE_GG_WGRAD_BOXES 1      // weight-gradient tiles: 2 = double-buffered boxes, 3 stages
+#endif
+template <bool MX, int EPI, bool WGRAD = false> struct EpiCfg {
   static constexpr int SWIGLU_STAGES = MX ? 3 : MOE_GG_SWIGLU_STAGES;
-  static constexpr int STORE_BOXES = MOE_GG_STORE_BOXES;
+  static constexpr int STORE_BOXES = WGRAD ? MOE_GG_WGRAD_BOXES : MOE_GG_STORE_BOXES;
   static constexpr int STAGES = EPI == EPI_STORE ? (STORE_BOXES == 1 ? 4 : 3)
                               : EPI == EPI_SWIGLU ? SWIGLU_STAGES : 3;
   static constexpr int BOXES = EPI == EPI_STORE ? STORE_BOXES
@@ -107,6 +110,7 @@ struct Params {
   // dense single-group mode (router): rows [0, dense_rows), no poff
   int dense_rows;
   int split_rows;     // router: rows per weight split in the B map (= d)
+  int a3d, b3d;       // MN-major operand maps are 3-D (chunk, row, chunk index): one load per stage
   int mma_n;          // > 0: MMA N (multiple of 16, <= 256) instead of BN
   int b_boxes;        // > 0: MN-major B boxes loaded per stage (<= BN / chunk)
   // router epilogue
@@ -185,9 +189,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmC2,
                     const __grid_constant__ CUtensorMap tmIn, const Params p) {
-  constexpr int STAGES = EpiCfg<MX, EPI>::STAGES;
-  constexpr int STG = EpiCfg<MX, EPI>::STG;
-  constexpr int B_STAGE = EpiCfg<MX, EPI>::B_STAGE;
+  using Cfg = EpiCfg<MX, EPI, A_MN>;      // A MN-major <=> weight-gradient tiles
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int STG = Cfg::STG;
+  constexpr int B_STAGE = Cfg::B_STAGE;
   constexpr int SPLIT_BYTES = 128 * 128;   // router: one split's B tile (2 boxes)
   constexpr int ELEM = MX ? 1 : 2;
   constexpr int BK = 128 / ELEM;                 // K per stage (128-byte rows)
@@ -285,6 +290,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           // A operand
           if constexpr (!A_MN) {
             tma_load_2d(a_dst, &tmA, fb, kb * BK, t.row0);
+          } else if (p.a3d) {
+            tma_load_3d(a_dst, &tmA, fb, 0, t.krow0 + kb * BK, t.m0 / MN_CHUNK);
           } else {
 #pragma unroll
             for (int i = 0; i < BM / MN_CHUNK; ++i)
@@ -300,12 +307,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 tma_load_2d(b_dst + sp * SPLIT_BYTES + i * MN_CHUNK_BYTES, &tmB, fb, i * MN_CHUNK,
                             sp * p.split_rows + kb * BK);
           } else if constexpr (BLOAD == B_MN) {
+            if (p.b3d) {
+              tma_load_3d(b_dst, &tmB, fb, 0, brow + kb * BK, t.nt * BN / MN_CHUNK);
+            } else {
 #pragma unroll
-            for (int i = 0; i < nbox; ++i)
-              tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * BN + i * MN_CHUNK,
-                          brow + kb * BK);
+              for (int i = 0; i < nbox; ++i)
+                tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * BN + i * MN_CHUNK,
+                            brow + kb * BK);
+            }
           } else if constexpr (BLOAD == B_MN_DUAL_N) {
             constexpr int HALF_CHUNKS = (BN / 2) / MN_CHUNK;
+            if (p.b3d) {
+              tma_load_3d(b_dst, &tmB, fb, 0, brow + kb * BK, t.nt * (BN / 2) / MN_CHUNK);
+              tma_load_3d(b_dst + HALF_CHUNKS * MN_CHUNK_BYTES, &tmB3, fb, 0, brow + kb * BK,
+                          t.nt * (BN / 2) / MN_CHUNK);
+            } else
 #pragma unroll
             for (int i = 0; i < HALF_CHUNKS; ++i) {
               tma_load_2d(b_dst + i * MN_CHUNK_BYTES, &tmB, fb, t.nt * (BN / 2) + i * MN_CHUNK,
@@ -518,7 +534,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               for (int i = 0; i < 32; ++i) av[i] = 0u;
             }
           }
-          constexpr int NB = EpiCfg<MX, EPI>::BOXES;
+          constexpr int NB = Cfg::BOXES;
           uint8_t* buf = stg + (NB > 1 ? (ci & 1) * BOX_BYTES : 0);
           if (lane == 0) {                       // the store that last used `buf` has read it
             if constexpr (NB > 1) bulk_wait_read<1>();
@@ -556,7 +572,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           const uint32_t* g = EARLY ? av + 32 * ci : gl;        // A W1
           const uint32_t* u = EARLY ? av + 64 + 32 * ci : ul;   // A W3
-          constexpr bool ONE_BOX = EpiCfg<MX, EPI>::BOXES == 1;
+          constexpr bool ONE_BOX = Cfg::BOXES == 1;
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
           uint4 hkeep[ONE_BOX ? 4 : 1], gkeep[ONE_BOX ? 4 : 1], ukeep[ONE_BOX ? 4 : 1];
@@ -819,6 +835,31 @@ moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t
   return MOE_OK;
 }
 
+// 3-D view of a row-major [rows, cols] array as (chunk columns, rows, chunk
+// index) with chunk = 128 bytes of a row: box (chunk, box_rows, nchunk) loads
+// nchunk consecutive 128-byte column chunks of box_rows rows in one op, laid
+// out in shared memory chunk after chunk (the MN-major operand layout).
+// Returns false (map unusable) when the driver does not accept the view.
+bool make_map_mn3(CUtensorMap* m, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                  uint32_t box_rows, uint32_t nchunk) {
+#ifdef MOE_GG_NO_3D
+  return false;
+#endif
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t ce = 128 / elem_bytes;
+  if (cols % ce) return false;
+  cuuint64_t dims[3] = {ce, rows, cols / ce};
+  cuuint64_t strides[2] = {cols * (uint64_t)elem_bytes, 128};
+  cuuint32_t box[3] = {(cuuint32_t)ce, box_rows, nchunk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // epilogue box map: [outer, inner] bf16, 32 x 32 box, 64-byte swizzle
 moe_status_t make_out_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
   return make_map(m, base, 2, inner, outer, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -831,7 +872,7 @@ struct Maps {
 template <bool MX, bool A_MN, int BLOAD, int EPI>
 moe_status_t launch(const Maps& m, const Params& p, int max_tiles, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI>;
-  const size_t smem = EpiCfg<MX, EPI>::SMEM;
+  const size_t smem = EpiCfg<MX, EPI, A_MN>::SMEM;
   static bool attr = false;   // one per instantiation
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -894,6 +935,34 @@ moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int
 }
 }  // namespace moe
 
+// Self-test of the bounded pipeline wait: one thread waits on an mbarrier
+// that nothing arrives at; after limit_ns the wait gives up, sets
+// MOE_DEV_TIMEOUT in *status and the kernel returns.
+namespace moe {
+namespace gg {
+__global__ void wait_timeout_selftest_kernel(int32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+}
+}  // namespace gg
+}  // namespace moe
+
+extern "C" moe_status_t moe_selftest_wait_timeout(int32_t* dev_status, uint64_t limit_ns,
+                                                  moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(dev_status != nullptr, "moe_selftest_wait_timeout: null status");
+  MOE_CHECK_ARG(limit_ns > 0 && limit_ns <= 2000000000ull,
+                "moe_selftest_wait_timeout: limit must be in (0, 2 s]");
+  moe::gg::wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(dev_status, limit_ns);
+  MOE_CHECK_LAUNCH("wait_timeout_selftest");
+  return MOE_OK;
+}
+
 extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc,
                                              const void* B, const uint8_t* B_sc, const void* B3,
                                              const uint8_t* B3_sc, const int32_t* poff, int E,
@@ -924,7 +993,8 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
     MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_fwd: N %% 256");
     p.n_tiles = N / BN;
     p.ldc = N;
-    MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    p.b3d = make_map_mn3(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, BN * eb / 128);
+    if (!p.b3d) MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
     MOE_TRY(make_out_map(&m.c, C, N, A_pad_max));
     m.b3 = m.c2 = m.in = m.a;
     const int max_tiles = (A_pad_max / BM) * p.n_tiles;
@@ -939,8 +1009,12 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   p.aux = static_cast<__nv_bfloat16*>(aux);
   p.ld_aux = 2LL * N;
   p.half = N;
-  MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
-  MOE_TRY(make_map(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  p.b3d = make_map_mn3(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, (BN / 2) * eb / 128) &&
+          make_map_mn3(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, (BN / 2) * eb / 128);
+  if (!p.b3d) {
+    MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    MOE_TRY(make_map(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+  }
   MOE_TRY(make_out_map(&m.c, C, N, A_pad_max));
   if (aux) MOE_TRY(make_out_map(&m.c2, aux, 2ULL * N, A_pad_max));
   else m.c2 = m.c;
@@ -1042,8 +1116,10 @@ extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint
   p.ldc = N;
   p.c_expert_stride = (long long)K * N;
   Maps m;
-  MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
-  MOE_TRY(make_map(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  p.a3d = make_map_mn3(&m.a, A, eb, K, A_pad_max, 128 / eb, BM * eb / 128);
+  if (!p.a3d) MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
+  p.b3d = make_map_mn3(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, BN * eb / 128);
+  if (!p.b3d) MOE_TRY(make_map(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
   MOE_TRY(make_out_map(&m.c, dB, N, (uint64_t)E * K));
   if (dB3) MOE_TRY(make_out_map(&m.c2, dB3, N, (uint64_t)E * K));
   else m.c2 = m.c;

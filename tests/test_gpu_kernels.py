@@ -231,3 +231,20 @@ def test_unpermute_sum_and_router_grads(T, d, E, k):
     dWr_o, dxr = oracle.router_backward(f64(x), f64(Wr), idx, dl.cpu().numpy().astype(np.float64))
     assert rel_err(f64(dx), dxs + dxr) < 1e-2
     assert rel_err(dWr.cpu().numpy(), dWr_o) < 1e-4
+
+
+def test_bounded_wait_reports_timeout_and_keeps_the_context_usable():
+    """Failure detection without a fault: a wait that nothing satisfies gives
+    up after 50 ms with MOE_DEV_TIMEOUT; the next launches still work."""
+    import ctypes
+    from mixture_experts_layer_25_b200 import _lib
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    _lib.call("moe_selftest_wait_timeout", ctypes.c_void_p(st.data_ptr()), 50_000_000, stream)
+    torch.cuda.synchronize()
+    assert st.item() == moe.MOE_DEV_TIMEOUT
+    x = moe_inputs.random_bf16((128, 128), 3, device="cuda")
+    q, s = moe.mx_quantize(x, 0)       # the context is still usable
+    torch.cuda.synchronize()
+    c, _ = oracle.mx_quantize_rows(f64(x))
+    np.testing.assert_array_equal(q.cpu().numpy(), c)

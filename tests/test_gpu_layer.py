@@ -34,9 +34,18 @@ def _run(cfg, inp):
     return L, out, dx
 
 
-@pytest.mark.parametrize("variant", ["bf16", "mx", "given", "skewed"])
+@pytest.mark.parametrize("variant", ["bf16", "mx", "given", "skewed", "one_token", "ragged",
+                                     "k_equals_E", "single_expert", "mx_ragged"])
 def test_tiny_layer_element_by_element(variant):
     cfg = moe_inputs.CONFIGS["tiny"]
+    if variant == "one_token":
+        cfg = cfg.with_(T=1)
+    if variant in ("ragged", "mx_ragged"):
+        cfg = cfg.with_(T=333, mx=variant == "mx_ragged")
+    if variant == "k_equals_E":
+        cfg = cfg.with_(T=200, k=8)
+    if variant == "single_expert":
+        cfg = cfg.with_(T=100, E=1, k=1)
     if variant == "mx":
         cfg = cfg.with_(mx=True)
     if variant == "given":
