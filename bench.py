@@ -185,11 +185,12 @@ def _barrier(world):
         dist.barrier()
 
 
-def _traffic(kernel_file):
+def _traffic(kernel_file, workload):
     """DRAM bytes per launch of the grouped GEMM from the committed ncu
-    summary (profiles/traffic_grouped_gemm.md: lines `source_sha256: <hex>`
-    and `dram_bytes_per_launch: <int>`), or None unless that capture was
-    taken on the current source of the kernel."""
+    summary (profiles/traffic_grouped_gemm.md: lines `workload: <name>`,
+    `source_sha256: <hex>` and `dram_bytes_per_launch: <int>`), or None
+    unless that capture was taken on the current source of the kernel and
+    on the workload being timed."""
     p = os.path.join(ROOT, "profiles", "traffic_grouped_gemm.md")
     if not os.path.exists(p):
         return None
@@ -200,6 +201,8 @@ def _traffic(kernel_file):
             fields[k.strip().strip("`- ")] = v.strip().strip("`")
     src = open(os.path.join(ROOT, "mixture_experts_layer_25_b200", "csrc", kernel_file), "rb").read()
     if fields.get("source_sha256") != hashlib.sha256(src).hexdigest():
+        return None
+    if fields.get("workload") != workload:
         return None
     try:
         return int(fields["dram_bytes_per_launch"])
@@ -382,7 +385,7 @@ def run_ours(args):
         except MemoryError:
             cpu = None
 
-    traffic = _traffic("grouped_gemm.cu")
+    traffic = _traffic("grouped_gemm.cu", cfg.name)
     line = {
         "metric": METRIC,
         "value": world * T * args.steps / (ms * 1e-3),
