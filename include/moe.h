@@ -373,6 +373,11 @@ MOE_API moe_status_t moe_layer_fwd(const moe_layer_desc* desc, const moe_layer_w
                            const void* x, void* out, void* ctx, size_t ctx_bytes,
                            int32_t* dev_status, moe_stream_t stream);
 
+/* Backward of the layer (after moe_layer_fwd on the same ctx): dx and the
+ * weight gradients.  In router mode the router's share of dx,
+ * sum_j dl[t,j] W_r[:, topk_idx[t,j]], is added to each permuted row of dXp
+ * by the GEMM1 dgrad epilogue (W_r^T staged in the ctx workspace), so dx is
+ * the plain sum of the k rows of dXp of each token. */
 MOE_API moe_status_t moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_weights* w,
                            const void* x, void* ctx, size_t ctx_bytes, const void* dout,
                            void* dx, moe_layer_grads* grads, int32_t* dev_status,

@@ -47,6 +47,17 @@ moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int
                        int k, float* logits, int32_t* topk, float* gates, int32_t* rank,
                        int32_t* hist, int32_t* status, cudaStream_t s);
 
+// moe_grouped_gemm_dgrad with an optional rank-1 epilogue term (EPI_NONE):
+// dA[row, n] += row_scale[row] * col_vec[e * K + n] on the rows of group e
+moe_status_t grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc, const void* B,
+                                const uint8_t* B_sc, const void* B3, const uint8_t* B3_sc,
+                                const int32_t* poff, int E, int A_pad_max, int N, int K,
+                                int epilogue, const void* aux, void* dA, const float* row_scale,
+                                const float* col_vec, int32_t* dev_status, cudaStream_t s);
+
+// out[cols, rows] = in[rows, cols]^T (fp32)
+moe_status_t transpose_f32(const float* in, int rows, int cols, float* out, cudaStream_t s);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int num_sms();

@@ -106,6 +106,8 @@ struct Params {
   __nv_bfloat16* C2; int n_split;
   __nv_bfloat16* aux; long long ld_aux; int half;
   long long c_expert_stride;
+  // rows-mode STORE: optional rank-1 term C[row, n] += row_scale[row] * col_vec[e * col_ld + n]
+  const float* row_scale; const float* col_vec; int col_ld;
   int k_out;          // wgrad: output rows per expert (K of the weight)
   // dense single-group mode (router): rows [0, dense_rows), no poff
   int dense_rows;
@@ -521,6 +523,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const CUtensorMap* map = &tmC;
         int x0 = n0;
         if (p.wgrad && p.n_split > 0 && n0 >= p.n_split) { map = &tmC2; x0 = n0 - p.n_split; }
+        // rank-1 term (rows mode): this thread's row scale and the expert's column vector
+        const bool r1 = !p.wgrad && p.row_scale != nullptr;
+        const float rs = r1 ? p.row_scale[y0 + r] : 0.f;
+        const float* cvec = r1 ? p.col_vec + (size_t)t.e * p.col_ld + n0 : nullptr;
 #pragma unroll(EARLY ? 4 : 1)
         for (int ci = 0; ci < 4; ++ci) {
           const int c = hc * (BN / 2) + ci * CHUNK;
@@ -543,11 +549,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __uint_as_float(v[8 * j + i]);
+            if (r1) {
+              const float4* cv = reinterpret_cast<const float4*>(cvec + c + 8 * j);
+              const float4 c0 = __ldg(cv), c1 = __ldg(cv + 1);
+              f[0] = fmaf(rs, c0.x, f[0]); f[1] = fmaf(rs, c0.y, f[1]);
+              f[2] = fmaf(rs, c0.z, f[2]); f[3] = fmaf(rs, c0.w, f[3]);
+              f[4] = fmaf(rs, c1.x, f[4]); f[5] = fmaf(rs, c1.y, f[5]);
+              f[6] = fmaf(rs, c1.z, f[6]); f[7] = fmaf(rs, c1.w, f[7]);
+            }
             uint4 w;
-            w.x = bf16x2_bits(__uint_as_float(v[8 * j + 0]), __uint_as_float(v[8 * j + 1]));
-            w.y = bf16x2_bits(__uint_as_float(v[8 * j + 2]), __uint_as_float(v[8 * j + 3]));
-            w.z = bf16x2_bits(__uint_as_float(v[8 * j + 4]), __uint_as_float(v[8 * j + 5]));
-            w.w = bf16x2_bits(__uint_as_float(v[8 * j + 6]), __uint_as_float(v[8 * j + 7]));
+            w.x = bf16x2_bits(f[0], f[1]);
+            w.y = bf16x2_bits(f[2], f[3]);
+            w.z = bf16x2_bits(f[4], f[5]);
+            w.w = bf16x2_bits(f[6], f[7]);
             *reinterpret_cast<uint4*>(buf + sw64(r, j)) = w;
           }
           fence_async_smem();
@@ -1030,7 +1047,21 @@ extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uin
                                                const int32_t* poff, int E, int A_pad_max, int N,
                                                int K, int epilogue, const void* aux, void* dA,
                                                int32_t* dev_status, moe_stream_t stream) {
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return moe::grouped_gemm_dgrad(dt, dC, dC_sc, B, B_sc, B3, B3_sc, poff, E, A_pad_max, N, K,
+                                 epilogue, aux, dA, nullptr, nullptr, dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+// moe_grouped_gemm_dgrad plus an optional rank-1 term in the EPI_NONE
+// epilogue: dA[row, n] += row_scale[row] * col_vec[e * K + n] for the rows
+// of group e (row_scale per padded row, col_vec [E, K] fp32, 16-byte
+// aligned).  The layer backward adds the router's share of dx this way.
+moe_status_t moe::grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc, const void* B,
+                                     const uint8_t* B_sc, const void* B3, const uint8_t* B3_sc,
+                                     const int32_t* poff, int E, int A_pad_max, int N, int K,
+                                     int epilogue, const void* aux, void* dA,
+                                     const float* row_scale, const float* col_vec,
+                                     int32_t* dev_status, cudaStream_t s) {
   const bool mx = dt == MOE_MXFP8;
   MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_dgrad: bad dtype");
   MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_dgrad: E must be in [1, %d]", MAX_E);
@@ -1072,6 +1103,11 @@ extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uin
               : launch<false, false, B_K, EPI_SWIGLU_BWD>(m, p, max_tiles, s);
   }
   MOE_CHECK_ARG(epilogue == MOE_EPI_NONE, "gemm_dgrad: epilogue must be NONE or SWIGLU_BWD");
+  MOE_CHECK_ARG((row_scale == nullptr) == (col_vec == nullptr) && (!col_vec || aligned16(col_vec)),
+                "gemm_dgrad: row_scale and col_vec go together (col_vec 16-byte aligned)");
+  p.row_scale = row_scale;
+  p.col_vec = col_vec;
+  p.col_ld = K;
   p.ldc = K;
   MOE_TRY(make_out_map(&m.c, dA, K, A_pad_max));
   m.c2 = m.in = m.a;

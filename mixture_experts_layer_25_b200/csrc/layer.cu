@@ -230,6 +230,9 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   const bool mx = L->dtype == MOE_MXFP8;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // W_r^T [E, d] (fp32) in the workspace: the GEMM1 dgrad epilogue adds
+  // dl_rows[r] * W_r[:, e] to each row r of expert e
+  float* wrT = router ? static_cast<float*>(c.ws) : nullptr;
   mark(S_COMBINE_BWD, false, s);
   MOE_TRY(moe_combine_bwd(dout, c.Y, c.gates, c.dst, c.offsets, c.poff, T, k, d, E, c.dY, c.dg,
                           router ? c.dl : nullptr, router ? c.dl_rows : nullptr, stream));
@@ -245,9 +248,11 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                    G->dW2, nullptr, dev_status, stream));
     mark(S_WGRAD2, true, s);
     mark(S_DGRAD1, false, s);
-    MOE_TRY(moe_grouped_gemm_dgrad(MOE_BF16, c.dA13, nullptr, w->W1, nullptr, w->W3, nullptr,
-                                   c.poff, E, A, F, d, MOE_EPI_NONE, nullptr, c.dXp, dev_status,
-                                   stream));
+    if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
+    MOE_TRY(moe::grouped_gemm_dgrad(MOE_BF16, c.dA13, nullptr, w->W1, nullptr, w->W3, nullptr, c.poff,
+                               E, A, F, d, MOE_EPI_NONE, nullptr, c.dXp,
+                               router ? c.dl_rows : nullptr, router ? wrT : nullptr, dev_status,
+                               s));
     mark(S_DGRAD1, true, s);
     mark(S_WGRAD1, false, s);
     MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, E, A, d, F,
@@ -275,9 +280,11 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
     MOE_TRY(mx_quantize_dual(c.dA13, A, 2 * F, nrows, c.dA_q, c.dA_s, c.dAT_q, c.dAT_s, stream));
     mark(S_QD1, true, s);
     mark(S_DGRAD1, false, s);
-    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, c.W13t_q, c.W13t_s, c.W13t_q + wq,
-                                   c.W13t_s + wq / 32, c.poff, E, A, F, d, MOE_EPI_NONE, nullptr,
-                                   c.dXp, dev_status, stream));
+    if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
+    MOE_TRY(moe::grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, c.W13t_q, c.W13t_s, c.W13t_q + wq,
+                               c.W13t_s + wq / 32, c.poff, E, A, F, d, MOE_EPI_NONE, nullptr,
+                               c.dXp, router ? c.dl_rows : nullptr, router ? wrT : nullptr,
+                               dev_status, s));
     mark(S_DGRAD1, true, s);
     // Xp down its rows (GEMM1 wgrad)
     mark(S_QW1, false, s);
@@ -289,8 +296,10 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
     mark(S_WGRAD1, true, s);
   }
   mark(S_UNPERMUTE, false, s);
-  MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, c.topk_idx, router ? c.dl : nullptr,
-                            router ? w->Wr : nullptr, T, k, d, E, dx, c.ws, c.ws_bytes, stream));
+  // the router's share of dx, sum_j dl[t, j] W_r[:, e_j], was added to the
+  // rows of dXp by the GEMM1 dgrad epilogue: dx is the plain sum of k rows
+  MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, nullptr, nullptr, nullptr, T, k, d, E, dx, nullptr, 0,
+                            stream));
   mark(S_UNPERMUTE, true, s);
   if (router && G->dWr) {
     mark(S_ROUTER_WGRAD, false, s);

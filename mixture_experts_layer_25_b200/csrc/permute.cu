@@ -413,9 +413,7 @@ extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
     }
     MOE_CHECK_ARG(aligned16(ws), "moe_unpermute_sum: unaligned workspace");
     WrT = static_cast<float*>(ws);
-    dim3 grid((E + 31) / 32, (d + 31) / 32), block(32, 8);
-    transpose_f32_kernel<<<grid, block, 0, s>>>(Wr, d, E, WrT);
-    MOE_CHECK_LAUNCH("transpose Wr");
+    MOE_TRY(transpose_f32(Wr, d, E, WrT, s));
   }
   const int tpb = kBlock / team_threads(d / 8);
   const int blocks = (T + tpb - 1) / tpb;
@@ -424,6 +422,14 @@ extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
       static_cast<uint4*>(dx));
   });
   MOE_CHECK_LAUNCH("unpermute_sum");
+  return MOE_OK;
+}
+
+moe_status_t moe::transpose_f32(const float* in, int rows, int cols, float* out,
+                                cudaStream_t s) {
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32), block(32, 8);
+  transpose_f32_kernel<<<grid, block, 0, s>>>(in, rows, cols, out);
+  MOE_CHECK_LAUNCH("transpose_f32");
   return MOE_OK;
 }
 
