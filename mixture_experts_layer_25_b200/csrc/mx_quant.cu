@@ -119,13 +119,10 @@ __global__ void mx_quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int r
 }
 
 // -------------------------------------------- both axes from one read
-// One warp per (128-row block, 128-column segment), 4 columns per lane, in
-// four 32-row sub-blocks held in registers (all loads in flight at once).
-// Pass 1 over a sub-block accumulates the column amaxes and gives each row's
-// 32-column blocks (8 lanes each) their scale; pass 2 writes both code sets.
 // Scale bytes are packed into the 4-byte words of the tensor-core layout
 // (one word = 4 consecutive K blocks of one MN index): a column's word holds
-// the four sub-blocks, a row's word the four 32-column blocks of the warp.
+// the four 32-row sub-blocks of a 128-row block, a row's word four
+// consecutive 32-column blocks.
 __device__ __forceinline__ void unpack4(const uint2& v, float* f) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
   const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
@@ -138,82 +135,6 @@ __device__ __forceinline__ uint32_t encode4(const float* f, const float* inv) {
   const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(
       make_float2(f[2] * inv[2], f[3] * inv[3]), __NV_SATFINITE, __NV_E4M3);
   return (uint32_t)c0 | ((uint32_t)c1 << 16);
-}
-
-__global__ void __launch_bounds__(128)
-mx_quant_dual_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols,
-                     const int32_t* __restrict__ nrows_dev, uint8_t* __restrict__ codes_r,
-                     uint8_t* __restrict__ scales_r, uint8_t* __restrict__ codes_c,
-                     uint8_t* __restrict__ scales_c) {
-  const int segs = cols / 128;
-  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (w >= (long long)(rows / 128) * segs) return;
-  const int rb4 = (int)(w / segs), seg = (int)(w % segs);
-  const int nrows = nrows_dev ? *nrows_dev : rows;
-  if (rb4 * 128 >= nrows) return;
-  const int col = seg * 128 + lane * 4;
-  uint32_t cword[4] = {0, 0, 0, 0};     // column scale words, byte = sub-block
-  for (int sb = 0; sb < 4; ++sb) {
-    const int r0 = rb4 * 128 + sb * 32;
-    if (r0 >= nrows) break;
-    uint2 raw[32];
-#pragma unroll
-    for (int r = 0; r < 32; ++r)
-      raw[r] = __ldg(reinterpret_cast<const uint2*>(in + (size_t)(r0 + r) * cols + col));
-    float amax[4] = {0, 0, 0, 0};
-    uint32_t rs[32];
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      float f[4];
-      unpack4(raw[r], f);
-      float ra = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        amax[i] = fmaxf(amax[i], fabsf(f[i]));
-        ra = fmaxf(ra, fabsf(f[i]));
-      }
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 1));
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 2));
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 4));
-      rs[r] = scale_byte(ra);
-      // word of row r0+r, K blocks seg*4 .. seg*4+3: bytes of lanes 0, 8, 16, 24
-      const uint32_t b1 = __shfl_down_sync(0xffffffffu, rs[r], 8);
-      const uint32_t b2 = __shfl_down_sync(0xffffffffu, rs[r], 16);
-      const uint32_t b3 = __shfl_down_sync(0xffffffffu, rs[r], 24);
-      if (lane == 0) {
-        const int mn = r0 + r;
-        const size_t off = ((size_t)(mn >> 7) * (cols / 128) + seg) * 512 + (mn & 31) * 16 +
-                           ((mn >> 5) & 3) * 4;
-        *reinterpret_cast<uint32_t*>(scales_r + off) = rs[r] | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      }
-    }
-    float inv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t b = scale_byte(amax[i]);
-      inv[i] = inv_scale(b);
-      cword[i] |= b << (8 * sb);
-    }
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      float f[4];
-      unpack4(raw[r], f);
-      const float ir = inv_scale(rs[r]);
-      const float irr[4] = {ir, ir, ir, ir};
-      *reinterpret_cast<uint32_t*>(codes_c + (size_t)(r0 + r) * cols + col) = encode4(f, inv);
-      *reinterpret_cast<uint32_t*>(codes_r + (size_t)(r0 + r) * cols + col) = encode4(f, irr);
-    }
-  }
-  // column words: MN = col + i, K blocks 4 rb4 .. 4 rb4 + 3 (sub-blocks past
-  // nrows keep byte 0; those rows are never read)
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int mn = col + i;
-    const size_t off = ((size_t)(mn >> 7) * (rows / 128) + rb4) * 512 + (mn & 31) * 16 +
-                       ((mn >> 5) & 3) * 4;
-    *reinterpret_cast<uint32_t*>(scales_c + off) = cword[i];
-  }
 }
 
 // ------------------------------ both axes, TMA-fed persistent variant
