@@ -47,6 +47,9 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (a smaller case of the same layer, e.g. for ncu captures)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E at fixed T, d, k, F (expert-count sweep: same active "
+                         "FLOPs per token, E times the expert weights)")
     return ap.parse_args()
 
 
@@ -223,12 +226,21 @@ def _cfg_dict(cfg, extra):
     return d
 
 
+def _config(args):
+    cfg = moe_inputs.CONFIGS[args.config]
+    if args.tokens:
+        cfg = cfg.with_(T=args.tokens)
+    if args.experts:
+        cfg = cfg.with_(E=args.experts)
+    return cfg
+
+
 # ------------------------------------------------------------ reference arm
 def run_reference(args):
     world, rank, local = _dist()
     if rank != 0:
         return
-    cfg = moe_inputs.CONFIGS[args.config]
+    cfg = _config(args)
     inp = moe_inputs.make_layer_inputs(cfg, "cpu")
     r = OracleRunner(cfg, inp, target_s=4.0)
     for _ in range(args.warmup):
@@ -259,9 +271,7 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    cfg = moe_inputs.CONFIGS[args.config]
-    if args.tokens:
-        cfg = cfg.with_(T=args.tokens)
+    cfg = _config(args)
     peaks, peak_kind = _peaks()
     inp = moe_inputs.make_layer_inputs(cfg, "cuda")
     layer = moe.MoELayer(T=cfg.T, d=cfg.d, E=cfg.E, k=cfg.k, F=cfg.F, W1=inp["W1"], W3=inp["W3"],
@@ -353,6 +363,16 @@ def run_ours(args):
                "frac_of_hbm": round(b / (stage_ms[n] * 1e-3) / 1e9 / hbm, 3),
                "ms": round(stage_ms[n], 4)} for n, b in mem_bytes.items() if n in stage_ms}
 
+    # expert load of this input (read after the timed region): the skewed
+    # workload's imbalance, empty experts and the rows the 128-row group
+    # padding adds to the GEMMs
+    counts = layer.ctx_tensor("counts", (E,), torch.int32).cpu().numpy().astype(np.int64)
+    poff = layer.ctx_tensor("poff", (E + 1,), torch.int32).cpu().numpy().astype(np.int64)
+    load = {"max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 3),
+            "hottest_share": round(float(counts.max() / A), 4),
+            "empty_experts": int((counts == 0).sum()),
+            "padded_rows": int(poff[-1]), "pad_overhead": round(float(poff[-1] / A - 1.0), 4)}
+
     # end to end through the C ABI with host buffers (copies inside)
     e2e = None
     if not args.no_e2e:
@@ -411,7 +431,7 @@ def run_ours(args):
         "gpu_launches": int(launches),
         "clocks": clk,
         "detail": {"stage_ms": {n: round(v, 4) for n, v in stage_ms.items()},
-                   "grouped_gemm_tflops": per_gemm, "memory_bound": mem,
+                   "grouped_gemm_tflops": per_gemm, "memory_bound": mem, "load": load,
                    "gemm_ms_per_step": round(gemm_ms, 4)},
     }
     if rank == 0:

@@ -55,6 +55,13 @@ moe_status_t grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc, co
                                 int epilogue, const void* aux, void* dA, const float* row_scale,
                                 const float* col_vec, int32_t* dev_status, cudaStream_t s);
 
+// moe_grouped_gemm_wgrad whose per-group reduction stops after the group's
+// last real row (offsets: unpadded group offsets, E + 1 ints, or null)
+moe_status_t grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, const void* dC,
+                                const uint8_t* dC_sc, const int32_t* poff, const int32_t* offsets,
+                                int E, int A_pad_max, int K, int N, void* dB, void* dB3,
+                                int32_t* dev_status, cudaStream_t s);
+
 // out[cols, rows] = in[rows, cols]^T (fp32)
 moe_status_t transpose_f32(const float* in, int rows, int cols, float* out, cudaStream_t s);
 

@@ -91,6 +91,7 @@ enum BLoad { B_MN = 0, B_MN_DUAL_N = 1, B_K = 2, B_K_DUAL_K = 3 };
 
 struct Params {
   const int32_t* poff;
+  const int32_t* offsets;   // wgrad: unpadded group offsets (E + 1) or null (use poff)
   int E;
   int wgrad;          // 0: rows mode; 1: weight-gradient mode
   int n_tiles;        // tiles along N
@@ -214,6 +215,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ __align__(8) uint64_t in_bar[NUM_EPI_WARPS][2];
   __shared__ uint32_t tmem_slot;
   __shared__ int poff_s[MAX_E + 1];
+  __shared__ int krows_s[A_MN ? MAX_E : 1];  // wgrad: reduction rows of each group
   __shared__ volatile int abort_flag;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -227,6 +229,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (!p.dense_rows)
     for (int i = threadIdx.x; i <= p.E; i += NUM_THREADS) poff_s[i] = p.poff[i];
+  if constexpr (A_MN) {
+    // a group's K loop stops after its last real row: padding rows are zero,
+    // so whole K blocks of padding are not loaded and the last block issues
+    // only the MMA K steps that hold real rows (the padded count otherwise)
+    for (int e = threadIdx.x; e < p.E; e += NUM_THREADS)
+      krows_s[e] = p.offsets ? p.offsets[e + 1] - p.offsets[e] : p.poff[e + 1] - p.poff[e];
+  }
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
@@ -265,7 +274,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                   : p.dense_rows ? ((p.dense_rows + BM - 1) / BM) * p.n_tiles
                                  : (poff_s[p.E] / BM) * p.n_tiles;
   auto group_kb = [&](const Tile& t) {
-    return p.wgrad ? (poff_s[t.e + 1] - poff_s[t.e]) / BK : t.nkb;
+    if constexpr (A_MN) return (krows_s[t.e] + BK - 1) / BK;
+    else return t.nkb;
   };
 
   if (warp == 0) {
@@ -397,6 +407,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!mbar_wait(&acc_empty[acc], acc_par ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * 256;
+        // K steps of the group's last block that hold real rows (wgrad)
+        int last_ks = KSTEPS;
+        if constexpr (A_MN) last_ks = (krows_s[t.e] - (nkb - 1) * BK + MMA_K - 1) / MMA_K;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, &abort_flag, p.status, kWaitLimitNs)) {
@@ -428,6 +441,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           } else
 #pragma unroll
           for (int ks = 0; ks < KSTEPS; ++ks) {
+            if (A_MN && kb == nkb - 1 && ks >= last_ks) break;
             uint64_t ad, bd;
             if constexpr (!A_MN) ad = smem_desc(sa + ks * 32, 16, 1024, 2);
             else ad = smem_desc(sa + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
@@ -1126,7 +1140,17 @@ extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint
                                                const int32_t* poff, int E, int A_pad_max, int K,
                                                int N, void* dB, void* dB3, int32_t* dev_status,
                                                moe_stream_t stream) {
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return moe::grouped_gemm_wgrad(dt, A, A_sc, dC, dC_sc, poff, nullptr, E, A_pad_max, K, N, dB,
+                                 dB3, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// moe_grouped_gemm_wgrad that stops each group's reduction after its last
+// real row (offsets = the unpadded group offsets, E + 1 ints, or null):
+// whole K blocks of zero padding rows are not loaded or multiplied.
+moe_status_t moe::grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, const void* dC,
+                                     const uint8_t* dC_sc, const int32_t* poff,
+                                     const int32_t* offsets, int E, int A_pad_max, int K, int N,
+                                     void* dB, void* dB3, int32_t* dev_status, cudaStream_t s) {
   const bool mx = dt == MOE_MXFP8;
   MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_wgrad: bad dtype");
   MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_wgrad: E must be in [1, %d]", MAX_E);
@@ -1139,6 +1163,7 @@ extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint
   const int Ncols = dB3 ? 2 * N : N;
   Params p = base_params(poff, E, dev_status);
   p.wgrad = 1;
+  p.offsets = offsets;
   p.m_tiles_w = K / BM;
   p.n_tiles = Ncols / BN;
   p.k_out = K;

@@ -244,8 +244,8 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                    dev_status, stream));
     mark(S_DGRAD2, true, s);
     mark(S_WGRAD2, false, s);
-    MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, E, A, F, d,
-                                   G->dW2, nullptr, dev_status, stream));
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, c.offsets, E,
+                                    A, F, d, G->dW2, nullptr, dev_status, s));
     mark(S_WGRAD2, true, s);
     mark(S_DGRAD1, false, s);
     if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
@@ -255,8 +255,8 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                s));
     mark(S_DGRAD1, true, s);
     mark(S_WGRAD1, false, s);
-    MOE_TRY(moe_grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, E, A, d, F,
-                                   G->dW1, G->dW3, dev_status, stream));
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, c.offsets,
+                                    E, A, d, F, G->dW1, G->dW3, dev_status, s));
     mark(S_WGRAD1, true, s);
   } else {
     const int32_t* nrows = c.poff + E;
@@ -272,8 +272,8 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                    dev_status, stream));
     mark(S_DGRAD2, true, s);
     mark(S_WGRAD2, false, s);
-    MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff, E, A, F,
-                                   d, G->dW2, nullptr, dev_status, stream));
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff,
+                                    c.offsets, E, A, F, d, G->dW2, nullptr, dev_status, s));
     mark(S_WGRAD2, true, s);
     // dA13 along 2F (GEMM1 dgrad) and down its rows (GEMM1 wgrad)
     mark(S_QD1, false, s);
@@ -291,8 +291,8 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
     MOE_TRY(mx_quantize(c.Xp, A, d, 1, c.poff, E, nrows, c.XpT_q, c.XpT_s, stream));
     mark(S_QW1, true, s);
     mark(S_WGRAD1, false, s);
-    MOE_TRY(moe_grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff, E, A, d,
-                                   F, G->dW1, G->dW3, dev_status, stream));
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff,
+                                    c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));
     mark(S_WGRAD1, true, s);
   }
   mark(S_UNPERMUTE, false, s);
