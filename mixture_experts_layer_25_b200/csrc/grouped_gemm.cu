@@ -720,48 +720,78 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         if (!ok) break;
       } else {  // EPI_ROUTER: accumulator = fp32 logits, 128 tokens x E experts
-        constexpr int KT = 8;                          // running top-8 list (k <= 8)
-        int* sel_s = reinterpret_cast<int*>(sStg);     // [128][k] chosen experts
-        int* cnt_s = sel_s + BM * KT;                  // [E] per-expert counters
+        // Both column halves of the epilogue warps scan half of the experts
+        // each for the running top-k of their token; the second half's list
+        // is merged into the first through shared memory.  Ranks inside the
+        // tile: each of four warps counts 32 tokens in order, then a prefix
+        // over the four warps' counts (same result as one pass in token order).
+        constexpr int KT = 8;                                   // k <= 8
+        int* sel_s = reinterpret_cast<int*>(sStg);              // [128][k] chosen experts
+        float* mv_s = reinterpret_cast<float*>(sel_s + BM * KT);  // [128][k] second half's list
+        int* me_s = reinterpret_cast<int*>(mv_s + BM * KT);
+        int* rank_s = reinterpret_cast<int*>(mv_s);            // after the merge: in-warp ranks
+        int* cnt4 = me_s;                                       // after the merge: [4][E] counts
         const int rloc = q * 32 + lane;
         const int row = t.row0 + rloc;
         const bool valid = row < p.dense_rows;
         const int k = p.r_k, E = p.r_E;
-        if (hc == 0) {
-          float bv[KT];
-          int be[KT];
+        const int ep = threadIdx.x - 64;                        // 0..255 over the epilogue warps
+        const int lo = hc ? E / 2 : 0, hi = hc ? E : E / 2;
+        float bv[KT];
+        int be[KT];
 #pragma unroll
-          for (int i = 0; i < KT; ++i) { bv[i] = -INFINITY; be[i] = 0x7fffffff; }
+        for (int i = 0; i < KT; ++i) { bv[i] = -INFINITY; be[i] = 0x7fffffff; }
 #pragma unroll 1
-          for (int c = 0; c < E; c += 32) {
-            uint32_t v[32];
-            tmem_ld32(tbase + c, v);
-            tmem_wait_ld();
-            float L[32];
+        for (int c = lo; c < hi; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c, v);
+          tmem_wait_ld();
+          float L[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              L[i] = __uint_as_float(v[i]) + ((p.r_bias && c + i < E) ? __ldg(p.r_bias + c + i) : 0.f);
-            if (valid && p.r_logits) {
+          for (int i = 0; i < 32; ++i)
+            L[i] = __uint_as_float(v[i]) + ((p.r_bias && c + i < hi) ? __ldg(p.r_bias + c + i) : 0.f);
+          if (valid && p.r_logits) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                if (c + i < E)
-                  *reinterpret_cast<float4*>(p.r_logits + (size_t)row * E + c + i) =
-                      make_float4(L[i], L[i + 1], L[i + 2], L[i + 3]);
+            for (int i = 0; i < 32; i += 4)
+              if (c + i < hi)
+                *reinterpret_cast<float4*>(p.r_logits + (size_t)row * E + c + i) =
+                    make_float4(L[i], L[i + 1], L[i + 2], L[i + 3]);
+          }
+          // experts arrive in increasing order, so a strict '>' keeps the
+          // lower index first among equal logits
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (c + i >= hi) break;
+            float cv = L[i];
+            int ce = c + i;
+            if (cv != cv) { cv = -INFINITY; if (valid) report(p.status, MOE_DEV_NONFINITE); }
+#pragma unroll
+            for (int s2 = 0; s2 < KT; ++s2) {
+              if (cv > bv[s2]) {
+                const float tv = bv[s2]; bv[s2] = cv; cv = tv;
+                const int te = be[s2]; be[s2] = ce; ce = te;
+              }
             }
-            // experts arrive in increasing order, so a strict '>' keeps the
-            // lower index first among equal logits
+          }
+        }
+        if (hc == 1)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (c + i >= E) break;
-              float cv = L[i];
-              int ce = c + i;
-              if (cv != cv) { cv = -INFINITY; if (valid) report(p.status, MOE_DEV_NONFINITE); }
+          for (int j = 0; j < KT; ++j)
+            if (j < k) { mv_s[rloc * k + j] = bv[j]; me_s[rloc * k + j] = be[j]; }
+        named_bar_sync(1, 256);
+        if (hc == 0) {
+          // the second half's experts all have higher indices: a strict '>'
+          // keeps the first half's entry ahead on equal logits
 #pragma unroll
-              for (int s2 = 0; s2 < KT; ++s2) {
-                if (cv > bv[s2]) {
-                  const float tv = bv[s2]; bv[s2] = cv; cv = tv;
-                  const int te = be[s2]; be[s2] = ce; ce = te;
-                }
+          for (int j = 0; j < KT; ++j) {
+            if (j >= k) break;
+            float cv = mv_s[rloc * k + j];
+            int ce = me_s[rloc * k + j];
+#pragma unroll
+            for (int s2 = 0; s2 < KT; ++s2) {
+              if (cv > bv[s2]) {
+                const float tv = bv[s2]; bv[s2] = cv; cv = tv;
+                const int te = be[s2]; be[s2] = ce; ce = te;
               }
             }
           }
@@ -778,26 +808,47 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             sel_s[rloc * k + j] = valid ? be[j] : -1;
           }
-          // rank of each assignment among this tile's assignments to the same
-          // expert, in token order, and the tile's per-expert histogram
-          named_bar_sync(1, 128);
-          for (int e = rloc; e < E; e += 128) cnt_s[e] = 0;
-          named_bar_sync(1, 128);
-          if (ew == 0) {
-            for (int tt = 0; tt < BM; ++tt) {
-              if (lane < k) {
-                const int e = sel_s[tt * k + lane];
-                int rk = -1;
-                if (e >= 0) { rk = cnt_s[e]; cnt_s[e] = rk + 1; }
-                if (t.row0 + tt < p.dense_rows) p.r_rank[(size_t)(t.row0 + tt) * k + lane] = rk;
-              }
-              __syncwarp();
-            }
-          }
-          named_bar_sync(1, 128);
-          for (int e = rloc; e < E; e += 128) p.r_hist[(size_t)(t.row0 / BM) * E + e] = cnt_s[e];
-          named_bar_sync(1, 128);
         }
+        named_bar_sync(1, 256);                  // sel_s complete; the merge buffers are free
+        for (int i = ep; i < 4 * E; i += 256) cnt4[i] = 0;
+        named_bar_sync(1, 256);
+        if (hc == 0) {
+          // warp ew counts tokens [32 ew, 32 ew + 32) in order, lane j = slot j
+          int* cw = cnt4 + ew * E;
+          for (int tt = 0; tt < 32; ++tt) {
+            const int tok = ew * 32 + tt;
+            if (lane < k) {
+              const int e = sel_s[tok * k + lane];
+              int rk = -1;
+              if (e >= 0) { rk = cw[e]; cw[e] = rk + 1; }
+              rank_s[tok * k + lane] = rk;
+            }
+            __syncwarp();
+          }
+        }
+        named_bar_sync(1, 256);
+        for (int e = ep; e < E; e += 256) {      // exclusive prefix over the warps; histogram
+          int run = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int n = cnt4[w * E + e];
+            cnt4[w * E + e] = run;
+            run += n;
+          }
+          p.r_hist[(size_t)(t.row0 / BM) * E + e] = run;
+        }
+        named_bar_sync(1, 256);
+        if (hc == 0 && valid) {
+#pragma unroll
+          for (int j = 0; j < KT; ++j) {
+            if (j >= k) continue;
+            const int e = sel_s[rloc * k + j];
+            int rk = rank_s[rloc * k + j];
+            if (e >= 0) rk += cnt4[(rloc >> 5) * E + e];
+            p.r_rank[(size_t)row * k + j] = rk;
+          }
+        }
+        named_bar_sync(1, 256);                  // shared memory is reused by the next tile
       }
       if constexpr (!EARLY) {
         tc_fence_before();

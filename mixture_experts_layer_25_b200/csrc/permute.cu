@@ -7,6 +7,8 @@
 // vector accesses, each row read once.
 #include <type_traits>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -197,6 +199,123 @@ combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
   }
 }
 
+// Persistent form for rows of at most kBlock 16-byte chunks (d <= 2048):
+// one chunk per thread, and while a token is reduced the loads of the next
+// token's rows (and the routing entries of the one after) are already in
+// flight, so the bytes in flight do not drop between tokens.  Same results
+// as combine_bwd_kernel (same per-thread arithmetic and reduction order).
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock, 3)
+combine_bwd_pf_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
+                      const float* __restrict__ gates, const int32_t* __restrict__ dst,
+                      const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
+                      int k, int d8, int tok_blocks, uint4* __restrict__ dY, float* __restrict__ dg,
+                      float* __restrict__ dl, float* __restrict__ dl_rows) {
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY);
+    return;
+  }
+  __shared__ float red[kBlock / 32][kMaxK];
+  const int tpt = team_threads(d8);
+  const int tpb = kBlock / tpt;
+  const int team = threadIdx.x / tpt, lt = threadIdx.x % tpt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stride = tok_blocks * tpb;
+  const bool has_c = lt < d8;
+  auto load_meta = [&](int t, int* r, float* g) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      const bool on = t < T && j < k;
+      r[j] = on ? dst[(size_t)t * k + j] : -1;
+      g[j] = on ? gates[(size_t)t * k + j] : 0.f;
+    }
+  };
+  auto load_rows = [&](int t, const int* r, uint4& dv, uint4* yv) {
+    if (t < T && has_c) {
+      dv = ldg_stream(dout + (size_t)t * d8 + lt);
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (r[j] >= 0) yv[j] = ldg_stream(Y + (size_t)r[j] * d8 + lt);
+    }
+  };
+  int base = blockIdx.x * tpb;
+  int r[kMaxK], rn[kMaxK];
+  float g[kMaxK], gn[kMaxK];
+  uint4 dv = make_uint4(0, 0, 0, 0), yv[kMaxK];
+  load_meta(base + team, r, g);
+  load_rows(base + team, r, dv, yv);
+  load_meta(base + stride + team, rn, gn);
+  for (; base < T; base += stride) {            // block-uniform trip count
+    const int t = base + team;
+    const bool live = t < T;
+    // next token: its rows now, the routing entries of the one after
+    uint4 dvn = make_uint4(0, 0, 0, 0), yvn[kMaxK];
+    load_rows(t + stride, rn, dvn, yvn);
+    int rn2[kMaxK];
+    float gn2[kMaxK];
+    load_meta(t + 2 * stride, rn2, gn2);
+
+    float dot[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) dot[j] = 0.f;
+    if (live && has_c) {
+      float fd[8];
+      unpack8(dv, fd);
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (r[j] < 0) continue;
+        float fy[8], sc[8];
+        unpack8(yv[j], fy);
+        float sdot = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          sdot = fmaf(fd[i], fy[i], sdot);
+          sc[i] = g[j] * fd[i];
+        }
+        dot[j] += sdot;
+        dY[(size_t)r[j] * d8 + lt] = pack8(sc);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (j < k) dot[j] = warp_sum(dot[j]);
+    if (lane == 0)
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (j < k) red[warp][j] = dot[j];
+    __syncthreads();
+    if (live && lt == 0) {
+      const int w0 = warp, nw = tpt / 32;
+      float gs = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j >= k) continue;
+        float sum = 0.f;
+        for (int w = 0; w < nw; ++w) sum += red[w0 + w][j];
+        dot[j] = sum;
+        gs = fmaf(g[j], sum, gs);
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j) {
+        if (j >= k) continue;
+        dg[(size_t)t * k + j] = dot[j];
+        if (dl) {
+          const float v = g[j] * (dot[j] - gs);
+          dl[(size_t)t * k + j] = v;
+          if (dl_rows && r[j] >= 0) dl_rows[r[j]] = v;
+        }
+      }
+    }
+    __syncthreads();                            // red is reused by the next token
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      r[j] = rn[j]; g[j] = gn[j]; yv[j] = yvn[j];
+      rn[j] = rn2[j]; gn[j] = gn2[j];
+    }
+    dv = dvn;
+  }
+}
+
 // ------------------------------------------------- dispatch backward (dx)
 __global__ void transpose_f32_kernel(const float* __restrict__ in, int rows, int cols,
                                      float* __restrict__ out) {
@@ -381,10 +500,23 @@ extern "C" moe_status_t moe_combine_bwd(const void* dout, const void* Y, const f
   MOE_CHECK_ARG(aligned16(dout) && aligned16(Y) && aligned16(dY), "moe_combine_bwd: unaligned");
   const int tpb = kBlock / team_threads(d / 8);
   const int tok_blocks = (T + tpb - 1) / tpb;
-  dispatch_k(k, [&](auto KM) {
-    combine_bwd_kernel<decltype(KM)::value><<<tok_blocks + E, kBlock, 0, s>>>(static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff, T,
-      k, d / 8, tok_blocks, static_cast<uint4*>(dY), dg, dl, dl_rows);
-  });
+  if (d / 8 <= kBlock && k <= 4) {
+    // persistent: three resident blocks per SM walk the tokens (80 registers
+    // at k <= 4; larger k would spill with two tokens' rows in registers)
+    const int pblocks = std::min(tok_blocks, 3 * num_sms());
+    auto go = [&](auto KM) {
+      combine_bwd_pf_kernel<decltype(KM)::value><<<pblocks + E, kBlock, 0, s>>>(
+          static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff,
+          T, k, d / 8, pblocks, static_cast<uint4*>(dY), dg, dl, dl_rows);
+    };
+    if (k <= 2) go(std::integral_constant<int, 2>{});
+    else go(std::integral_constant<int, 4>{});
+  } else {
+    dispatch_k(k, [&](auto KM) {
+      combine_bwd_kernel<decltype(KM)::value><<<tok_blocks + E, kBlock, 0, s>>>(static_cast<const uint4*>(dout), static_cast<const uint4*>(Y), gates, dst, offsets, poff, T,
+        k, d / 8, tok_blocks, static_cast<uint4*>(dY), dg, dl, dl_rows);
+    });
+  }
   MOE_CHECK_LAUNCH("combine_bwd");
   return MOE_OK;
 }

@@ -184,8 +184,13 @@ def test_mx_quantize_dual_equals_both_axes(R, C):
     np.testing.assert_array_equal(scales_to_plain(sc, R, C, 1), s1)
 
 
-@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (257, 2048, 32, 4), (64, 6144, 384, 8)])
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (257, 2048, 32, 4), (64, 6144, 384, 8),
+                                     (3000, 1024, 16, 3), (5000, 2048, 64, 4), (1, 2048, 8, 4)])
 def test_combine_and_its_backward(T, d, E, k):
+    """Gate-weighted combine and its backward against the oracle; the cases
+    cover both backward kernels (persistent with prefetch for d <= 2048 and
+    k <= 4, one token per team otherwise), several persistent sweeps
+    (T = 3000, 5000), two tokens per block (d = 1024), k = 3 and T = 1."""
     idx, gates, meta = _meta_for(T, E, k, 5)
     A = meta["A_pad_max"]
     Y = moe_inputs.random_bf16((A, d), 9, device="cuda")
