@@ -115,6 +115,82 @@ combine_kernel(const uint4* __restrict__ Y, const float* __restrict__ gates,
   }
 }
 
+// Persistent form of the k-row gather-sum (combine with gates, the dx sum
+// without) for rows of at most kBlock 16-byte chunks and k <= 4: each team
+// walks tokens with a stride of the whole grid, and the next token's k rows
+// (and the routing entries of the one after) are loaded while the current
+// token is summed.  Same per-element arithmetic as combine_kernel /
+// unpermute_sum_kernel.
+template <int kMaxK, bool kGated>
+__global__ void __launch_bounds__(kBlock, 3)
+gather_sum_pf_kernel(const uint4* __restrict__ rows, const float* __restrict__ gates,
+                     const int32_t* __restrict__ dst, int T, int k, int d8, int nblocks,
+                     uint4* __restrict__ out) {
+  const int tpt = team_threads(d8);
+  const int tpb = kBlock / tpt;
+  const int team = threadIdx.x / tpt, lt = threadIdx.x % tpt;
+  if (lt >= d8) return;                      // no block-wide barriers below
+  const int stride = nblocks * tpb;
+  auto load_meta = [&](int t, int* r, float* g) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      const bool on = t < T && j < k;
+      r[j] = on ? dst[(size_t)t * k + j] : -1;
+      g[j] = (on && kGated) ? gates[(size_t)t * k + j] : 1.f;
+    }
+  };
+  auto load_rows = [&](const int* r, uint4* v) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (r[j] >= 0) v[j] = ldg_stream(rows + (size_t)r[j] * d8 + lt);
+  };
+  int t = blockIdx.x * tpb + team;
+  int r[kMaxK], rn[kMaxK];
+  float g[kMaxK], gn[kMaxK];
+  uint4 v[kMaxK];
+  load_meta(t, r, g);
+  load_rows(r, v);
+  load_meta(t + stride, rn, gn);
+  for (; t < T; t += stride) {
+    uint4 vn[kMaxK];
+    load_rows(rn, vn);
+    int rn2[kMaxK];
+    float gn2[kMaxK];
+    load_meta(t + 2 * stride, rn2, gn2);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      if (r[j] < 0) continue;
+      float f[8];
+      unpack8(v[j], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = kGated ? fmaf(g[j], f[i], acc[i]) : acc[i] + f[i];
+    }
+    out[(size_t)t * d8 + lt] = pack8(acc);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      r[j] = rn[j]; g[j] = gn[j]; v[j] = vn[j];
+      rn[j] = rn2[j]; gn[j] = gn2[j];
+    }
+  }
+}
+
+// launch the persistent gather-sum if it applies (d <= 2048, k <= 4)
+template <bool kGated>
+bool launch_gather_sum_pf(const void* rows, const float* gates, const int32_t* dst, int T, int k,
+                          int d8, void* out, cudaStream_t s) {
+  if (d8 > kBlock || k > 4) return false;
+  const int tpb = kBlock / team_threads(d8);
+  const int nblocks = std::min((T + tpb - 1) / tpb, 3 * num_sms());
+  auto go = [&](auto KM) {
+    gather_sum_pf_kernel<decltype(KM)::value, kGated><<<nblocks, kBlock, 0, s>>>(
+        static_cast<const uint4*>(rows), gates, dst, T, k, d8, nblocks, static_cast<uint4*>(out));
+  };
+  if (k <= 2) go(std::integral_constant<int, 2>{});
+  else go(std::integral_constant<int, 4>{});
+  return true;
+}
+
 // ------------------------------------------------------- combine backward
 template <int kMaxK>
 __global__ void __launch_bounds__(kBlock)
@@ -479,10 +555,13 @@ extern "C" moe_status_t moe_unpermute_combine(const void* Y, const float* gates,
                 "moe_unpermute_combine: null or unaligned pointer");
   const int tpb = kBlock / team_threads(d / 8);
   const int blocks = (T + tpb - 1) / tpb;
-  dispatch_k(k, [&](auto KM) {
-    combine_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(Y), gates, dst,
-                                                        T, k, d / 8, static_cast<uint4*>(out));
-  });
+  const bool pf = gates ? launch_gather_sum_pf<true>(Y, gates, dst, T, k, d / 8, out, s)
+                        : launch_gather_sum_pf<false>(Y, nullptr, dst, T, k, d / 8, out, s);
+  if (!pf)
+    dispatch_k(k, [&](auto KM) {
+      combine_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(Y), gates, dst,
+                                                          T, k, d / 8, static_cast<uint4*>(out));
+    });
   MOE_CHECK_LAUNCH("combine");
   return MOE_OK;
 }
@@ -549,10 +628,11 @@ extern "C" moe_status_t moe_unpermute_sum(const void* dXp, const int32_t* dst,
   }
   const int tpb = kBlock / team_threads(d / 8);
   const int blocks = (T + tpb - 1) / tpb;
-  dispatch_k(k, [&](auto KM) {
-    unpermute_sum_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(dXp), dst, topk_idx, dl, WrT, T, k, d / 8, E,
-      static_cast<uint4*>(dx));
-  });
+  if (WrT || !launch_gather_sum_pf<false>(dXp, nullptr, dst, T, k, d / 8, dx, s))
+    dispatch_k(k, [&](auto KM) {
+      unpermute_sum_kernel<decltype(KM)::value><<<blocks, kBlock, 0, s>>>(static_cast<const uint4*>(dXp), dst, topk_idx, dl, WrT, T, k, d / 8, E,
+        static_cast<uint4*>(dx));
+    });
   MOE_CHECK_LAUNCH("unpermute_sum");
   return MOE_OK;
 }

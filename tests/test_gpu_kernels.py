@@ -214,7 +214,8 @@ def test_combine_and_its_backward(T, d, E, k):
     np.testing.assert_allclose(dl_rows.cpu().numpy()[dst], dl.cpu().numpy(), rtol=0, atol=0)
 
 
-@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (300, 2048, 128, 4)])
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (300, 2048, 128, 4), (5000, 2048, 64, 4),
+                                     (777, 1024, 16, 3), (1, 2048, 8, 4), (96, 6144, 384, 8)])
 def test_unpermute_sum_and_router_grads(T, d, E, k):
     idx, gates, meta = _meta_for(T, E, k, 6)
     A = meta["A_pad_max"]
