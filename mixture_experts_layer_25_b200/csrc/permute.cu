@@ -80,6 +80,47 @@ permute_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
   }
 }
 
+// Persistent form for rows of at most kBlock 16-byte chunks and k <= 4: the
+// next token's row and routing entries are loaded while the current row is
+// written to its k slots.  Blocks from nblocks on zero the pad rows.
+template <int kMaxK>
+__global__ void __launch_bounds__(kBlock, 3)
+permute_pf_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
+                  const int32_t* __restrict__ offsets, const int32_t* __restrict__ poff, int T,
+                  int k, int d8, int nblocks, uint4* __restrict__ Xp) {
+  if ((int)blockIdx.x >= nblocks) {
+    zero_pad_rows(offsets, poff, blockIdx.x - nblocks, d8, Xp);
+    return;
+  }
+  const int tpt = team_threads(d8);
+  const int tpb = kBlock / tpt;
+  const int team = threadIdx.x / tpt, lt = threadIdx.x % tpt;
+  if (lt >= d8) return;                      // no block-wide barriers below
+  const int stride = nblocks * tpb;
+  auto load_meta = [&](int t, int* r) {
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) r[j] = (t < T && j < k) ? dst[(size_t)t * k + j] : -1;
+  };
+  int t = blockIdx.x * tpb + team;
+  int r[kMaxK];
+  uint4 v = make_uint4(0, 0, 0, 0);
+  load_meta(t, r);
+  if (t < T) v = ldg_stream(x + (size_t)t * d8 + lt);
+  for (; t < T; t += stride) {
+    const int tn = t + stride;
+    int rn[kMaxK];
+    load_meta(tn, rn);
+    uint4 vn = make_uint4(0, 0, 0, 0);
+    if (tn < T) vn = ldg_stream(x + (size_t)tn * d8 + lt);
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (r[j] >= 0) Xp[(size_t)r[j] * d8 + lt] = v;
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) r[j] = rn[j];
+    v = vn;
+  }
+}
+
 // ------------------------------------------------------------------ combine
 template <int kMaxK>
 __global__ void __launch_bounds__(kBlock)
@@ -538,6 +579,18 @@ extern "C" moe_status_t moe_permute(const void* x, const int32_t* dst, const int
   if (Xq) return moe_permute_mx_launch(x, dst, offsets, poff, T, k, d, E, A_pad_max, Xp, Xq, Xs, s);
   const int tpb = kBlock / team_threads(d / 8);
   const int tok_blocks = (T + tpb - 1) / tpb;
+  if (d / 8 <= kBlock && k <= 4) {
+    const int nblocks = std::min(tok_blocks, 3 * num_sms());
+    auto go = [&](auto KM) {
+      permute_pf_kernel<decltype(KM)::value><<<nblocks + E, kBlock, 0, s>>>(
+          static_cast<const uint4*>(x), dst, offsets, poff, T, k, d / 8, nblocks,
+          static_cast<uint4*>(Xp));
+    };
+    if (k <= 2) go(std::integral_constant<int, 2>{});
+    else go(std::integral_constant<int, 4>{});
+    MOE_CHECK_LAUNCH("permute");
+    return MOE_OK;
+  }
   dispatch_k(k, [&](auto KM) {
     permute_kernel<decltype(KM)::value><<<tok_blocks + E, kBlock, 0, s>>>(static_cast<const uint4*>(x), dst, offsets, poff, T, k, d / 8, tok_blocks,
       static_cast<uint4*>(Xp));

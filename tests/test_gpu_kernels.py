@@ -115,7 +115,8 @@ def _meta_for(T, E, k, seed):
     return idx, gates, meta
 
 
-@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (333, 2048, 64, 4), (50, 6144, 384, 8)])
+@pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (333, 2048, 64, 4), (50, 6144, 384, 8),
+                                     (5000, 2048, 128, 4), (700, 1024, 16, 3), (1, 2048, 8, 4)])
 def test_permute_bit_exact_and_pad_rows_zero(T, d, E, k):
     idx, gates, meta = _meta_for(T, E, k, 3)
     x = moe_inputs.random_bf16((T, d), 7, device="cuda")
