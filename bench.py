@@ -115,16 +115,22 @@ class ClockSampler:
 # ------------------------------------------------------------ CPU baseline
 def _oracle_step(oracle, cfg, x, dout, W, Wr, b, topk=None, gates=None):
     if topk is None:
-        ctx = oracle.layer_forward(x, *W, cfg.k, Wr=Wr, bias=b)
+        ctx = oracle.layer_forward(x, *W, cfg.k, Wr=Wr, bias=b, mx=cfg.mx)
     else:
-        ctx = oracle.layer_forward(x, *W, cfg.k, topk_idx=topk, gates=gates)
+        ctx = oracle.layer_forward(x, *W, cfg.k, topk_idx=topk, gates=gates, mx=cfg.mx)
     oracle.layer_backward(ctx, dout)
 
 
 class OracleRunner:
-    """The CPU oracle, as it stands, on a token sample of the workload."""
+    """The CPU oracle, as it stands, on a token sample of the workload.
 
-    def __init__(self, cfg, inp, target_s):
+    Router workloads: the first n tokens with all experts.  Given-routing
+    workloads (the trillion shape): the first n tokens with only the experts
+    they are routed to (expert ids renumbered in order), which gives the same
+    per-token results, so that the fp64 weights stay within `mem_limit`
+    bytes of host memory (all 384 experts would need 116 GB)."""
+
+    def __init__(self, cfg, inp, target_s, mem_limit=8e9):
         import oracle
         from threadpoolctl import threadpool_limits
         self.oracle = oracle
@@ -132,37 +138,60 @@ class OracleRunner:
         self.cores = len(os.sched_getaffinity(0))
         self._limit = threadpool_limits(self.cores)
         f64 = moe_inputs.to_f64
-        self.W = [inp[n].to(torch.float64).cpu().numpy() if inp[n].is_cuda else f64(inp[n])
-                  for n in ("W1", "W3", "W2")]
+        self.given = cfg.routing != "router"
+        self.Wsrc = [inp[n] for n in ("W1", "W3", "W2")]
+        self.W = None if self.given else [
+            w.to(torch.float64).cpu().numpy() if w.is_cuda else f64(w) for w in self.Wsrc]
         self.x = f64(inp["x"]); self.dout = f64(inp["dout"])
         self.Wr = f64(inp["Wr"]); self.b = f64(inp["bias"])
-        self.topk = None if cfg.routing == "router" else inp["topk_idx"].cpu().numpy()
-        self.gates = None if cfg.routing == "router" else f64(inp["gates"])
+        self.topk = inp["topk_idx"].cpu().numpy() if self.given else None
+        self.gates = f64(inp["gates"]) if self.given else None
+        self.e_used = cfg.E
+        per_expert = 3 * cfg.d * cfg.F * 8
         # grow the sample (doubling) until one step takes about target_s / 2
         # or more; the groups are padded to 128 rows, so the cost is far from
         # linear in the sample at small sizes
-        n = min(cfg.T, 256)
+        n = 1 if self.given else min(cfg.T, 256)
         while True:
+            self._prepare(n)
             t = self._time(n)
+            nxt = min(cfg.T, 2 * n)
             if t >= target_s / 2 or n >= cfg.T:
                 break
-            n = min(cfg.T, 2 * n)
+            if self.given and len(np.unique(self.topk[:nxt])) * per_expert > mem_limit:
+                break
+            n = nxt
         self.n, self.last_t = n, t
+
+    def _prepare(self, n):
+        """fp64 weights of the experts the first n tokens use (given routing)."""
+        if not self.given:
+            self._Wn, self._topk_n = self.W, None
+            return
+        used = np.unique(self.topk[:n])
+        remap = np.full(self.cfg.E, -1, np.int64)
+        remap[used] = np.arange(len(used))
+        sel = torch.from_numpy(used).to(self.Wsrc[0].device)
+        self._Wn = [w.index_select(0, sel).to(torch.float64).cpu().numpy() for w in self.Wsrc]
+        self._topk_n = remap[self.topk[:n]].astype(np.int32)
+        self.e_used = len(used)
 
     def _time(self, n):
         sl = slice(0, n)
         t0 = time.perf_counter()
-        _oracle_step(self.oracle, self.cfg, self.x[sl], self.dout[sl], self.W, self.Wr, self.b,
-                     None if self.topk is None else self.topk[sl],
-                     None if self.gates is None else self.gates[sl])
+        _oracle_step(self.oracle, self.cfg, self.x[sl], self.dout[sl], self._Wn, self.Wr, self.b,
+                     self._topk_n, None if self.gates is None else self.gates[sl])
         return time.perf_counter() - t0
 
     def step(self):
         return self._time(self.n)
 
     def describe(self):
+        experts = (f"the {self.e_used} of {self.cfg.E} experts they are routed to"
+                   if self.given else f"all {self.cfg.E} experts")
         return (f"first {self.n} of {self.cfg.T} tokens of the workload, full fwd+bwd of the fp64 "
-                f"NumPy oracle (all {self.cfg.E} experts, groups padded to 128 rows)")
+                f"NumPy oracle ({experts}, groups padded to 128 rows"
+                f"{', MXFP8 operands' if self.cfg.mx else ''})")
 
 
 # ----------------------------------------------------------------- helpers
