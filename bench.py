@@ -271,7 +271,11 @@ def run_reference(args):
         return
     cfg = _config(args)
     inp = moe_inputs.make_layer_inputs(cfg, "cpu")
-    r = OracleRunner(cfg, inp, target_s=4.0)
+    # each step is a token sample sized so that the whole run takes about
+    # four minutes (at most ~15 s per step, the sample of the cpu_baseline).
+    # Small samples run slower per token: every expert group is padded to 128
+    # rows, a fixed cost of E * 128 rows whatever the sample.
+    r = OracleRunner(cfg, inp, target_s=min(15.0, 240.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         r.step()
     t = 0.0
