@@ -271,6 +271,31 @@ MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t
                                     int A_pad_max, int K, int N, void* dB, void* dB3,
                                     int32_t* dev_status, moe_stream_t stream);
 
+/* Grouped GEMM with the tokens on the MMA's N side, BF16 (Olmo-core 3
+ * オープン混合エキスパート学習インフラストラクチャ, "ルーティングと計算の最適化": the
+ * expert matmuls as one grouped GEMM).  The weights form the 128-row M side
+ * of each tile; group e's real rows (offsets[e+1] - offsets[e], or all of
+ * its padded rows when offsets is NULL) are split evenly into token blocks
+ * of at most 256 (multiples of 32) on the N side, so padding rows are not
+ * multiplied; output rows from the last real row to poff[e+1] are written
+ * as zeros.  Same results as moe_grouped_gemm_fwd / _dgrad (BF16) up to
+ * rounding, except that in the SwiGLU form h uses the bf16-rounded X W3.
+ *   epilogue MOE_EPI_SWIGLU: X [A_pad_max, K], W and W3 [E, K, N] (N % 64
+ *     == 0) -> C = h [A_pad_max, N], aux = [X W | X W3] [A_pad_max, 2N].
+ *   MOE_EPI_NONE, w_kmajor = 0: C = X W, W [E, K, N], W3 NULL (N % 128).
+ *   MOE_EPI_NONE, w_kmajor = 1: W (and W3) [E, N, Kw], K = Kw (W3 NULL) or
+ *     2 Kw: C = X[:, :Kw] W^T (+ X[:, Kw:] W3^T), plus, when row_scale and
+ *     col_vec are given, row_scale[row] * col_vec[e * N + n] (fp32,
+ *     col_vec 16-byte aligned).  N % 128 == 0.
+ * K % 64 == 0; E <= 1024; A_pad_max % 128 == 0.  Pointers are device
+ * memory owned by the caller; returns MOE_ERR_INVALID_ARG on bad shapes. */
+MOE_API moe_status_t moe_grouped_gemm_tn(int epilogue, const void* X, const void* W,
+                                         const void* W3, int w_kmajor, const int32_t* poff,
+                                         const int32_t* offsets, int E, int A_pad_max, int N,
+                                         int K, void* C, void* aux, const float* row_scale,
+                                         const float* col_vec, int32_t* dev_status,
+                                         moe_stream_t stream);
+
 /* Self-test of the failure detection the grouped GEMM relies on: a kernel
  * waits on an mbarrier that nothing arrives at, gives up after limit_ns
  * (at most 2 s), ORs MOE_DEV_TIMEOUT into *dev_status and returns, leaving

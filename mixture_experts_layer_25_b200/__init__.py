@@ -159,6 +159,24 @@ def moe_grouped_gemm_wgrad(A, dC, poff, E: int, *, split: bool = False, A_sc=Non
     return (dB, dB3) if split else dB
 
 
+def moe_grouped_gemm_tn(X, W, poff, E: int, *, epilogue=MOE_EPI_NONE, W3=None,
+                        w_kmajor: bool = False, offsets=None, row_scale=None, col_vec=None,
+                        status=None, stream=None):
+    """Tokens-N grouped GEMM (BF16): only the real rows of each group are
+    multiplied (``offsets``), the padding rows of the output are zeros.
+    SwiGLU: returns (h, aux); otherwise C."""
+    Ap, K = X.shape
+    N = W.shape[1] if w_kmajor else W.shape[2]
+    C = torch.empty((Ap, N), dtype=torch.bfloat16, device=X.device)
+    aux = None
+    if epilogue == MOE_EPI_SWIGLU:
+        aux = torch.empty((Ap, 2 * N), dtype=torch.bfloat16, device=X.device)
+    _lib.call("moe_grouped_gemm_tn", epilogue, _p(X), _p(W), _p(W3), 1 if w_kmajor else 0,
+              _p(poff), _p(offsets), E, Ap, N, K, _p(C), _p(aux), _p(row_scale), _p(col_vec),
+              _p(status), _s(stream))
+    return (C, aux) if epilogue == MOE_EPI_SWIGLU else C
+
+
 # ---------------------------------------------------- combine and backward
 def moe_unpermute_combine(Y, gates, dst, *, stream=None):
     T, k = dst.shape

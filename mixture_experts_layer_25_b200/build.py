@@ -16,7 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["common.cu", "route.cu", "permute.cu", "mx_quant.cu", "grouped_gemm.cu", "layer.cu"]
+SOURCES = ["common.cu", "route.cu", "permute.cu", "mx_quant.cu", "grouped_gemm.cu",
+           "grouped_gemm_tn.cu", "layer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -62,6 +62,19 @@ moe_status_t grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, cons
                                 int E, int A_pad_max, int K, int N, void* dB, void* dB3,
                                 int32_t* dev_status, cudaStream_t s);
 
+// Tokens-N grouped GEMM (BF16; grouped_gemm_tn.cu): weights on the MMA's M
+// side, an expert's real rows split evenly over token blocks of <= 256 on
+// the N side, padding rows after the last real row written as zeros.
+// epilogue MOE_EPI_SWIGLU: C = h [A_pad, N], aux = [XW | XW3]; MOE_EPI_NONE:
+// C = X W (MN-major weights [E, K, N]) or, with w_kmajor, C = X[:, :K/2] W^T
+// + X[:, K/2:] W3^T (weights [E, N, K/2]; W3 null: C = X W^T) plus the
+// optional rank-1 term row_scale[row] * col_vec[e * N + n].  offsets: the
+// unpadded group offsets, or null (every padded row counts as real).
+moe_status_t gemm_tn(int epilogue, const void* X, const void* W, const void* W3, int w_kmajor,
+                     const int32_t* poff, const int32_t* offsets, int E, int A_pad_max, int N,
+                     int K, void* C, void* aux, const float* row_scale, const float* col_vec,
+                     int32_t* dev_status, cudaStream_t s);
+
 // out[cols, rows] = in[rows, cols]^T (fp32)
 moe_status_t transpose_f32(const float* in, int rows, int cols, float* out, cudaStream_t s);
 

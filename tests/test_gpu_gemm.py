@@ -198,3 +198,89 @@ def test_fwd_full_width_sampled_experts():
         H1 = Xe @ f64(W1[e]); H3 = Xe @ f64(W3[e])
         assert rel_err(f64(h[a:b]), oracle.silu(H1) * H3) < 1e-2
         assert rel_err(f64(aux[a:b, :F]), H1) < 1e-2
+
+
+# ------------------------------------------------ tokens-N grouped GEMM (BF16)
+# groups with 1, 2 and 3 token blocks, a block of 5 rows (MMA N = 16), and a
+# last block whose padding runs past 256 rows (385 rows: blocks of 224 and 161)
+COUNTS_TN = [0, 5, 300, 128, 1, 0, 513, 700, 256, 257, 385]
+
+
+def _tn_setup(counts, cols, seed, garbage):
+    poff, A, real = _groups(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    X = moe_inputs.random_bf16((A, cols), seed, device="cuda")
+    # padding rows hold garbage: they must be neither multiplied nor copied
+    X[torch.from_numpy(~real).cuda()] = 100.0 if garbage else 0.0
+    return poff, offs, A, real, X
+
+
+def _pad_rows(poff, real):
+    P = int(poff[-1])
+    return ~real[:P]
+
+
+@pytest.mark.parametrize("with_offsets", [True, False])
+def test_tn_fwd_swiglu(with_offsets):
+    E, K, F = len(COUNTS_TN), 256, 384
+    poff, offs, A, real, X = _tn_setup(COUNTS_TN, K, 21, with_offsets)
+    W1, W3 = _w(E, K, F, 22), _w(E, K, F, 23)
+    tp, to = torch.from_numpy(poff).cuda(), torch.from_numpy(offs).cuda()
+    h, aux = moe.moe_grouped_gemm_tn(X, W1, tp, E, epilogue=moe.MOE_EPI_SWIGLU, W3=W3,
+                                     offsets=to if with_offsets else None)
+    torch.cuda.synchronize()
+    P = int(poff[-1])
+    Xd = f64(X)
+    Xd[~real] = 0.0
+    H1 = oracle.grouped_matmul(Xd, f64(W1), poff)
+    H3 = oracle.grouped_matmul(Xd, f64(W3), poff)
+    r = real[:P]
+    assert rel_err(f64(aux[:P, :F])[r], H1[:P][r]) < 1e-2
+    assert rel_err(f64(aux[:P, F:])[r], H3[:P][r]) < 1e-2
+    assert rel_err(f64(h[:P])[r], (oracle.silu(H1) * H3)[:P][r]) < 1e-2
+    pad = _pad_rows(poff, real)
+    assert np.all(f64(h[:P])[pad] == 0) and np.all(f64(aux[:P])[pad] == 0)
+
+
+def test_tn_fwd_plain():
+    E, K, N = len(COUNTS_TN), 512, 512
+    poff, offs, A, real, X = _tn_setup(COUNTS_TN, K, 24, True)
+    W = _w(E, K, N, 25)
+    tp, to = torch.from_numpy(poff).cuda(), torch.from_numpy(offs).cuda()
+    C = moe.moe_grouped_gemm_tn(X, W, tp, E, offsets=to)
+    torch.cuda.synchronize()
+    P = int(poff[-1])
+    Xd = f64(X)
+    Xd[~real] = 0.0
+    ref = oracle.grouped_matmul(Xd, f64(W), poff)
+    r = real[:P]
+    assert rel_err(f64(C[:P])[r], ref[:P][r]) < 1e-2
+    assert np.all(f64(C[:P])[_pad_rows(poff, real)] == 0)
+
+
+@pytest.mark.parametrize("rank1", [False, True])
+def test_tn_dgrad_dual(rank1):
+    """dA = dC[:, :Kw] W^T + dC[:, Kw:] W3^T (+ row_scale x col_vec), the
+    GEMM1 dgrad of the layer with the router's share of dx."""
+    E, Nout, Kw = len(COUNTS_TN), 512, 256
+    poff, offs, A, real, X = _tn_setup(COUNTS_TN, 2 * Kw, 26, True)
+    W, W3 = _w(E, Nout, Kw, 27), _w(E, Nout, Kw, 28)
+    tp, to = torch.from_numpy(poff).cuda(), torch.from_numpy(offs).cuda()
+    g = torch.Generator(device="cuda"); g.manual_seed(29)
+    rs = torch.randn(A, generator=g, device="cuda") if rank1 else None
+    cv = torch.randn((E, Nout), generator=g, device="cuda") * 0.02 if rank1 else None
+    C = moe.moe_grouped_gemm_tn(X, W, tp, E, W3=W3, w_kmajor=True, offsets=to, row_scale=rs,
+                                col_vec=cv)
+    torch.cuda.synchronize()
+    P = int(poff[-1])
+    Xd = f64(X)
+    Xd[~real] = 0.0
+    ref = (oracle.grouped_matmul_t(Xd[:, :Kw], f64(W), poff) +
+           oracle.grouped_matmul_t(Xd[:, Kw:], f64(W3), poff))
+    if rank1:
+        rsd, cvd = rs.double().cpu().numpy(), cv.double().cpu().numpy()
+        for e in range(E):
+            ref[poff[e]:poff[e + 1]] += np.outer(rsd[poff[e]:poff[e + 1]], cvd[e])
+    r = real[:P]
+    assert rel_err(f64(C[:P])[r], ref[:P][r]) < 1e-2
+    assert np.all(f64(C[:P])[_pad_rows(poff, real)] == 0)
