@@ -6,26 +6,30 @@
 // feed-forward compute.
 //
 // Design (sm_100a):
-//  * persistent CTAs (one per SM), 192 threads: warp 0 issues TMA loads,
-//    warp 1 issues tcgen05.mma (one thread) and owns TMEM, warps 2..5 are
-//    the epilogue: each owns 32 accumulator rows, moves 32-column chunks
-//    TMEM -> registers -> a 64-byte-swizzled shared-memory box -> TMA bulk
-//    store (the SwiGLU backward also TMA-loads its H1/H3 chunks), so global
-//    traffic is whole coalesced boxes.
+//  * persistent CTAs (one per SM), 320 threads: warp 0 issues TMA loads,
+//    warp 1 issues tcgen05.mma (one thread) and owns TMEM, warps 2..9 are
+//    the epilogue: two per TMEM lane quarter (32 accumulator rows), one per
+//    half of the tile's columns; each moves 32-column chunks TMEM ->
+//    registers -> a 64-byte-swizzled shared-memory box -> TMA bulk store, so
+//    global traffic is whole coalesced boxes.
 //  * tile 128 x 256, fp32 accumulators in TMEM (two buffers for BF16, so the
 //    epilogue of tile i overlaps the main loop of tile i+1), a 3- or 4-stage
-//    shared-memory ring fed by TMA with 128-byte swizzle.
+//    shared-memory ring fed by TMA with 128-byte swizzle; MN-major operands
+//    come through 3-D tensor maps (one TMA op per operand and stage).
 //  * device-side tile schedule read from poff: "rows" mode walks the
 //    128-row tiles of the expert-contiguous buffer (every group starts on a
 //    multiple of 128, so a tile never mixes experts) times the N tiles;
 //    "wgrad" mode walks (expert, M tile, N tile) and reduces over the rows
-//    of the expert's group.
+//    of the expert's group, stopping at its last real row.
+//  * epilogues: plain store (+ an optional rank-1 term), SwiGLU (h, H1, H3),
+//    SwiGLU backward, and the router's top-k / gates / ranks / histograms.
 //  * every mbarrier wait is bounded; a wait that gives up raises
 //    MOE_DEV_TIMEOUT in the caller's status word and the CTA drains and
 //    exits.
 //  * MXFP8: E4M3 operands with kind::mxf8f6f4.block_scale; the E8M0 scales
 //    of each stage are bulk-copied to shared memory and moved into TMEM
-//    with tcgen05.cp; one accumulator buffer (TMEM also holds the scales).
+//    with tcgen05.cp; one accumulator buffer (TMEM also holds the scales),
+//    handed back to the MMA warp as soon as the epilogue has it in registers.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
