@@ -284,3 +284,24 @@ def test_tn_dgrad_dual(rank1):
     r = real[:P]
     assert rel_err(f64(C[:P])[r], ref[:P][r]) < 1e-2
     assert np.all(f64(C[:P])[_pad_rows(poff, real)] == 0)
+
+
+def test_max_expert_count():
+    """E = 1024 groups (the kernels' limit), most of them empty: the tile
+    schedules of both GEMM kernels and the tokens-N kernel's per-expert
+    tables at their largest."""
+    E, K, N = 1024, 256, 256
+    counts = np.zeros(E, np.int64)
+    counts[[0, 17, 511, 1023]] = [5, 300, 129, 64]
+    poff, A, real = _groups(counts, extra_rows=0)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    X = _act(A, K, real, 31)
+    W = _w(E, K, N, 32)
+    tp, to = torch.from_numpy(poff).cuda(), torch.from_numpy(offs).cuda()
+    C = moe.moe_grouped_gemm_fwd(X, W, tp, E)
+    Ct = moe.moe_grouped_gemm_tn(X, W, tp, E, offsets=to)
+    torch.cuda.synchronize()
+    ref = oracle.grouped_matmul(f64(X), f64(W), poff)
+    P = int(poff[-1])
+    assert rel_err(f64(C[:P]), ref[:P]) < 1e-2
+    assert rel_err(f64(Ct[:P]), ref[:P]) < 1e-2

@@ -35,9 +35,13 @@ def _run(cfg, inp):
 
 
 @pytest.mark.parametrize("variant", ["bf16", "mx", "given", "skewed", "one_token", "ragged",
-                                     "k_equals_E", "single_expert", "mx_ragged"])
+                                     "k_equals_E", "single_expert", "mx_ragged", "many_experts"])
 def test_tiny_layer_element_by_element(variant):
     cfg = moe_inputs.CONFIGS["tiny"]
+    if variant == "many_experts":
+        # the largest expert count the layer's router takes (512): the SIMT
+        # router, most groups empty or with a few rows, the tokens-N GEMMs
+        cfg = cfg.with_(T=512, E=512, k=4, F=256)
     if variant == "one_token":
         cfg = cfg.with_(T=1)
     if variant in ("ragged", "mx_ragged"):
