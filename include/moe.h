@@ -351,8 +351,14 @@ MOE_API moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const f
 
 /* --------------------------------------------------------------- layer
  * The whole layer: route -> permute -> GEMM1+SwiGLU -> GEMM2 -> combine, and
- * its backward.  All saved tensors live in the caller's context buffer
- * `ctx` of at least moe_layer_ctx_bytes(desc) bytes (256-byte aligned).
+ * its backward, on `stream`, with no host synchronisation and no device
+ * allocation.  All saved tensors live in the caller's context buffer `ctx`
+ * of at least moe_layer_ctx_bytes(desc) bytes (256-byte aligned).  BF16
+ * layers whose experts average fewer than 256 rows (T k < 256 E) run the
+ * forward GEMMs and the GEMM1 dgrad on the tokens-N kernel
+ * (moe_grouped_gemm_tn) with the unpadded group offsets; the others on
+ * moe_grouped_gemm_fwd / _dgrad.  Either way every padded row of the saved
+ * tensors is zero.
  */
 typedef struct {
   int T, d, E, k, F;
