@@ -319,7 +319,7 @@ MOE_API moe_status_t moe_unpermute_combine(const void* Y, const float* gates, co
  *   dg[t,j]  = <dout[t], Y[r]>  (fp32)
  *   and, when dl != NULL (router mode), the logit gradient of the chosen
  *   experts dl[t,j] = g_j (dg_j - sum_i g_i dg_i) (fp32), also scattered to
- *   dl_rows[r] (nullable, [A_pad_max] fp32, pad rows untouched).
+ *   dl_rows[r] (nullable, [A_pad_max] fp32, pad rows of each group set to 0).
  */
 MOE_API moe_status_t moe_combine_bwd(const void* dout, const void* Y, const float* gates,
                              const int32_t* dst, const int32_t* offsets, const int32_t* poff,

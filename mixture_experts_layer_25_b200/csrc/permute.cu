@@ -26,14 +26,17 @@ void dispatch_k(int k, F&& f) {
 }
 
 // zero the pad rows [poff[e] + counts[e], poff[e+1]) of one expert group
+// (and, when given, the same entries of a per-row fp32 vector)
 __device__ __forceinline__ void zero_pad_rows(const int32_t* offsets, const int32_t* poff, int e,
-                                              int d8, uint4* buf) {
+                                              int d8, uint4* buf, float* row_vec = nullptr) {
   const int r0 = poff[e] + (offsets[e + 1] - offsets[e]);
   const int r1 = poff[e + 1];
   const size_t n = (size_t)(r1 - r0) * d8;
   const uint4 z = make_uint4(0, 0, 0, 0);
   uint4* base = buf + (size_t)r0 * d8;
   for (size_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = z;
+  if (row_vec)
+    for (int r = r0 + (int)threadIdx.x; r < r1; r += blockDim.x) row_vec[r] = 0.f;
 }
 
 // Row teams: `tpt` threads (a multiple of 32, at most 256) share one token
@@ -241,7 +244,7 @@ combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
                    int k, int d8, int tok_blocks, uint4* __restrict__ dY, float* __restrict__ dg,
                    float* __restrict__ dl, float* __restrict__ dl_rows) {
   if ((int)blockIdx.x >= tok_blocks) {
-    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY);
+    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY, dl_rows);
     return;
   }
   __shared__ float red[kBlock / 32][kMaxK];
@@ -329,7 +332,7 @@ combine_bwd_pf_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ 
                       int k, int d8, int tok_blocks, uint4* __restrict__ dY, float* __restrict__ dg,
                       float* __restrict__ dl, float* __restrict__ dl_rows) {
   if ((int)blockIdx.x >= tok_blocks) {
-    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY);
+    zero_pad_rows(offsets, poff, blockIdx.x - tok_blocks, d8, dY, dl_rows);
     return;
   }
   __shared__ float red[kBlock / 32][kMaxK];

@@ -209,6 +209,7 @@ def test_combine_and_its_backward(T, d, E, k):
     assert rel_err(f64(dY[:P]), dY_o[:P]) < 1e-2
     pad = ref["src"] < 0
     assert np.all(f64(dY[:P])[pad] == 0)
+    assert np.all(dl_rows.cpu().numpy()[:P][pad] == 0)      # pad rows of dl_rows are zero too
     assert rel_err(dg.cpu().numpy(), dg_o) < 1e-4
     dl_o = oracle.gate_logit_grad(g64, dg_o)
     assert rel_err(dl.cpu().numpy(), dl_o) < 1e-4
