@@ -533,6 +533,17 @@ moe_status_t gemm_tn(int epilogue, const void* X, const void* W, const void* W3,
   MOE_CHECK_ARG(K > 0 && K % BK == 0, "gemm_tn: K %% %d", BK);
   MOE_CHECK_ARG((row_scale == nullptr) == (col_vec == nullptr) && (!col_vec || aligned16(col_vec)),
                 "gemm_tn: row_scale and col_vec go together");
+  // every argument is checked before the first driver call
+  if (epilogue == MOE_EPI_SWIGLU) {
+    MOE_CHECK_ARG(W3 && aux && !w_kmajor && N % 64 == 0 && !row_scale,
+                  "gemm_tn: SwiGLU needs W3, aux, MN-major weights and N %% 64");
+  } else {
+    MOE_CHECK_ARG(epilogue == MOE_EPI_NONE, "gemm_tn: epilogue must be NONE or SWIGLU");
+    MOE_CHECK_ARG(N % BM == 0, "gemm_tn: N %% %d", BM);
+    MOE_CHECK_ARG(w_kmajor || (!W3 && !row_scale),
+                  "gemm_tn: MN-major weights take neither W3 nor a rank-1 term");
+    MOE_CHECK_ARG(!w_kmajor || (W3 ? K / 2 : K) % BK == 0, "gemm_tn: K per weight %% %d", BK);
+  }
   Params p{};
   p.poff = poff;
   p.offsets = offsets;
@@ -546,8 +557,6 @@ moe_status_t gemm_tn(int epilogue, const void* X, const void* W, const void* W3,
   MOE_TRY(map2d(&mx, X, K, A_pad_max, BK, BNMAX, CU_TENSOR_MAP_SWIZZLE_128B));
   MOE_TRY(map2d(&mc, C, N, A_pad_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B));
   if (epilogue == MOE_EPI_SWIGLU) {
-    MOE_CHECK_ARG(W3 && aux && !w_kmajor && N % 64 == 0 && !row_scale,
-                  "gemm_tn: SwiGLU needs W3, aux, MN-major weights and N %% 64");
     p.n_fb = N / 64;
     p.feat_per_fb = 64;
     p.a_rows_per_e = K;
@@ -558,19 +567,15 @@ moe_status_t gemm_tn(int epilogue, const void* X, const void* W, const void* W3,
     const int max_tiles = (A_pad_max / 32) * p.n_fb;
     return launch<TN_SWIGLU, A_MN>(mw, mw3, mx, mc, maux, p, max_tiles, s);
   }
-  MOE_CHECK_ARG(epilogue == MOE_EPI_NONE, "gemm_tn: epilogue must be NONE or SWIGLU");
-  MOE_CHECK_ARG(N % BM == 0, "gemm_tn: N %% %d", BM);
   p.n_fb = N / BM;
   p.feat_per_fb = BM;
   const int max_tiles = (A_pad_max / 32) * p.n_fb;
   if (!w_kmajor) {
-    MOE_CHECK_ARG(!W3 && !row_scale, "gemm_tn: MN-major weights take neither W3 nor a rank-1 term");
     p.a_rows_per_e = K;
     MOE_TRY(map2d(&mw, W, N, (uint64_t)E * K, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B));
     return launch<TN_STORE, A_MN>(mw, mw, mx, mc, mc, p, max_tiles, s);
   }
   const int Kw = W3 ? K / 2 : K;          // K columns of each weight
-  MOE_CHECK_ARG(Kw % BK == 0, "gemm_tn: K per weight %% %d", BK);
   p.a_rows_per_e = N;
   p.k_split = Kw;
   MOE_TRY(map2d(&mw, W, Kw, (uint64_t)E * N, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B));

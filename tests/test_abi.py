@@ -73,3 +73,25 @@ def test_argument_errors_need_no_gpu():
     assert b"bad T/E/k" in lib.moe_last_error()
     code = lib.mx_quantize(None, 100, 128, 0, None, 0, None, None, None, None)
     assert code == _lib.MOE_ERR_INVALID_ARG
+
+
+def test_grouped_gemm_argument_errors_need_no_gpu():
+    lib = _lib.lib()
+    fake = ctypes.c_void_p(256)     # never dereferenced: the checks fail first
+    # E out of range
+    assert lib.moe_grouped_gemm_tn(0, fake, fake, None, 0, fake, None, 0, 128, 128, 64, fake,
+                                   None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    # K not a multiple of 64
+    assert lib.moe_grouped_gemm_tn(0, fake, fake, None, 0, fake, None, 4, 128, 128, 100, fake,
+                                   None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    # SwiGLU without W3 / aux
+    assert lib.moe_grouped_gemm_tn(1, fake, fake, None, 0, fake, None, 4, 128, 128, 64, fake,
+                                   None, None, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    # a rank-1 term needs both vectors
+    assert lib.moe_grouped_gemm_tn(0, fake, fake, None, 1, fake, None, 4, 128, 128, 64, fake,
+                                   None, fake, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    # A_pad_max not a multiple of 128
+    assert lib.moe_grouped_gemm_fwd(0, fake, None, fake, None, None, None, fake, 4, 100, 256, 64,
+                                    0, fake, None, None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_wgrad(0, fake, None, fake, None, fake, 4, 128, 100, 256, fake,
+                                      None, None, None) == _lib.MOE_ERR_INVALID_ARG
