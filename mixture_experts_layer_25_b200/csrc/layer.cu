@@ -4,11 +4,14 @@
 // Forward:  route -> permute (rowwise dispatch) -> GEMM1 + SwiGLU -> GEMM2
 //           -> gate-weighted combine.
 // Backward: combine bwd (dY = g dout, dg, dl) -> GEMM2 dgrad fused with the
-//           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad -> GEMM1 wgrad ->
-//           unpermute-sum (+ router input grad) -> router weight grad.
+//           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad (+ the router's
+//           share of dx as a rank-1 epilogue term) -> GEMM1 wgrad ->
+//           unpermute-sum -> router weight grad.
 // In MXFP8 mode every GEMM operand is quantised along that GEMM's K first
 // (weights included, inside the step); operands used by two GEMMs with
-// different K axes are quantised along both in one pass.
+// different K axes are quantised along both in one pass.  BF16 layers whose
+// experts average fewer than 256 rows take the tokens-N kernel for the
+// forward GEMMs and the GEMM1 dgrad (see tokens_n below).
 #include "common.cuh"
 
 namespace {
