@@ -254,7 +254,7 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
                          ((mn >> 5) & 3) * 4;
       *reinterpret_cast<uint32_t*>(scales_c + off) = word;
     }
-    __syncthreads();   // buffer `buf`, camax and cbyte are free for the next round
+    __syncthreads();   // buffer `buf`, camax and cbyte are free for the next tile
   }
 }
 
