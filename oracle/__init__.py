@@ -31,6 +31,7 @@ from .moe_oracle import (  # noqa: F401
     permute_rows, expert_forward, combine, layer_forward, layer_backward,
     silu, round_bf16, grouped_matmul, grouped_matmul_t, grouped_wgrad, swiglu_backward,
     combine_backward, gate_logit_grad, unpermute_sum, router_backward,
+    gemm1_fwd, gemm2_fwd, gemm2_dgrad, gemm2_wgrad, gemm1_dgrad, gemm1_wgrad,
 )
 from .mx import (  # noqa: F401
     e4m3_decode_table, e4m3_encode, mx_scale_exponent, mx_quantize_rows,

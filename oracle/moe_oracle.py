@@ -159,6 +159,44 @@ def _gemm(a, b, mx, a_blocks_along, b_blocks_along):
     return a @ b
 
 
+# The six expert GEMMs of one group ([OC3-ja] "MXFP8による精度最適化": the
+# expert feed-forward matmuls run in MXFP8).  In MX mode each operand is
+# quantised in blocks of 32 along that GEMM's reduction axis K: for a
+# row-major a [M, K] that is along its rows ('rows'), for b [K, N] down its
+# columns ('cols').  Xe, he, dYe, dA1, dA3 are the group's rows.
+
+def gemm1_fwd(Xe, W1e, W3e, mx=False):
+    """H1 = Xe W1e, H3 = Xe W3e; K = d."""
+    return _gemm(Xe, W1e, mx, "rows", "cols"), _gemm(Xe, W3e, mx, "rows", "cols")
+
+
+def gemm2_fwd(he, W2e, mx=False):
+    """Y = he W2e; K = F."""
+    return _gemm(he, W2e, mx, "rows", "cols")
+
+
+def gemm2_dgrad(dYe, W2e, mx=False):
+    """dh = dYe W2e^T; K = d."""
+    return _gemm(dYe, W2e.T, mx, "rows", "cols")
+
+
+def gemm2_wgrad(he, dYe, mx=False):
+    """dW2e = he^T dYe; K = the group's rows (blocks of 32 rows from the
+    group's first row)."""
+    return _gemm(he.T, dYe, mx, "rows", "cols")
+
+
+def gemm1_dgrad(dA1, dA3, W1e, W3e, mx=False):
+    """dXe = dA1 W1e^T + dA3 W3e^T, i.e. [dA1 | dA3] [W1e | W3e]^T; K = 2F
+    (F is a multiple of 32, so no block straddles the two halves)."""
+    return _gemm(dA1, W1e.T, mx, "rows", "cols") + _gemm(dA3, W3e.T, mx, "rows", "cols")
+
+
+def gemm1_wgrad(Xe, dA1, dA3, mx=False):
+    """dW1e = Xe^T dA1, dW3e = Xe^T dA3; K = the group's rows."""
+    return _gemm(Xe.T, dA1, mx, "rows", "cols"), _gemm(Xe.T, dA3, mx, "rows", "cols")
+
+
 def expert_forward(Xp, W1, W3, W2, poff, mx=False):
     """Per group e (rows poff[e]..poff[e+1]): H1 = Xe W1[e], H3 = Xe W3[e],
     h = silu(H1) * H3, Y = h W2[e].  Returns (H1, H3, h, Y) over all rows."""
@@ -171,12 +209,10 @@ def expert_forward(Xp, W1, W3, W2, poff, mx=False):
         if a == b:
             continue
         Xe = Xp[a:b]
-        # fwd GEMM1: K = d; x blocks along its row, W blocks down its columns
-        H1[a:b] = _gemm(Xe, W1[e], mx, "rows", "cols")
-        H3[a:b] = _gemm(Xe, W3[e], mx, "rows", "cols")
+        H1[a:b], H3[a:b] = gemm1_fwd(Xe, W1[e], W3[e], mx)
         h[a:b] = silu(H1[a:b]) * H3[a:b]
         he = round_bf16(h[a:b]) if mx else h[a:b]
-        Y[a:b] = _gemm(he, W2[e], mx, "rows", "cols")   # fwd GEMM2: K = F
+        Y[a:b] = gemm2_fwd(he, W2[e], mx)
     return H1, H3, h, Y
 
 
@@ -316,32 +352,29 @@ def layer_backward(ctx, dout):
 
     dW1 = np.zeros_like(W1); dW3 = np.zeros_like(W3); dW2 = np.zeros_like(W2)
     dXp = np.zeros_like(Xp)
+    dh = np.zeros_like(h); dA1 = np.zeros_like(h); dA3 = np.zeros_like(h)
     for e in range(E):
         a, b = int(poff[e]), int(poff[e + 1])
         if a == b:
             continue
         dYe = dY[a:b]
         he = round_bf16(h[a:b]) if mx else h[a:b]
-        # GEMM2 dgrad (K = d) and wgrad (K = rows of the group)
-        dh = _gemm(dYe, W2[e].T, mx, "rows", "cols")
-        dW2[e] = _gemm(he.T, dYe, mx, "rows", "cols")
+        dh[a:b] = gemm2_dgrad(dYe, W2[e], mx)
+        dW2[e] = gemm2_wgrad(he, dYe, mx)
         if mx:
             # the saved activations enter the backward at their stored (bf16)
-            # precision, so the quantised dA operands are the device's
-            dA1, dA3 = swiglu_backward(dh, round_bf16(H1[a:b]), round_bf16(H3[a:b]))
+            # precision, and dA is stored in bf16 before it is quantised, so
+            # the quantised dA operands are the device's
+            g1, g3 = swiglu_backward(dh[a:b], round_bf16(H1[a:b]), round_bf16(H3[a:b]))
+            dA1[a:b], dA3[a:b] = round_bf16(g1), round_bf16(g3)
         else:
-            dA1, dA3 = swiglu_backward(dh, H1[a:b], H3[a:b])
-        if mx:
-            dA1 = round_bf16(dA1); dA3 = round_bf16(dA3)
-        # GEMM1 dgrad (K = 2F) and wgrad (K = rows of the group)
-        dXp[a:b] = _gemm(dA1, W1[e].T, mx, "rows", "cols") + \
-            _gemm(dA3, W3[e].T, mx, "rows", "cols")
-        Xe = Xp[a:b]
-        dW1[e] = _gemm(Xe.T, dA1, mx, "rows", "cols")
-        dW3[e] = _gemm(Xe.T, dA3, mx, "rows", "cols")
+            dA1[a:b], dA3[a:b] = swiglu_backward(dh[a:b], H1[a:b], H3[a:b])
+        dXp[a:b] = gemm1_dgrad(dA1[a:b], dA3[a:b], W1[e], W3[e], mx)
+        dW1[e], dW3[e] = gemm1_wgrad(Xp[a:b], dA1[a:b], dA3[a:b], mx)
 
     dx = unpermute_sum(dXp, dst)
-    out = dict(dx=dx, dW1=dW1, dW3=dW3, dW2=dW2, dg=dg, dY=dY, dXp=dXp)
+    out = dict(dx=dx, dW1=dW1, dW3=dW3, dW2=dW2, dg=dg, dY=dY, dXp=dXp, dh=dh, dA1=dA1,
+               dA3=dA3)
     if ctx["router"]:
         dl = gate_logit_grad(g, dg)
         dWr, dx_r = router_backward(ctx["x"], ctx["Wr"], ctx["topk_idx"], dl)
