@@ -352,7 +352,12 @@ MOE_API moe_status_t moe_router_wgrad(const void* x, const int32_t* src, const f
 /* --------------------------------------------------------------- layer
  * The whole layer: route -> permute -> GEMM1+SwiGLU -> GEMM2 -> combine, and
  * its backward, on `stream`, with no host synchronisation and no device
- * allocation.  All saved tensors live in the caller's context buffer `ctx`
+ * allocation.  ([OC3-ja] "ルーティングと計算の最適化": the steps of one MoE
+ * layer -- route, keep the metadata on the GPU, write the rows into the
+ * experts' buffers, grouped GEMM, combine; "MXFP8による精度最適化": the
+ * expert GEMMs in MXFP8 when desc.dtype is MOE_MXFP8; [OC3-hu] first
+ * section and [JUPITER] model paragraph: the layer shapes, 128 experts with
+ * 4 chosen per token, 384 with 8.)  All saved tensors live in the caller's context buffer `ctx`
  * of at least moe_layer_ctx_bytes(desc) bytes (256-byte aligned).  BF16
  * layers whose experts average fewer than 256 rows (T k < 256 E) run the
  * forward GEMMs and the GEMM1 dgrad on the tokens-N kernel
@@ -397,9 +402,15 @@ typedef struct {
   int A_pad_max;
 } moe_ctx_view;
 
+/* Bytes of the context buffer the layer needs (host-side, no GPU work; 0
+ * for a description the layer rejects).  The context holds what the
+ * backward reuses from the forward ([OC3-ja] "ルーティングと計算の最適化":
+ * routing metadata and expert buffers stay on the GPU). */
 MOE_API size_t moe_layer_ctx_bytes(const moe_layer_desc* desc);
 MOE_API moe_status_t moe_layer_ctx_view(const moe_layer_desc* desc, void* ctx, moe_ctx_view* view);
 
+/* Forward of the layer: out [T,d] bf16 from x [T,d] bf16; saves into ctx
+ * what the backward needs.  (Passages: as for the layer above.) */
 MOE_API moe_status_t moe_layer_fwd(const moe_layer_desc* desc, const moe_layer_weights* w,
                            const void* x, void* out, void* ctx, size_t ctx_bytes,
                            int32_t* dev_status, moe_stream_t stream);
@@ -417,9 +428,15 @@ MOE_API moe_status_t moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_w
 /* One training step of the layer from HOST buffers: copies x and dout
  * (pinned host memory recommended) to the device buffers x_dev / dout_dev,
  * runs moe_layer_fwd and moe_layer_bwd, and copies out and dx back to
- * out_host / dx_host (all copies cudaMemcpyAsync on `stream`; the call
- * returns once they are enqueued -- synchronise the stream before reading
- * the host outputs).
+ * out_host / dx_host.  x and dx move on `stream`; dout and out move on a
+ * copy stream the library creates once per device (non-blocking, kept until
+ * exit) and orders with events, so that the dout upload overlaps the forward
+ * and the out download overlaps the backward.  The call returns once the
+ * work is enqueued and leaves `stream` ordered after every copy: synchronise
+ * `stream` before reading the host outputs.  The call creates and releases
+ * four CUDA events per call; it allocates no device memory.
+ * ([OC3-th] scaling/optimisation section: the host queues the work without
+ * waiting for copies.)
  */
 MOE_API moe_status_t moe_layer_step_host(const moe_layer_desc* desc, const moe_layer_weights* w,
                                  const void* x_host, const void* dout_host, void* out_host,

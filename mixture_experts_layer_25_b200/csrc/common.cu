@@ -2,7 +2,10 @@
 #include <stdarg.h>
 
 #include <atomic>
+#include <map>
+#include <mutex>
 #include <stdio.h>
+#include <utility>
 
 #include "common.cuh"
 
@@ -27,6 +30,42 @@ int num_sms() {
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     return 148;
   return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+moe_status_t set_smem_limit(const void* kernel, size_t bytes, const char* what) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;   // (kernel, device) -> bytes set
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    set_error("%s: no current device", what);
+    return MOE_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(kernel, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return MOE_OK;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    set_error("%s: shared-memory limit %zu bytes: %s", what, bytes, cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  done[key] = bytes;
+  return MOE_OK;
 }
 
 }  // namespace moe

@@ -3,6 +3,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include "moe.h"
@@ -77,6 +78,15 @@ moe_status_t gemm_tn(int epilogue, const void* X, const void* W, const void* W3,
 
 // out[cols, rows] = in[rows, cols]^T (fp32)
 moe_status_t transpose_f32(const float* in, int rows, int cols, float* out, cudaStream_t s);
+
+// The driver's tensor-map encoder, looked up once per process (thread-safe);
+// null if the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute is per device, so it is set once per (kernel,
+// device) under a lock, and recorded only when the call succeeds.
+moe_status_t set_smem_limit(const void* kernel, size_t bytes, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }

@@ -33,8 +33,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -881,26 +879,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 2-D map over a row-major [outer, inner] array of 1- or 2-byte elements,
 // box {box_inner, box_outer}, 128-byte swizzle.
 moe_status_t make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner,
                       uint64_t outer, uint32_t box_inner, uint32_t box_outer,
                       CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) {
     set_error("cuTensorMapEncodeTiled unavailable");
     return MOE_ERR_CUDA;
@@ -931,7 +915,7 @@ bool make_map_mn3(CUtensorMap* m, const void* base, int elem_bytes, uint64_t col
 #ifdef MOE_GG_NO_3D
   return false;
 #endif
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   const uint64_t ce = 128 / elem_bytes;
   if (cols % ce) return false;
@@ -959,15 +943,7 @@ template <bool MX, bool A_MN, int BLOAD, int EPI>
 moe_status_t launch(const Maps& m, const Params& p, int max_tiles, cudaStream_t s) {
   auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI>;
   const size_t smem = EpiCfg<MX, EPI, A_MN>::SMEM;
-  static bool attr = false;   // one per instantiation
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-      set_error("grouped_gemm: smem attribute: %s", cudaGetErrorString(e));
-      return MOE_ERR_CUDA;
-    }
-    attr = true;
-  }
+  MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(kern), smem, "grouped_gemm"));
   const int grid = max(1, min(num_sms(), max_tiles));
   kern<<<grid, NUM_THREADS, smem, s>>>(m.a, m.b, m.b3, m.c, m.c2, m.in, p);
   MOE_CHECK_LAUNCH("grouped_gemm");

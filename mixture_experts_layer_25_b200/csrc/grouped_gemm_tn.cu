@@ -446,25 +446,10 @@ gemm_tn_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 // 2-D map over a row-major [outer, inner] bf16 array, box {box_inner, box_outer}
 moe_status_t map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                    uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) {
     set_error("cuTensorMapEncodeTiled unavailable");
     return MOE_ERR_CUDA;
@@ -495,15 +480,7 @@ moe_status_t launch(const CUtensorMap& w, const CUtensorMap& w3, const CUtensorM
                     cudaStream_t s) {
   auto kern = gemm_tn_kernel<EPI, ALOAD>;
   const size_t smem = smem_bytes(p.E);
-  static size_t attr = 0;   // one per instantiation: the largest size set so far
-  if (smem > attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-      set_error("gemm_tn: smem attribute: %s", cudaGetErrorString(e));
-      return MOE_ERR_CUDA;
-    }
-    attr = smem;
-  }
+  MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(kern), smem, "gemm_tn"));
   const int grid = std::max(1, std::min(num_sms(), max_tiles));
   kern<<<grid, NUM_THREADS, smem, s>>>(w, w3, x, c, aux, p);
   MOE_CHECK_LAUNCH("gemm_tn");

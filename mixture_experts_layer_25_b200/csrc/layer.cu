@@ -12,6 +12,8 @@
 // different K axes are quantised along both in one pass.  BF16 layers whose
 // experts average fewer than 256 rows take the tokens-N kernel for the
 // forward GEMMs and the GEMM1 dgrad (see tokens_n below).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -339,6 +341,47 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   return MOE_OK;
 }
 
+namespace {
+
+constexpr int kMaxCopyDevices = 64;
+std::mutex g_copy_mu;
+cudaStream_t g_copy_stream[kMaxCopyDevices] = {};
+
+// The library's copy stream on the current device (non-blocking, created on
+// first use and kept until the process exits).
+moe_status_t copy_stream(cudaStream_t* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxCopyDevices) {
+    set_error("moe_layer_step_host: no usable current device");
+    return MOE_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  if (!g_copy_stream[dev] &&
+      cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    g_copy_stream[dev] = nullptr;
+    set_error("moe_layer_step_host: copy stream creation failed");
+    return MOE_ERR_CUDA;
+  }
+  *out = g_copy_stream[dev];
+  return MOE_OK;
+}
+
+struct Events {
+  cudaEvent_t ev[4] = {};
+  ~Events() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);   // released by the driver once the event has completed
+  }
+};
+
+}  // namespace
+
+// Schedule (s = the caller's stream, c = the library's copy stream):
+//   s: record start | H2D x | fwd | record fwd_done | wait dout_in | bwd | D2H dx | wait out_out
+//   c: wait start   | H2D dout | record dout_in | wait fwd_done | D2H out | record out_out
+// so the dout upload runs under the forward and the out download under the
+// backward; the call leaves s ordered after every copy, as if all of them
+// had been issued on s.
 extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_layer_weights* w,
                                             const void* x_host, const void* dout_host,
                                             void* out_host, void* dx_host, void* x_dev,
@@ -349,18 +392,45 @@ extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_l
   MOE_CHECK_ARG(x_host && dout_host && out_host && dx_host && x_dev && dout_dev && out_dev && dx_dev,
                 "moe_layer_step_host: null pointer");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t c = nullptr;
+  MOE_TRY(copy_stream(&c));
+  Events E;
+  for (cudaEvent_t& e : E.ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      e = nullptr;
+      set_error("moe_layer_step_host: event creation failed");
+      return MOE_ERR_CUDA;
+    }
+  cudaEvent_t start = E.ev[0], dout_in = E.ev[1], fwd_done = E.ev[2], out_out = E.ev[3];
   const size_t bytes = (size_t)L->T * L->d * 2;
-  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-    set_error("moe_layer_step_host: host-to-device copy failed");
+  auto fail = [](const char* what) {
+    set_error("moe_layer_step_host: %s failed", what);
     return MOE_ERR_CUDA;
+  };
+  if (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(c, start, 0) != cudaSuccess)
+    return fail("ordering the copy stream");
+  if (cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, c) != cudaSuccess ||
+      cudaEventRecord(dout_in, c) != cudaSuccess)
+    return fail("host-to-device copy of dout");
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return fail("host-to-device copy of x");
+  // from here on every error path still joins the copy stream into s
+  moe_status_t st = moe_layer_fwd(L, w, x_dev, out_dev, ctx, ctx_bytes, dev_status, stream);
+  const bool rec = cudaEventRecord(fwd_done, s) == cudaSuccess;
+  const bool waited = rec && cudaStreamWaitEvent(c, fwd_done, 0) == cudaSuccess;
+  bool copied_out = false;
+  if (st == MOE_OK && waited)
+    copied_out = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, c) == cudaSuccess;
+  const bool rec_out = cudaEventRecord(out_out, c) == cudaSuccess;
+  if (st == MOE_OK) {
+    if (cudaStreamWaitEvent(s, dout_in, 0) != cudaSuccess) st = fail("ordering the backward");
+    else st = moe_layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream);
   }
-  MOE_TRY(moe_layer_fwd(L, w, x_dev, out_dev, ctx, ctx_bytes, dev_status, stream));
-  MOE_TRY(moe_layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream));
-  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
-    set_error("moe_layer_step_host: device-to-host copy failed");
-    return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  if (st == MOE_OK &&
+      cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    st = fail("device-to-host copy of dx");
+  if ((!rec_out || cudaStreamWaitEvent(s, out_out, 0) != cudaSuccess) && st == MOE_OK)
+    st = fail("joining the copy stream");
+  if (st == MOE_OK && !(waited && copied_out)) st = fail("device-to-host copy of out");
+  return st;
 }

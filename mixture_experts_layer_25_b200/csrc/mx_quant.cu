@@ -12,8 +12,6 @@
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -361,22 +359,6 @@ extern "C" moe_status_t mx_quantize(const void* in, int rows, int cols, int axis
   return MOE_OK;
 }
 
-namespace {
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_q() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-}  // namespace
-
 extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
                                          const int32_t* nrows_dev, uint8_t* codes_rows,
                                          uint8_t* scales_rows, uint8_t* codes_cols,
@@ -387,7 +369,7 @@ extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
   MOE_CHECK_ARG(in && codes_rows && scales_rows && codes_cols && scales_cols && aligned16(in) &&
                     aligned16(codes_rows) && aligned16(codes_cols),
                 "mx_quantize_dual: null or unaligned pointer");
-  auto fn = encode_fn_q();
+  auto fn = tensor_map_encoder();
   if (!fn) {
     set_error("mx_quantize_dual: cuTensorMapEncodeTiled unavailable");
     return MOE_ERR_CUDA;
@@ -404,12 +386,8 @@ extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
     return MOE_ERR_CUDA;
   }
   const size_t smem = 2 * (size_t)kDualTileBytes;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(mx_quant_dual_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    attr = true;
-  }
+  MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(mx_quant_dual_tma_kernel), smem,
+                         "mx_quantize_dual"));
   const long long ntiles = (long long)(rows / 128) * (cols / 128);
   const int grid = (int)std::min<long long>(ntiles, (long long)MOE_QDUAL_MIN_BLOCKS * num_sms());
   mx_quant_dual_tma_kernel<<<grid, 32 * kDualWarps, smem, s>>>(m, rows, cols, nrows_dev, codes_rows,

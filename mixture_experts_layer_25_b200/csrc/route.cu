@@ -394,12 +394,8 @@ extern "C" moe_status_t moe_route(const void* x, const float* Wr, const float* b
     MOE_CHECK_ARG(E <= kMaxRouterE, "moe_route: router mode supports E <= %d", kMaxRouterE);
     MOE_CHECK_ARG(d > 0 && d % 8 == 0 && aligned16(x), "moe_route: d %% 8 and 16B-aligned x");
     const size_t smem = (size_t)kTok * (E + 1) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)((size_t)kTok * (kMaxRouterE + 1) * sizeof(float)));
-      attr_set = true;
-    }
+    MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(route_topk_kernel),
+                           (size_t)kTok * (kMaxRouterE + 1) * sizeof(float), "route_topk"));
     const int nblk = (T + kTok - 1) / kTok;
     route_topk_kernel<<<nblk, kRouteThreads, smem, s>>>(
         static_cast<const __nv_bfloat16*>(x), Wr, bias, T, d, E, k, topk_idx, gates, logits, dst,

@@ -185,6 +185,86 @@ def test_mx_quantize_dual_equals_both_axes(R, C):
     np.testing.assert_array_equal(scales_to_plain(sc, R, C, 1), s1)
 
 
+def _every_finite_bf16_in_blocks():
+    """Blocks of 32 that hold every finite bf16 value (both zeros and the
+    subnormals included) in several roles, as float64 [n_blocks, 32]:
+    * each value v as its block's maximum, with 31 companions v * (-1)^j
+      2^(-j/2) rounded to bf16 (down to E4M3 subnormals and to zero);
+    * each value v with |v| <= M as an ordinary element of a block whose
+      maximum is a fixed M (the largest finite bf16, 1, 1.5, 2^100, 2^-120 and
+      the subnormal 2^-130), 31 values per block, either sign of M."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    v = f[np.isfinite(f)].astype(np.float64)
+    to_bf16 = lambda a: torch.tensor(a).to(torch.bfloat16).to(torch.float64).numpy()  # noqa: E731
+    j = np.arange(1, 32)
+    comp = to_bf16(v[:, None] * ((-1.0) ** j * 2.0 ** (-j / 2.0))[None, :])
+    fam = [np.concatenate([v[:, None], comp], axis=1)]
+    bmax = float(np.max(v))
+    for i, M in enumerate([bmax, 1.0, 1.5, 2.0 ** 100, 2.0 ** -120, 2.0 ** -130]):
+        u = v[np.abs(v) <= M]
+        n = -(-len(u) // 31)
+        body = np.concatenate([u, np.zeros(n * 31 - len(u))]).reshape(n, 31)
+        head = np.full((n, 1), M if i % 2 == 0 else -M)
+        fam.append(np.concatenate([head, body], axis=1))
+    return np.concatenate(fam, axis=0)
+
+
+def _blocks_as(blocks, axis, C=128):
+    """[n, 32] blocks -> a [R, C] array (R, C multiples of 128) whose 32-blocks
+    along rows (axis 0) or down columns (axis 1) are the given blocks, in
+    order, padded with zero blocks."""
+    per = C // 32 if axis == 0 else C
+    n = -(-len(blocks) // per)
+    rows_per = 1 if axis == 0 else 32
+    R = -(-n * rows_per // 128) * 128
+    pad = R // rows_per * per - len(blocks)
+    b = np.concatenate([blocks, np.zeros((pad, 32))], axis=0)
+    if axis == 0:
+        return b.reshape(R, C)
+    return b.reshape(R // 32, C, 32).transpose(0, 2, 1).reshape(R, C)
+
+
+def test_mx_quantisers_on_every_finite_bf16_value():
+    """Every finite bf16 value through the row and column quantisers, the
+    dual quantiser (both arrangements) and the permute's fused MX codes,
+    bit-exact against the oracle's quantiser."""
+    blocks = _every_finite_bf16_in_blocks()
+    for axis in (0, 1):
+        a = _blocks_as(blocks, axis)
+        R, C = a.shape
+        t = torch.tensor(a).to(torch.bfloat16).cuda()
+        np.testing.assert_array_equal(f64(t), a)             # every value is a bf16 number
+        if axis == 0:
+            c_ref, s_ref = oracle.mx_quantize_rows(a)
+        else:
+            c_ref, s_ref = oracle.mx_quantize_cols_grouped(a, np.array([0, R]))
+        codes, scales = moe.mx_quantize(t, axis)
+        (cr, sr), (cc, sc) = moe.mx_quantize_dual(t)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+        np.testing.assert_array_equal(scales_to_plain(scales, R, C, axis), s_ref)
+        c0, s0 = oracle.mx_quantize_rows(a)
+        c1, s1 = oracle.mx_quantize_cols_grouped(a, np.array([0, R]))
+        np.testing.assert_array_equal(cr.cpu().numpy(), c0)
+        np.testing.assert_array_equal(scales_to_plain(sr, R, C, 0), s0)
+        np.testing.assert_array_equal(cc.cpu().numpy(), c1)
+        np.testing.assert_array_equal(scales_to_plain(sc, R, C, 1), s1)
+    # the permute's fused quantisation: the rows of the axis-0 arrangement
+    # as tokens, each routed to k = 2 of 8 experts
+    x64 = _blocks_as(blocks, 0)
+    T, d = x64.shape
+    x = torch.tensor(x64).to(torch.bfloat16).cuda()
+    idx, gates, meta = _meta_for(T, 8, 2, 5)
+    Xp, Xq, Xs = moe.moe_permute(x, meta, 2, 8, mx=True)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, 8, 128)
+    P = int(ref["poff"][8])
+    c, s = oracle.mx_quantize_rows(oracle.permute_rows(x64, ref))
+    np.testing.assert_array_equal(Xq[:P].cpu().numpy(), c)
+    np.testing.assert_array_equal(scales_to_plain(Xs, meta["A_pad_max"], d, 0)[:P], s)
+
+
 @pytest.mark.parametrize("T,d,E,k", [(1024, 256, 8, 2), (257, 2048, 32, 4), (64, 6144, 384, 8),
                                      (3000, 1024, 16, 3), (5000, 2048, 64, 4), (1, 2048, 8, 4)])
 def test_combine_and_its_backward(T, d, E, k):

@@ -1,8 +1,10 @@
 """moe_route_noalloc: routing for callers that cannot allocate device memory
 while they run (a pooling allocator owns the device memory, or a
 latency-critical loop must not call cudaMalloc).  Its scratch is a fixed
-array the library keeps in device memory.  The test compares two calls in a
-row with the ordinary moe_route (caller workspace) through the C ABI.  It is
+array the library keeps in device memory, shared by every call.  The test
+makes two calls in a row on different inputs (the second smaller, so scratch
+left over from the first would show) and compares each with the ordinary
+moe_route (caller workspace) on the same input, through the C ABI.  It is
 collected last, needs nothing from other test files, and runs alone or after
 them."""
 import ctypes
@@ -22,15 +24,16 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _case(mode):
+def _case(mode, call):
+    """Input of the call-th call: a different size and different data."""
     if mode == "router":
-        T, d, E, k = 4096, 2048, 128, 4
-        x = moe_inputs.random_bf16((T, d), 21, device="cuda")
-        g = torch.Generator(device="cuda"); g.manual_seed(22)
+        T, d, E, k = (4096, 2048, 128, 4) if call == 0 else (1000, 2048, 128, 4)
+        x = moe_inputs.random_bf16((T, d), 21 + 10 * call, device="cuda")
+        g = torch.Generator(device="cuda"); g.manual_seed(22 + 10 * call)
         Wr = torch.randn((d, E), generator=g, device="cuda") * 0.02
         return dict(T=T, d=d, E=E, k=k, x=x, Wr=Wr, topk=None, gates=None)
-    T, E, k = 8192, 384, 8
-    idx, gates = moe_inputs.random_routing(T, E, k, 23)
+    T, E, k = (8192, 384, 8) if call == 0 else (3000, 384, 8)
+    idx, gates = moe_inputs.random_routing(T, E, k, 23 + 10 * call)
     return dict(T=T, d=0, E=E, k=k, x=None, Wr=None, topk=torch.from_numpy(idx).cuda(),
                 gates=torch.from_numpy(gates).cuda())
 
@@ -51,11 +54,12 @@ def _fresh_outputs(c):
 
 @pytest.mark.parametrize("mode", ["router", "given"])
 def test_noalloc_route_matches_route_on_two_calls(mode):
-    c = _case(mode)
-    ref = moe.moe_route(c["x"], c["Wr"], None, c["k"], c["E"], topk_idx=c["topk"], gates=c["gates"])
-    torch.cuda.synchronize()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for _ in range(2):
+    for call in range(2):
+        c = _case(mode, call)
+        ref = moe.moe_route(c["x"], c["Wr"], None, c["k"], c["E"], topk_idx=c["topk"],
+                            gates=c["gates"])
+        torch.cuda.synchronize()
         o = _fresh_outputs(c)
         st = torch.zeros(1, dtype=torch.int32, device="cuda")
         _lib.call("moe_route_noalloc", _p(c["x"]), _p(c["Wr"]), None, c["T"], c["d"], c["E"],
