@@ -273,6 +273,45 @@ def _tensor_peak(peaks, peak_kind, clk, timed_s, mx):
                                                  "nominal": NOMINAL_BF16_TFLOPS * f}
 
 
+def schedule_efficiency(work, workers):
+    """Busy fraction of `workers` persistent CTAs (or CTA pairs) that take
+    tiles round-robin (tile i -> worker i mod workers, as the grouped GEMMs
+    walk their schedules): mean worker load over the largest one."""
+    work = np.asarray(work, np.float64)
+    if work.size == 0 or work.sum() == 0:
+        return 1.0
+    loads = np.bincount(np.arange(work.size) % workers, weights=work, minlength=workers)
+    return float(loads.mean() / loads.max())
+
+
+def load_metrics(counts, poff, cfg, num_sms=148):
+    """Expert load of one routing: imbalance, a histogram of the per-expert
+    row counts, the rows the 128-row group padding adds, and how evenly the
+    GEMM tile schedules spread that load over the SMs (value-dependent
+    kernel timing: the same FLOPs take longer when a few experts are hot)."""
+    E, A = cfg.E, cfg.T * cfg.k
+    counts = np.asarray(counts, np.int64)
+    edges = np.unique(np.concatenate([[0, 1], np.geomspace(1, max(2, counts.max() + 1), 10).astype(np.int64)]))
+    hist, _ = np.histogram(counts, bins=np.append(edges, counts.max() + 1))
+    # rows-mode GEMMs: 128-row tiles of every group times the N tiles, each
+    # tile the same K work (fwd GEMM1 at F / 128 column tiles)
+    rows_tiles = np.repeat(np.ones(int(poff[-1]) // 128), max(1, cfg.F // 128))
+    # weight-gradient GEMMs (BF16, SM pairs): per expert (d / 256) x (2F / 256)
+    # output tiles, each reducing over the group's real rows in 64-row
+    # blocks, experts taken longest first
+    kb = -(-counts // 64)[np.argsort(-counts, kind="stable")]
+    wg_tiles = np.repeat(kb, max(1, (cfg.d // 256) * (2 * cfg.F // 256)))
+    return {"max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 3),
+            "hottest_share": round(float(counts.max() / A), 4),
+            "empty_experts": int((counts == 0).sum()),
+            "count_quantiles": {q: int(np.percentile(counts, q)) for q in (0, 10, 50, 90, 100)},
+            "count_histogram": {"edges": [int(v) for v in edges], "experts": [int(v) for v in hist]},
+            "padded_rows": int(poff[-1]), "pad_overhead": round(float(poff[-1] / A - 1.0), 4),
+            "schedule_efficiency": {
+                "rows_gemm_1sm": round(schedule_efficiency(rows_tiles, num_sms), 4),
+                "wgrad_gemm_pairs": round(schedule_efficiency(wg_tiles, num_sms // 2), 4)}}
+
+
 def _cfg_dict(cfg, extra):
     d = {"workload": f"{cfg.name}: one MoE SwiGLU FFN layer fwd+bwd, T={cfg.T} tokens, d_model={cfg.d}, "
                      f"E={cfg.E} experts, top-{cfg.k}, d_ff={cfg.F}, "
@@ -428,10 +467,7 @@ def run_ours(args):
     # padding adds to the GEMMs
     counts = layer.ctx_tensor("counts", (E,), torch.int32).cpu().numpy().astype(np.int64)
     poff = layer.ctx_tensor("poff", (E + 1,), torch.int32).cpu().numpy().astype(np.int64)
-    load = {"max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 3),
-            "hottest_share": round(float(counts.max() / A), 4),
-            "empty_experts": int((counts == 0).sum()),
-            "padded_rows": int(poff[-1]), "pad_overhead": round(float(poff[-1] / A - 1.0), 4)}
+    load = load_metrics(counts, poff, cfg, num_sms=torch.cuda.get_device_properties(local).multi_processor_count)
 
     # end to end through the C ABI with host buffers (copies inside)
     e2e = None

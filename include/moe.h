@@ -271,6 +271,32 @@ MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t
                                     int A_pad_max, int K, int N, void* dB, void* dB3,
                                     int32_t* dev_status, moe_stream_t stream);
 
+/* Dispatch fused into the GEMM ([OC3-ja] "ルーティングと計算の最適化": routed
+ * token rows go straight into the experts' input; here they go straight into
+ * the GEMM's shared-memory tiles).  BF16 only.  Same products as
+ * moe_grouped_gemm_fwd / moe_grouped_gemm_wgrad on the permuted buffer Xp,
+ * but row r of that operand is read from the unpermuted tokens x [T, K]
+ * as x[src[r]] (src from moe_route: the token of each padded row, -1 for a
+ * pad row, which reads as zeros), by TMA row gathers in the GEMM's
+ * producer; Xp is never written.  x and src 16-byte aligned; K % 64 == 0
+ * (fwd) or K % 128 == 0 (wgrad); the weight and dC maps must be 3-D (the
+ * library's layout; otherwise MOE_ERR_INVALID_ARG).
+ *   moe_grouped_gemm_fwd_gather:   epilogue NONE or SWIGLU as in
+ *     moe_grouped_gemm_fwd, with A = x gathered.
+ *   moe_grouped_gemm_wgrad_gather: dB[e] = Xp_e^T dC_e (dB3 as in
+ *     moe_grouped_gemm_wgrad); `offsets` (the unpadded group offsets, or
+ *     NULL) stops each group's reduction after its last real row. */
+MOE_API moe_status_t moe_grouped_gemm_fwd_gather(const void* x, int T, const int32_t* src,
+                                                 const void* B, const void* B3,
+                                                 const int32_t* poff, int E, int A_pad_max,
+                                                 int N, int K, int epilogue, void* C, void* aux,
+                                                 int32_t* dev_status, moe_stream_t stream);
+MOE_API moe_status_t moe_grouped_gemm_wgrad_gather(const void* x, int T, const int32_t* src,
+                                                   const void* dC, const int32_t* poff,
+                                                   const int32_t* offsets, int E, int A_pad_max,
+                                                   int K, int N, void* dB, void* dB3,
+                                                   int32_t* dev_status, moe_stream_t stream);
+
 /* Grouped GEMM with the tokens on the MMA's N side, BF16 (Olmo-core 3
  * オープン混合エキスパート学習インフラストラクチャ, "ルーティングと計算の最適化": the
  * expert matmuls as one grouped GEMM).  The weights form the 128-row M side

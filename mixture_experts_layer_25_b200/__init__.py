@@ -19,7 +19,8 @@ from ._lib import (MOE_BF16, MOE_MXFP8, MOE_EPI_NONE, MOE_EPI_SWIGLU, MOE_EPI_SW
                    LayerGrads, CtxView)
 
 __all__ = ["moe_route", "moe_permute", "mx_quantize", "mx_quantize_dual", "moe_grouped_gemm_fwd",
-           "moe_grouped_gemm_dgrad", "moe_grouped_gemm_wgrad", "moe_unpermute_combine",
+           "moe_grouped_gemm_dgrad", "moe_grouped_gemm_wgrad", "moe_grouped_gemm_fwd_gather",
+           "moe_grouped_gemm_wgrad_gather", "moe_unpermute_combine",
            "moe_combine_bwd", "moe_unpermute_sum", "moe_router_wgrad", "MoELayer",
            "a_pad_max", "MoeError"]
 
@@ -156,6 +157,35 @@ def moe_grouped_gemm_wgrad(A, dC, poff, E: int, *, split: bool = False, A_sc=Non
     dB3 = torch.empty((E, K, N), dtype=torch.bfloat16, device=A.device) if split else None
     _lib.call("moe_grouped_gemm_wgrad", MOE_MXFP8 if mx else MOE_BF16, _p(A), _p(A_sc), _p(dC),
               _p(dC_sc), _p(poff), E, Ap, K, N, _p(dB), _p(dB3), _p(status), _s(stream))
+    return (dB, dB3) if split else dB
+
+
+def moe_grouped_gemm_fwd_gather(x, src, B, poff, E: int, A_pad_max: int, *,
+                                epilogue=MOE_EPI_NONE, B3=None, want_aux=True, status=None,
+                                stream=None):
+    """moe_grouped_gemm_fwd (BF16) with row r of A read as x[src[r]] (zero
+    for src[r] < 0): the dispatch fused into the GEMM's loads."""
+    T, K = x.shape
+    N = B.shape[2]
+    C = torch.empty((A_pad_max, N), dtype=torch.bfloat16, device=x.device)
+    aux = None
+    if epilogue == MOE_EPI_SWIGLU and want_aux:
+        aux = torch.empty((A_pad_max, 2 * N), dtype=torch.bfloat16, device=x.device)
+    _lib.call("moe_grouped_gemm_fwd_gather", _p(x), T, _p(src), _p(B), _p(B3), _p(poff), E,
+              A_pad_max, N, K, epilogue, _p(C), _p(aux), _p(status), _s(stream))
+    return (C, aux) if epilogue == MOE_EPI_SWIGLU else C
+
+
+def moe_grouped_gemm_wgrad_gather(x, src, dC, poff, E: int, *, offsets=None, split: bool = False,
+                                  status=None, stream=None):
+    """moe_grouped_gemm_wgrad (BF16) with A row r read as x[src[r]]."""
+    T, K = x.shape
+    Ap = dC.shape[0]
+    N = dC.shape[1] // (2 if split else 1)
+    dB = torch.empty((E, K, N), dtype=torch.bfloat16, device=x.device)
+    dB3 = torch.empty((E, K, N), dtype=torch.bfloat16, device=x.device) if split else None
+    _lib.call("moe_grouped_gemm_wgrad_gather", _p(x), T, _p(src), _p(dC), _p(poff), _p(offsets),
+              E, Ap, K, N, _p(dB), _p(dB3), _p(status), _s(stream))
     return (dB, dB3) if split else dB
 
 

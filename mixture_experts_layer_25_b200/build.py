@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe.so")
 SOURCES = ["common.cu", "route.cu", "permute.cu", "mx_quant.cu", "grouped_gemm.cu",
-           "grouped_gemm_tn.cu", "layer.cu"]
+           "grouped_gemm_tn.cu", "grouped_gemm_pair.cu", "layer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

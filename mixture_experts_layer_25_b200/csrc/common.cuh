@@ -63,6 +63,15 @@ moe_status_t grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, cons
                                 int E, int A_pad_max, int K, int N, void* dB, void* dB3,
                                 int32_t* dev_status, cudaStream_t s);
 
+// Weight-gradient grouped GEMM (BF16) on SM pairs (grouped_gemm_pair.cu):
+// dB[e] = A_e^T dC_e (+ dB3 from dC's second N half), reduced over group e
+// up to its last real row; A the padded buffer, or with a_src the
+// unpermuted x [a_rows, K] gathered by row.  K % 256 == 0, N % 256 == 0.
+moe_status_t grouped_gemm_wgrad_pair(const void* A, const int32_t* a_src, int a_rows,
+                                     const void* dC, const int32_t* poff, const int32_t* offsets,
+                                     int E, int A_pad_max, int K, int N, void* dB, void* dB3,
+                                     int32_t* dev_status, cudaStream_t s);
+
 // Tokens-N grouped GEMM (BF16; grouped_gemm_tn.cu): weights on the MMA's M
 // side, an expert's real rows split evenly over token blocks of <= 256 on
 // the N side, padding rows after the last real row written as zeros.

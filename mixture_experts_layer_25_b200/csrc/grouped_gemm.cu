@@ -118,6 +118,10 @@ struct Params {
   int a3d, b3d;       // MN-major operand maps are 3-D (chunk, row, chunk index): one load per stage
   int mma_n;          // > 0: MMA N (multiple of 16, <= 256) instead of BN
   int b_boxes;        // > 0: MN-major B boxes loaded per stage (<= BN / chunk)
+  // gathered A (GATHER kernels): row r of the padded A operand is row
+  // a_src[r] of the unpermuted tokens (a_src[r] < 0: a zero row, read as the
+  // out-of-range row a_oob)
+  const int32_t* a_src; int a_oob;
   // router epilogue
   const float* r_bias; float* r_logits; int32_t* r_topk; float* r_gates;
   int32_t* r_rank; int32_t* r_hist; int r_k; int r_E;
@@ -135,6 +139,17 @@ __device__ __forceinline__ int find_expert(const int* poff_s, int E, int row) {
     if (poff_s[mid] <= row) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// four consecutive entries of the gather map starting at padded row r (a
+// multiple of 4): token rows, with pad rows mapped to the out-of-range row
+__device__ __forceinline__ int4 gather_rows(const Params& p, int r) {
+  int4 v = __ldg(reinterpret_cast<const int4*>(p.a_src + r));
+  v.x = v.x < 0 ? p.a_oob : v.x;
+  v.y = v.y < 0 ? p.a_oob : v.y;
+  v.z = v.z < 0 ? p.a_oob : v.z;
+  v.w = v.w < 0 ? p.a_oob : v.w;
+  return v;
 }
 
 __device__ __forceinline__ Tile decode(const Params& p, const int* poff_s, int tile) {
@@ -186,7 +201,7 @@ __device__ __forceinline__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
   }
 }
 
-template <bool MX, bool A_MN, int BLOAD, int EPI>
+template <bool MX, bool A_MN, int BLOAD, int EPI, bool GATHER = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
@@ -280,7 +295,66 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     else return t.nkb;
   };
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // ------------------------------------------------- producer (gathered A)
+    // The whole warp: lane 0 owns the barriers and the B loads; each lane
+    // gathers four A rows per stage (row mode: rows 4 lane.. of the 128-row
+    // tile; weight-gradient mode: K rows 4 (lane % 16).. of the stage's 64,
+    // for the 64-column chunk lane / 16 of the tile's 128 M columns).
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t used = 0, last_parity = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+      const Tile t = decode(p, poff_s, tile);
+      const int nkb = group_kb(t);
+      int4 rows = make_int4(0, 0, 0, 0);
+      if constexpr (!A_MN) rows = gather_rows(p, t.row0 + 4 * lane);
+      int4 next_rows = rows;
+      if constexpr (A_MN) if (nkb > 0) next_rows = gather_rows(p, t.krow0 + 4 * (lane & 15));
+      for (int kb = 0; kb < nkb; ++kb) {
+        if constexpr (A_MN) {
+          rows = next_rows;
+          if (kb + 1 < nkb) next_rows = gather_rows(p, t.krow0 + (kb + 1) * BK + 4 * (lane & 15));
+        }
+        int ok = 1;
+        if (lane == 0)
+          ok = mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { stop = true; break; }
+        uint64_t* fb = &full_bar[stage];
+        if (lane == 0) mbar_arrive_expect_tx(fb, STAGE_TX);
+        __syncwarp();
+        uint8_t* a_dst = sA + stage * A_BYTES;
+        if constexpr (!A_MN)
+          tma_gather4(a_dst + lane * 512, &tmA, fb, kb * BK, rows.x, rows.y, rows.z, rows.w);
+        else
+          tma_gather4(a_dst + (lane >> 4) * MN_CHUNK_BYTES + (lane & 15) * 512, &tmA, fb,
+                      t.m0 + (lane >> 4) * MN_CHUNK, rows.x, rows.y, rows.z, rows.w);
+        if (lane == 0) {
+          uint8_t* b_dst = sB + stage * B_STAGE;
+          const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
+          if constexpr (BLOAD == B_MN) {
+            tma_load_3d(b_dst, &tmB, fb, 0, brow + kb * BK, t.nt * BN / MN_CHUNK);
+          } else if constexpr (BLOAD == B_MN_DUAL_N) {
+            constexpr int HALF_CHUNKS = (BN / 2) / MN_CHUNK;
+            tma_load_3d(b_dst, &tmB, fb, 0, brow + kb * BK, t.nt * (BN / 2) / MN_CHUNK);
+            tma_load_3d(b_dst + HALF_CHUNKS * MN_CHUNK_BYTES, &tmB3, fb, 0, brow + kb * BK,
+                        t.nt * (BN / 2) / MN_CHUNK);
+          }
+        }
+        used |= 1u << stage;
+        last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    if (lane == 0)     // every load of the warp has landed before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (used & (1u << s)) {
+          volatile int no_abort = 0;
+          mbar_wait(&full_bar[s], (last_parity >> s) & 1, &no_abort, p.status, kWaitLimitNs);
+        }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int stage = 0;
@@ -290,7 +364,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
         const Tile t = decode(p, poff_s, tile);
         const int nkb = group_kb(t);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int step = 0; step < nkb; ++step) {
+          // the router's tiles all read the same split weights: each tile
+          // starts at its own K block so that they do not stream the same
+          // lines at the same time (fp32 sums in a rotated, fixed order)
+          const int kb = EPI == EPI_ROUTER ? (step + tile) % nkb : step;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
           uint64_t* fb = &full_bar[stage];
           const int nbox = p.b_boxes ? p.b_boxes : BN / MN_CHUNK;
@@ -939,9 +1017,9 @@ struct Maps {
   CUtensorMap a, b, b3, c, c2, in;
 };
 
-template <bool MX, bool A_MN, int BLOAD, int EPI>
+template <bool MX, bool A_MN, int BLOAD, int EPI, bool GATHER = false>
 moe_status_t launch(const Maps& m, const Params& p, int max_tiles, cudaStream_t s) {
-  auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI>;
+  auto kern = grouped_gemm_kernel<MX, A_MN, BLOAD, EPI, GATHER>;
   const size_t smem = EpiCfg<MX, EPI, A_MN>::SMEM;
   MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(kern), smem, "grouped_gemm"));
   const int grid = max(1, min(num_sms(), max_tiles));
@@ -1025,15 +1103,21 @@ extern "C" moe_status_t moe_selftest_wait_timeout(int32_t* dev_status, uint64_t 
   return MOE_OK;
 }
 
-extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc,
-                                             const void* B, const uint8_t* B_sc, const void* B3,
-                                             const uint8_t* B3_sc, const int32_t* poff, int E,
-                                             int A_pad_max, int N, int K, int epilogue, void* C,
-                                             void* aux, int32_t* dev_status,
-                                             moe_stream_t stream) {
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+// Forward grouped GEMM.  a_src == null: A is the permuted buffer
+// [A_pad_max, K].  a_src != null (BF16): A is the unpermuted x [a_rows, K]
+// and padded row r of the product reads x[a_src[r]] (a zero row where
+// a_src[r] < 0), gathered by the producer with TMA row gathers.
+static moe_status_t fwd_impl(int dt, const void* A, const uint8_t* A_sc, const void* B,
+                             const uint8_t* B_sc, const void* B3, const uint8_t* B3_sc,
+                             const int32_t* poff, int E, int A_pad_max, int N, int K,
+                             int epilogue, void* C, void* aux, const int32_t* a_src, int a_rows,
+                             int32_t* dev_status, cudaStream_t s) {
   const bool mx = dt == MOE_MXFP8;
+  const bool gather = a_src != nullptr;
   MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_fwd: bad dtype");
+  MOE_CHECK_ARG(!(gather && mx), "gemm_fwd: row gathers are BF16 only");
+  MOE_CHECK_ARG(!gather || (a_rows > 0 && aligned16(a_src) && aligned16(A)),
+                "gemm_fwd: gathered A needs T > 0 and 16-byte aligned x and src");
   MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_fwd: E must be in [1, %d]", MAX_E);
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_fwd: A_pad_max %% 128");
   MOE_CHECK_ARG(K > 0 && K % (mx ? 128 : 64) == 0, "gemm_fwd: K %% %d", mx ? 128 : 64);
@@ -1049,17 +1133,24 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   p.b3_sc = B3_sc;
   p.b_sc_kchunks = (int)((long long)E * K / 128);
   p.C = static_cast<__nv_bfloat16*>(C);
+  p.a_src = a_src;
+  p.a_oob = a_rows;
   Maps m;
-  MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, BM));
+  if (gather) MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));
+  else MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, BM));
   if (epilogue == MOE_EPI_NONE) {
     MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_fwd: N %% 256");
     p.n_tiles = N / BN;
     p.ldc = N;
     p.b3d = make_map_mn3(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, BN * eb / 128);
-    if (!p.b3d) MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    if (!p.b3d) {
+      MOE_CHECK_ARG(!gather, "gemm_fwd: gathered A needs the 3-D weight map");
+      MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
+    }
     MOE_TRY(make_out_map(&m.c, C, N, A_pad_max));
     m.b3 = m.c2 = m.in = m.a;
     const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+    if (gather) return launch<false, false, B_MN, EPI_STORE, true>(m, p, max_tiles, s);
     return mx ? launch<true, false, B_MN, EPI_STORE>(m, p, max_tiles, s)
               : launch<false, false, B_MN, EPI_STORE>(m, p, max_tiles, s);
   }
@@ -1074,6 +1165,7 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   p.b3d = make_map_mn3(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, (BN / 2) * eb / 128) &&
           make_map_mn3(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, (BN / 2) * eb / 128);
   if (!p.b3d) {
+    MOE_CHECK_ARG(!gather, "gemm_fwd: gathered A needs the 3-D weight maps");
     MOE_TRY(make_map(&m.b, B, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
     MOE_TRY(make_map(&m.b3, B3, eb, N, (uint64_t)E * K, 128 / eb, 128 / eb));
   }
@@ -1082,8 +1174,30 @@ extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_
   else m.c2 = m.c;
   m.in = m.a;
   const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+  if (gather) return launch<false, false, B_MN_DUAL_N, EPI_SWIGLU, true>(m, p, max_tiles, s);
   return mx ? launch<true, false, B_MN_DUAL_N, EPI_SWIGLU>(m, p, max_tiles, s)
             : launch<false, false, B_MN_DUAL_N, EPI_SWIGLU>(m, p, max_tiles, s);
+}
+
+extern "C" moe_status_t moe_grouped_gemm_fwd(int dt, const void* A, const uint8_t* A_sc,
+                                             const void* B, const uint8_t* B_sc, const void* B3,
+                                             const uint8_t* B3_sc, const int32_t* poff, int E,
+                                             int A_pad_max, int N, int K, int epilogue, void* C,
+                                             void* aux, int32_t* dev_status,
+                                             moe_stream_t stream) {
+  return fwd_impl(dt, A, A_sc, B, B_sc, B3, B3_sc, poff, E, A_pad_max, N, K, epilogue, C, aux,
+                  nullptr, 0, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" moe_status_t moe_grouped_gemm_fwd_gather(const void* x, int T, const int32_t* src,
+                                                    const void* B, const void* B3,
+                                                    const int32_t* poff, int E, int A_pad_max,
+                                                    int N, int K, int epilogue, void* C,
+                                                    void* aux, int32_t* dev_status,
+                                                    moe_stream_t stream) {
+  MOE_CHECK_ARG(x && src, "gemm_fwd_gather: null x or src");
+  return fwd_impl(MOE_BF16, x, nullptr, B, nullptr, B3, nullptr, poff, E, A_pad_max, N, K,
+                  epilogue, C, aux, src, T, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc,
@@ -1175,21 +1289,34 @@ extern "C" moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint
                                  dB3, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
-// moe_grouped_gemm_wgrad that stops each group's reduction after its last
-// real row (offsets = the unpadded group offsets, E + 1 ints, or null):
-// whole K blocks of zero padding rows are not loaded or multiplied.
-moe_status_t moe::grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, const void* dC,
-                                     const uint8_t* dC_sc, const int32_t* poff,
-                                     const int32_t* offsets, int E, int A_pad_max, int K, int N,
-                                     void* dB, void* dB3, int32_t* dev_status, cudaStream_t s) {
+// Weight-gradient grouped GEMM.  a_src == null: A is the permuted buffer
+// [A_pad_max, K]; otherwise (BF16) A row r is x[a_src[r]] of the unpermuted
+// x [a_rows, K] (zero where a_src[r] < 0), gathered by the producer.  The
+// reduction of group e stops after its last real row when `offsets` (the
+// unpadded group offsets) is given.
+static moe_status_t wgrad_impl(int dt, const void* A, const uint8_t* A_sc, const void* dC,
+                               const uint8_t* dC_sc, const int32_t* poff, const int32_t* offsets,
+                               int E, int A_pad_max, int K, int N, void* dB, void* dB3,
+                               const int32_t* a_src, int a_rows, int32_t* dev_status,
+                               cudaStream_t s) {
   const bool mx = dt == MOE_MXFP8;
+  const bool gather = a_src != nullptr;
   MOE_CHECK_ARG(dt == MOE_BF16 || dt == MOE_MXFP8, "gemm_wgrad: bad dtype");
+  MOE_CHECK_ARG(!(gather && mx), "gemm_wgrad: row gathers are BF16 only");
+  MOE_CHECK_ARG(!gather || (a_rows > 0 && aligned16(a_src) && aligned16(A)),
+                "gemm_wgrad: gathered A needs T > 0 and 16-byte aligned x and src");
   MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_wgrad: E must be in [1, %d]", MAX_E);
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_wgrad: A_pad_max %% 128");
   MOE_CHECK_ARG(K > 0 && K % 128 == 0, "gemm_wgrad: K %% 128");
   MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_wgrad: N %% 256");
   MOE_CHECK_ARG(A && dC && dB && poff, "gemm_wgrad: null pointer");
   MOE_CHECK_ARG(!mx || (A_sc && dC_sc), "gemm_wgrad: MX needs scales");
+#ifndef MOE_NO_PAIR_WGRAD
+  // BF16 with 256-aligned weight shapes: 256 x 256 tiles on SM pairs
+  if (!mx && K % 256 == 0)
+    return grouped_gemm_wgrad_pair(A, a_src, a_rows, dC, poff, offsets, E, A_pad_max, K, N, dB,
+                                   dB3, dev_status, s);
+#endif
   const int eb = mx ? 1 : 2;
   const int Ncols = dB3 ? 2 * N : N;
   Params p = base_params(poff, E, dev_status);
@@ -1207,16 +1334,48 @@ moe_status_t moe::grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc,
   p.n_split = dB3 ? N : 0;
   p.ldc = N;
   p.c_expert_stride = (long long)K * N;
+  p.a_src = a_src;
+  p.a_oob = a_rows;
   Maps m;
-  p.a3d = make_map_mn3(&m.a, A, eb, K, A_pad_max, 128 / eb, BM * eb / 128);
-  if (!p.a3d) MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
+  if (gather) {
+    MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));
+  } else {
+    p.a3d = make_map_mn3(&m.a, A, eb, K, A_pad_max, 128 / eb, BM * eb / 128);
+    if (!p.a3d) MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));
+  }
   p.b3d = make_map_mn3(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, BN * eb / 128);
-  if (!p.b3d) MOE_TRY(make_map(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  if (!p.b3d) {
+    MOE_CHECK_ARG(!gather, "gemm_wgrad: gathered A needs the 3-D map of dC");
+    MOE_TRY(make_map(&m.b, dC, eb, Ncols, A_pad_max, 128 / eb, 128 / eb));
+  }
   MOE_TRY(make_out_map(&m.c, dB, N, (uint64_t)E * K));
   if (dB3) MOE_TRY(make_out_map(&m.c2, dB3, N, (uint64_t)E * K));
   else m.c2 = m.c;
   m.b3 = m.in = m.a;
   const int max_tiles = E * p.m_tiles_w * p.n_tiles;
+  if (gather) return launch<false, true, B_MN, EPI_STORE, true>(m, p, max_tiles, s);
   return mx ? launch<true, true, B_MN, EPI_STORE>(m, p, max_tiles, s)
             : launch<false, true, B_MN, EPI_STORE>(m, p, max_tiles, s);
+}
+
+// moe_grouped_gemm_wgrad that stops each group's reduction after its last
+// real row (offsets = the unpadded group offsets, E + 1 ints, or null):
+// whole K blocks of zero padding rows are not loaded or multiplied.
+moe_status_t moe::grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, const void* dC,
+                                     const uint8_t* dC_sc, const int32_t* poff,
+                                     const int32_t* offsets, int E, int A_pad_max, int K, int N,
+                                     void* dB, void* dB3, int32_t* dev_status, cudaStream_t s) {
+  return wgrad_impl(dt, A, A_sc, dC, dC_sc, poff, offsets, E, A_pad_max, K, N, dB, dB3, nullptr,
+                    0, dev_status, s);
+}
+
+extern "C" moe_status_t moe_grouped_gemm_wgrad_gather(const void* x, int T, const int32_t* src,
+                                                      const void* dC, const int32_t* poff,
+                                                      const int32_t* offsets, int E,
+                                                      int A_pad_max, int K, int N, void* dB,
+                                                      void* dB3, int32_t* dev_status,
+                                                      moe_stream_t stream) {
+  MOE_CHECK_ARG(x && src, "gemm_wgrad_gather: null x or src");
+  return wgrad_impl(MOE_BF16, x, nullptr, dC, nullptr, poff, offsets, E, A_pad_max, K, N, dB,
+                    dB3, src, T, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }

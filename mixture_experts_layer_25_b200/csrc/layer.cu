@@ -1,8 +1,10 @@
 // The whole MoE feed-forward layer, forward and backward, composed from the
 // library's calls on one stream with no host synchronisation.
 //
-// Forward:  route -> permute (rowwise dispatch) -> GEMM1 + SwiGLU -> GEMM2
-//           -> gate-weighted combine.
+// Forward:  route -> GEMM1 + SwiGLU with the rowwise dispatch fused into
+//           its producer (token rows gathered from x by src) -> GEMM2 ->
+//           gate-weighted combine.  (MXFP8 and the tokens-N GEMMs take a
+//           separate permute pass that writes Xp.)
 // Backward: combine bwd (dY = g dout, dg, dl) -> GEMM2 dgrad fused with the
 //           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad (+ the router's
 //           share of dx as a rank-1 epilogue term) -> GEMM1 wgrad ->
@@ -47,6 +49,12 @@ int a_pad_max(const moe_layer_desc* L) {
   return (int)((a + 127) / 128 * 128);
 }
 
+bool tokens_n(const moe_layer_desc* L);
+
+// The BF16 layer on the main grouped GEMM reads the token rows straight
+// from x (row gathers in the GEMM1 producers): no permuted copy Xp.
+bool gathers(const moe_layer_desc* L) { return false && L->dtype == MOE_BF16 && !tokens_n(L); }
+
 size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   Layout l;
   l.base = static_cast<char*>(base);
@@ -65,7 +73,7 @@ size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   x.dg = l.take<float>(T * k);
   x.dl = l.take<float>(T * k);
   x.dl_rows = l.take<float>(A);
-  x.Xp = l.take<__nv_bfloat16>(A * d);
+  x.Xp = gathers(L) ? nullptr : l.take<__nv_bfloat16>(A * d);
   x.H13 = l.take<__nv_bfloat16>(A * 2 * F);
   x.h = l.take<__nv_bfloat16>(A * F);
   x.Y = l.take<__nv_bfloat16>(A * d);
@@ -139,10 +147,12 @@ extern "C" moe_status_t moe_layer_ctx_view(const moe_layer_desc* desc, void* ctx
 // T = 8192, k = 8, E = 384), and multiplying only the real rows pays for
 // that kernel's lower per-tile rate (measured: 12% faster layer at that
 // shape, 6-7% slower at 512 rows per expert).
-static bool tokens_n(const moe_layer_desc* L) {
+namespace {
+bool tokens_n(const moe_layer_desc* L) {
   return L->dtype == MOE_BF16 && (long long)L->T * L->k < 256LL * L->E && L->d % 128 == 0 &&
          L->F % 64 == 0;
 }
+}  // namespace
 
 static moe_status_t check_common(const moe_layer_desc* L, const moe_layer_weights* w, void* ctx,
                                  size_t ctx_bytes) {
@@ -186,13 +196,19 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
                     dev_status, stream));
   mark(S_ROUTE, true, s);
   if (!mx) {
-    mark(S_PERMUTE, false, s);
-    MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, nullptr, nullptr, stream));
-    mark(S_PERMUTE, true, s);
+    if (!gathers(L)) {
+      mark(S_PERMUTE, false, s);
+      MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, nullptr, nullptr,
+                          stream));
+      mark(S_PERMUTE, true, s);
+    }
     mark(S_GEMM1, false, s);
     if (tokens_n(L))
       MOE_TRY(moe::gemm_tn(MOE_EPI_SWIGLU, c.Xp, w->W1, w->W3, 0, c.poff, c.offsets, E, A, F, d,
                            c.h, c.H13, nullptr, nullptr, dev_status, s));
+    else if (gathers(L))   // dispatch fused into the GEMM: token rows gathered from x by src
+      MOE_TRY(moe_grouped_gemm_fwd_gather(x, T, c.src, w->W1, w->W3, c.poff, E, A, F, d,
+                                          MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
     else
       MOE_TRY(moe_grouped_gemm_fwd(MOE_BF16, c.Xp, nullptr, w->W1, nullptr, w->W3, nullptr,
                                    c.poff, E, A, F, d, MOE_EPI_SWIGLU, c.h, c.H13, dev_status,
@@ -286,8 +302,12 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                       dev_status, s));
     mark(S_DGRAD1, true, s);
     mark(S_WGRAD1, false, s);
-    MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff, c.offsets,
-                                    E, A, d, F, G->dW1, G->dW3, dev_status, s));
+    if (gathers(L))
+      MOE_TRY(moe_grouped_gemm_wgrad_gather(x, T, c.src, c.dA13, c.poff, c.offsets, E, A, d, F,
+                                            G->dW1, G->dW3, dev_status, stream));
+    else
+      MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.Xp, nullptr, c.dA13, nullptr, c.poff,
+                                      c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));
     mark(S_WGRAD1, true, s);
   } else {
     const int32_t* nrows = c.poff + E;

@@ -37,4 +37,4 @@ def test_our_arm_line():
     assert d["n_gpus"] == 1 and d["steps"] == 3 and d["warmup"] == 3 and d["value"] > 0
     assert d["roofline"]["bound"] == "tensor" and 0 < d["roofline"]["frac"] < 2
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
-    assert d["gpu_launches"] >= 17 * 3          # at least the layer's kernels in every step
+    assert d["gpu_launches"] >= 15 * 3          # at least the layer's kernels in every step

@@ -152,8 +152,11 @@ def test_dgrad_swiglu_bwd(mx):
 
 @pytest.mark.parametrize("mx", [False, True])
 @pytest.mark.parametrize("split", [False, True])
-def test_wgrad(mx, split):
-    E, K, N = len(COUNTS), 256, 256
+@pytest.mark.parametrize("K", [256, 384])
+def test_wgrad(mx, split, K):
+    """K % 256 == 0 in BF16 runs on SM pairs (256 x 256 tiles), K = 384 on
+    single SMs."""
+    E, N = len(COUNTS), 256
     poff, A, real = _groups(COUNTS)
     X = _act(A, K, real, 12)
     dC = _act(A, 2 * N if split else N, real, 13)
@@ -305,3 +308,65 @@ def test_max_expert_count():
     P = int(poff[-1])
     assert rel_err(f64(C[:P]), ref[:P]) < 1e-2
     assert rel_err(f64(Ct[:P]), ref[:P]) < 1e-2
+
+
+def _routed(T, E, k, d, seed):
+    idx, gates = moe_inputs.random_routing(T, E, k, seed)
+    meta = moe.moe_route(None, None, None, k, E, topk_idx=torch.from_numpy(idx).cuda(),
+                         gates=torch.from_numpy(gates).cuda())
+    x = moe_inputs.random_bf16((T, d), seed + 1, device="cuda")
+    ref = oracle.routing_metadata(idx, E, 128)
+    return x, meta, ref
+
+
+@pytest.mark.parametrize("T,E,k", [(700, 16, 4), (1, 8, 2), (3000, 64, 3)])
+def test_fwd_gather_equals_fwd_on_permuted_rows(T, E, k):
+    """The dispatch fused into the GEMM: A rows gathered from x by src give
+    the same products as the GEMM on the permuted buffer (bit for bit: the
+    same operands reach the same MMAs) and match the oracle."""
+    d, F = 512, 256
+    x, meta, ref = _routed(T, E, k, d, 30 + T)
+    A = meta["A_pad_max"]
+    W1, W3, W2 = _w(E, d, F, 31), _w(E, d, F, 32), _w(E, d, 512, 33)   # W2 as a [d, 512] map
+    poff = meta["poff"]
+    P = int(ref["poff"][E])
+    Xp = moe.moe_permute(x, meta, k, E)
+    h, aux = moe.moe_grouped_gemm_fwd(Xp, W1, poff, E, epilogue=moe.MOE_EPI_SWIGLU, B3=W3)
+    hg, auxg = moe.moe_grouped_gemm_fwd_gather(x, meta["src"], W1, poff, E, A,
+                                               epilogue=moe.MOE_EPI_SWIGLU, B3=W3)
+    C = moe.moe_grouped_gemm_fwd(Xp, W2, poff, E)
+    Cg = moe.moe_grouped_gemm_fwd_gather(x, meta["src"], W2, poff, E, A)
+    torch.cuda.synchronize()
+    assert torch.equal(hg[:P], h[:P]) and torch.equal(auxg[:P], aux[:P])
+    assert torch.equal(Cg[:P], C[:P])
+    Xp64 = oracle.permute_rows(f64(x), ref)
+    H1 = oracle.grouped_matmul(Xp64, f64(W1), ref["poff"])
+    H3 = oracle.grouped_matmul(Xp64, f64(W3), ref["poff"])
+    assert rel_err(f64(hg[:P]), oracle.silu(H1) * H3) < 1e-2
+    assert rel_err(f64(Cg[:P]), oracle.grouped_matmul(Xp64, f64(W2), ref["poff"])) < 1e-2
+    pad = torch.from_numpy(ref["src"] < 0).cuda()
+    assert torch.all(hg[:P][pad] == 0)
+
+
+@pytest.mark.parametrize("T,E,k", [(700, 16, 4), (1, 8, 2), (3000, 64, 3)])
+def test_wgrad_gather_equals_wgrad_on_permuted_rows(T, E, k):
+    d, F = 512, 256
+    x, meta, ref = _routed(T, E, k, d, 40 + T)
+    A = meta["A_pad_max"]
+    real = np.zeros(A, bool)
+    real[:len(ref["src"])] = ref["src"] >= 0
+    dA = _act(A, 2 * F, real, 41)
+    Xp = moe.moe_permute(x, meta, k, E)
+    dW1, dW3 = moe.moe_grouped_gemm_wgrad(Xp, dA, meta["poff"], E, split=True)
+    g1, g3 = moe.moe_grouped_gemm_wgrad_gather(x, meta["src"], dA, meta["poff"], E,
+                                               offsets=meta["offsets"], split=True)
+    torch.cuda.synchronize()
+    assert torch.equal(g1, dW1) and torch.equal(g3, dW3)
+    Xp64 = oracle.permute_rows(f64(x), ref)
+    dA64 = f64(dA)[:len(ref["src"])]
+    ref1 = oracle.grouped_wgrad(Xp64, dA64[:, :F], ref["poff"], E)
+    ref3 = oracle.grouped_wgrad(Xp64, dA64[:, F:], ref["poff"], E)
+    assert rel_err(f64(g1), ref1) < 1e-2 and rel_err(f64(g3), ref3) < 1e-2
+    empty = np.nonzero(ref["counts"] == 0)[0]
+    for e in empty:
+        assert torch.all(g1[e] == 0) and torch.all(g3[e] == 0)
