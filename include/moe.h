@@ -271,6 +271,62 @@ MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t
                                     int A_pad_max, int K, int N, void* dB, void* dB3,
                                     int32_t* dev_status, moe_stream_t stream);
 
+/* Rowwise dispatch straight into MX codes ([OC3-ja] "ルーティングと計算の最適化":
+ * routed token rows go directly into the experts' input buffers; "MXFP8に
+ * よる精度最適化").  Row r of the expert-contiguous buffer is token src[r]
+ * (src from moe_route; -1 = a zero pad row); it is written only as MX codes,
+ * along d (Xq [A_pad_max, d], Xs: scales along the row, K = d; the forward
+ * GEMM1 operand) and down the rows in blocks of 32 inside each group (XqT
+ * [A_pad_max, d], XsT: K = A_pad_max; the GEMM1 weight-gradient operand),
+ * bit-identical to mx_quantize_dual of the bf16 permuted buffer.  No bf16
+ * copy is written; rows from poff[E] on are not touched.  d % 256 == 0,
+ * A_pad_max % 128 == 0, x / Xq / XqT 16-byte aligned. */
+MOE_API moe_status_t moe_permute_mx(const void* x, const int32_t* src, const int32_t* poff,
+                                    int T, int d, int E, int A_pad_max, uint8_t* Xq,
+                                    uint8_t* Xs, uint8_t* XqT, uint8_t* XsT,
+                                    moe_stream_t stream);
+
+/* The backward's gate-scaled upstream rows straight into MX codes: row r of
+ * the expert-contiguous buffer, in group e, is dY[r] = bf16(g * dout[t])
+ * with t = src[r] and g = gates[t, j] for the slot j where topk_idx[t, j] =
+ * e (a zero row for src[r] < 0), written only as MX codes along d (dYq /
+ * dYs, K = d: GEMM2 dgrad) and down the rows (dYTq / dYTs, K = A_pad_max:
+ * GEMM2 weight gradient); bit-identical to mx_quantize_dual of the dY that
+ * moe_combine_bwd writes.  Rows from poff[E] on are not touched.  d % 256
+ * == 0, k <= 16. */
+MOE_API moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
+                                        const int32_t* topk_idx, const int32_t* src,
+                                        const int32_t* poff, int T, int k, int d, int E,
+                                        int A_pad_max, uint8_t* dYq, uint8_t* dYs,
+                                        uint8_t* dYTq, uint8_t* dYTs, moe_stream_t stream);
+
+/* MXFP8 GEMMs whose SwiGLU epilogues quantise their bf16 result instead of
+ * storing it ([OC3-ja] "MXFP8による精度最適化": the FP8 gain comes from
+ * faster feed-forward compute and less data movement).  Each epilogue warp
+ * owns a 32 x 32 block of the result, so both MX blocks of an element are
+ * local: along the row (32 columns of one row) and down the column (32 rows
+ * of one column, always inside one expert group).  Codes and scales are
+ * bit-identical to mx_quantize_dual of the bf16 result the plain MX call
+ * would store.  Scales in the tensor-core layout: along the row with K =
+ * the row length, down the columns with K = A_pad_max.  Rows >= poff[E]
+ * are not written.
+ *   moe_grouped_gemm_fwd_swiglu_mxq: as moe_grouped_gemm_fwd(MOE_MXFP8,
+ *     EPI_SWIGLU) with N = F; aux = [H1 | H3] bf16 (required); h -> h_q /
+ *     h_s (along F) and hT_q / hT_s (down the rows).  F % 128 == 0.
+ *   moe_grouped_gemm_dgrad_swiglu_mxq: as moe_grouped_gemm_dgrad(MOE_MXFP8,
+ *     EPI_SWIGLU_BWD) with B = W2 codes along N = d, K = F; dA = [dA1 | dA3]
+ *     [A_pad_max, 2F] -> dA_q / dA_s (along 2F) and dAT_q / dAT_s (down the
+ *     rows).  K % 256 == 0. */
+MOE_API moe_status_t moe_grouped_gemm_fwd_swiglu_mxq(
+    const void* A, const uint8_t* A_sc, const void* B, const uint8_t* B_sc, const void* B3,
+    const uint8_t* B3_sc, const int32_t* poff, int E, int A_pad_max, int F, int K, void* aux,
+    uint8_t* h_q, uint8_t* h_s, uint8_t* hT_q, uint8_t* hT_s, int32_t* dev_status,
+    moe_stream_t stream);
+MOE_API moe_status_t moe_grouped_gemm_dgrad_swiglu_mxq(
+    const void* dC, const uint8_t* dC_sc, const void* B, const uint8_t* B_sc,
+    const int32_t* poff, int E, int A_pad_max, int N, int K, const void* aux, uint8_t* dA_q,
+    uint8_t* dA_s, uint8_t* dAT_q, uint8_t* dAT_s, int32_t* dev_status, moe_stream_t stream);
+
 /* Dispatch fused into the GEMM ([OC3-ja] "ルーティングと計算の最適化": routed
  * token rows go straight into the experts' input; here they go straight into
  * the GEMM's shared-memory tiles).  BF16 only.  Same products as
@@ -342,6 +398,7 @@ MOE_API moe_status_t moe_unpermute_combine(const void* Y, const float* gates, co
 
 /* Backward of the combine: for each assignment (t,j) with r = dst[t,j]
  *   dY[r]    = bf16(gates[t,j] * dout[t]);  pad rows of dY are zeroed
+ *              (dY nullable: then only dg / dl / dl_rows are written)
  *   dg[t,j]  = <dout[t], Y[r]>  (fp32)
  *   and, when dl != NULL (router mode), the logit gradient of the chosen
  *   experts dl[t,j] = g_j (dg_j - sum_i g_i dg_i) (fp32), also scattered to

@@ -18,10 +18,10 @@ from ._lib import (MOE_BF16, MOE_MXFP8, MOE_EPI_NONE, MOE_EPI_SWIGLU, MOE_EPI_SW
                    MOE_DEV_TIMEOUT, MOE_DEV_NONFINITE, MoeError, LayerDesc, LayerWeights,
                    LayerGrads, CtxView)
 
-__all__ = ["moe_route", "moe_permute", "mx_quantize", "mx_quantize_dual", "moe_grouped_gemm_fwd",
+__all__ = ["moe_route", "moe_permute", "moe_permute_mx", "mx_quantize", "mx_quantize_dual", "moe_grouped_gemm_fwd",
            "moe_grouped_gemm_dgrad", "moe_grouped_gemm_wgrad", "moe_grouped_gemm_fwd_gather",
            "moe_grouped_gemm_wgrad_gather", "moe_unpermute_combine",
-           "moe_combine_bwd", "moe_unpermute_sum", "moe_router_wgrad", "MoELayer",
+           "moe_combine_bwd", "moe_combine_bwd_mx", "moe_unpermute_sum", "moe_router_wgrad", "MoELayer",
            "a_pad_max", "MoeError"]
 
 
@@ -91,6 +91,31 @@ def moe_permute(x, meta: dict, k: int, E: int, *, mx: bool = False, stream=None)
     _lib.call("moe_permute", _p(x), _p(meta["dst"]), _p(meta["offsets"]), _p(meta["poff"]), T, k,
               d, E, A, _p(Xp), _p(Xq), _p(Xs), _s(stream))
     return (Xp, Xq, Xs) if mx else Xp
+
+
+def moe_permute_mx(x, meta: dict, E: int, *, stream=None):
+    """Dispatch straight into MX codes: returns (codes, scales) of the
+    permuted rows along d and (codes, scales) down the rows."""
+    T, d = x.shape
+    A = meta["A_pad_max"]
+    mk = lambda *s: torch.empty(s, dtype=torch.uint8, device=x.device)  # noqa: E731
+    q, qs, qT, qTs = mk(A, d), mk(A * d // 32), mk(A, d), mk(A * d // 32)
+    _lib.call("moe_permute_mx", _p(x), _p(meta["src"]), _p(meta["poff"]), T, d, E, A, _p(q),
+              _p(qs), _p(qT), _p(qTs), _s(stream))
+    return (q, qs), (qT, qTs)
+
+
+def moe_combine_bwd_mx(dout, gates, meta: dict, E: int, *, stream=None):
+    """dY rows (gate-scaled dout, bf16-rounded) straight into MX codes:
+    (codes, scales) along d and (codes, scales) down the rows."""
+    T, d = dout.shape
+    k = meta["topk_idx"].shape[1]
+    A = meta["A_pad_max"]
+    mk = lambda *s: torch.empty(s, dtype=torch.uint8, device=dout.device)  # noqa: E731
+    q, qs, qT, qTs = mk(A, d), mk(A * d // 32), mk(A, d), mk(A * d // 32)
+    _lib.call("moe_combine_bwd_mx", _p(dout), _p(gates), _p(meta["topk_idx"]), _p(meta["src"]),
+              _p(meta["poff"]), T, k, d, E, A, _p(q), _p(qs), _p(qT), _p(qTs), _s(stream))
+    return (q, qs), (qT, qTs)
 
 
 def mx_quantize(t, axis: int, *, nrows=None, codes=None, scales=None, stream=None):
@@ -174,6 +199,37 @@ def moe_grouped_gemm_fwd_gather(x, src, B, poff, E: int, A_pad_max: int, *,
     _lib.call("moe_grouped_gemm_fwd_gather", _p(x), T, _p(src), _p(B), _p(B3), _p(poff), E,
               A_pad_max, N, K, epilogue, _p(C), _p(aux), _p(status), _s(stream))
     return (C, aux) if epilogue == MOE_EPI_SWIGLU else C
+
+
+def moe_grouped_gemm_fwd_swiglu_mxq(A, A_sc, B, B_sc, B3, B3_sc, poff, E: int, *, status=None,
+                                    stream=None):
+    """MXFP8 GEMM1 + SwiGLU whose h leaves as MX codes: returns aux = [H1 |
+    H3] bf16 and (h codes, h scales) along F and (codes, scales) down the rows."""
+    Ap, K = A.shape
+    F = B.shape[2]
+    dev = A.device
+    aux = torch.empty((Ap, 2 * F), dtype=torch.bfloat16, device=dev)
+    mk = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)  # noqa: E731
+    hq, hs, hTq, hTs = mk(Ap, F), mk(Ap * F // 32), mk(Ap, F), mk(Ap * F // 32)
+    _lib.call("moe_grouped_gemm_fwd_swiglu_mxq", _p(A), _p(A_sc), _p(B), _p(B_sc), _p(B3),
+              _p(B3_sc), _p(poff), E, Ap, F, K, _p(aux), _p(hq), _p(hs), _p(hTq), _p(hTs),
+              _p(status), _s(stream))
+    return aux, (hq, hs), (hTq, hTs)
+
+
+def moe_grouped_gemm_dgrad_swiglu_mxq(dC, dC_sc, B, B_sc, aux, poff, E: int, *, status=None,
+                                      stream=None):
+    """MXFP8 GEMM2 dgrad + SwiGLU backward whose dA = [dA1 | dA3] leaves as MX
+    codes: returns (codes, scales) along 2F and (codes, scales) down the rows.
+    B: W2 codes [E, F, d] quantised along d."""
+    Ap, N = dC.shape
+    K = B.shape[1]
+    dev = dC.device
+    mk = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)  # noqa: E731
+    q, qs, qT, qTs = mk(Ap, 2 * K), mk(Ap * 2 * K // 32), mk(Ap, 2 * K), mk(Ap * 2 * K // 32)
+    _lib.call("moe_grouped_gemm_dgrad_swiglu_mxq", _p(dC), _p(dC_sc), _p(B), _p(B_sc), _p(poff),
+              E, Ap, N, K, _p(aux), _p(q), _p(qs), _p(qT), _p(qTs), _p(status), _s(stream))
+    return (q, qs), (qT, qTs)
 
 
 def moe_grouped_gemm_wgrad_gather(x, src, dC, poff, E: int, *, offsets=None, split: bool = False,

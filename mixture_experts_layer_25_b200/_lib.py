@@ -70,6 +70,10 @@ _SIGS = {
     "moe_grouped_gemm_wgrad": (I, [I, P, P, P, P, P, I, I, I, I, P, P, P, P]),
     "moe_grouped_gemm_tn": (I, [I, P, P, P, I, P, P, I, I, I, I, P, P, P, P, P, P]),
     "moe_grouped_gemm_fwd_gather": (I, [P, I, P, P, P, P, I, I, I, I, I, P, P, P, P]),
+    "moe_permute_mx": (I, [P, P, P, I, I, I, I, P, P, P, P, P]),
+    "moe_combine_bwd_mx": (I, [P, P, P, P, P, I, I, I, I, I, P, P, P, P, P]),
+    "moe_grouped_gemm_fwd_swiglu_mxq": (I, [P, P, P, P, P, P, P, I, I, I, I, P, P, P, P, P, P, P]),
+    "moe_grouped_gemm_dgrad_swiglu_mxq": (I, [P, P, P, P, P, I, I, I, I, P, P, P, P, P, P, P]),
     "moe_grouped_gemm_wgrad_gather": (I, [P, I, P, P, P, P, I, I, I, I, P, P, P, P]),
     "moe_selftest_wait_timeout": (I, [P, ctypes.c_uint64, P]),
     "moe_unpermute_combine": (I, [P, P, P, I, I, I, P, P]),

@@ -34,6 +34,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "mx.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -125,6 +126,13 @@ struct Params {
   // router epilogue
   const float* r_bias; float* r_logits; int32_t* r_topk; float* r_gates;
   int32_t* r_rank; int32_t* r_hist; int r_k; int r_E;
+  // MXFP8 epilogues that quantise their bf16 output in place of storing it
+  // (SwiGLU: h; SwiGLU backward: dA1 | dA3): codes along the row and down
+  // the columns through the tmQr / tmQc maps, scale bytes in the
+  // tensor-core layouts with K = the row length (q_row_kchunks = cols / 128)
+  // and K = the padded rows (q_col_kchunks = A_pad_max / 128)
+  int quant;
+  uint8_t* q_sr; uint8_t* q_sc; int q_row_kchunks; int q_col_kchunks;
   int32_t* status;
 };
 
@@ -208,7 +216,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB3,
                     const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmC2,
-                    const __grid_constant__ CUtensorMap tmIn, const Params p) {
+                    const __grid_constant__ CUtensorMap tmIn,
+                    const __grid_constant__ CUtensorMap tmQr,
+                    const __grid_constant__ CUtensorMap tmQc, const Params p) {
   using Cfg = EpiCfg<MX, EPI, A_MN>;      // A MN-major <=> weight-gradient tiles
   constexpr int STAGES = Cfg::STAGES;
   constexpr int STG = Cfg::STG;
@@ -687,6 +697,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
           uint4 hkeep[ONE_BOX ? 4 : 1], gkeep[ONE_BOX ? 4 : 1], ukeep[ONE_BOX ? 4 : 1];
+          const bool q = MX && p.quant;       // h leaves as MX codes, not bf16
+          uint32_t hbits[MX ? 16 : 1];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint4 hw, gw, uw;
@@ -706,9 +718,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             if constexpr (ONE_BOX) {
               hkeep[j] = hw; gkeep[j] = gw; ukeep[j] = uw;
             } else {
-              *reinterpret_cast<uint4*>(stg + sw64(r, j)) = hw;
+              if constexpr (MX) {
+                hbits[4 * j] = hw.x; hbits[4 * j + 1] = hw.y;
+                hbits[4 * j + 2] = hw.z; hbits[4 * j + 3] = hw.w;
+              }
+              if (!q) *reinterpret_cast<uint4*>(stg + sw64(r, j)) = hw;
               *reinterpret_cast<uint4*>(stg + BOX_BYTES + sw64(r, j)) = gw;
               *reinterpret_cast<uint4*>(stg + 2 * BOX_BYTES + sw64(r, j)) = uw;
+            }
+          }
+          if constexpr (MX && !ONE_BOX) {
+            if (q) {
+              // the bf16-rounded h of this warp's 32 x 32 block, quantised
+              // along F (fwd GEMM2) and down the rows (GEMM2 weight grad)
+              float hv[32];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hbits[i]));
+                hv[2 * i] = f2.x;
+                hv[2 * i + 1] = f2.y;
+              }
+              mx_quant_block32(hv, stg, stg + 1024, p.q_sr, y0 + r, n0 + c, p.q_row_kchunks,
+                               p.q_sc, y0, p.q_col_kchunks);
             }
           }
           if constexpr (ONE_BOX) {
@@ -735,7 +766,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&tmC, stg, n0 + c, y0);
+              if (q) {
+                tma_store_2d(&tmQr, stg, n0 + c, y0);
+                tma_store_2d(&tmQc, stg + 1024, n0 + c, y0);
+              } else {
+                tma_store_2d(&tmC, stg, n0 + c, y0);
+              }
               if (p.aux) {
                 tma_store_2d(&tmC2, stg + BOX_BYTES, n0 + c, y0);
                 tma_store_2d(&tmC2, stg + 2 * BOX_BYTES, p.half + n0 + c, y0);
@@ -774,6 +810,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             in_pending &= ~(1u << pr);
           }
           if (!got) { ok = 0; break; }
+          const bool q = MX && p.quant;     // dA1 | dA3 leave as MX codes, not bf16
+          uint4 o1k[MX ? 4 : 1], o3k[MX ? 4 : 1];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float f1[8], f3[8], o1[8], o3[8];
@@ -787,14 +825,47 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               o1[i] = dh * f3[i] * sg * (1.0f + z * (1.0f - sg));
               o3[i] = dh * z * sg;
             }
-            *reinterpret_cast<uint4*>(b1 + sw64(r, j)) = pack8(o1);
-            *reinterpret_cast<uint4*>(b3 + sw64(r, j)) = pack8(o3);
+            const uint4 w1 = pack8(o1), w3 = pack8(o3);
+            if constexpr (MX) {
+              o1k[j] = w1;
+              o3k[j] = w3;
+            }
+            if (!q) {
+              *reinterpret_cast<uint4*>(b1 + sw64(r, j)) = w1;
+              *reinterpret_cast<uint4*>(b3 + sw64(r, j)) = w3;
+            }
+          }
+          if constexpr (MX) {
+            if (q) {
+              // the bf16-rounded dA1 and dA3 of this warp's 32 x 32 blocks,
+              // quantised along 2F (GEMM1 dgrad) and down the rows (GEMM1
+              // weight grad); the codes reuse the H1 / H3 boxes once every
+              // lane has read its row of them
+              __syncwarp();
+#pragma unroll
+              for (int o = 0; o < 2; ++o) {
+                const uint4* k4 = o == 0 ? o1k : o3k;
+                float dv[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) unpack8(k4[j], dv + 8 * j);
+                uint8_t* box = o == 0 ? b1 : b3;
+                mx_quant_block32(dv, box, box + 1024, p.q_sr, y0 + r, (o ? p.half : 0) + n0 + c,
+                                 p.q_row_kchunks, p.q_sc, y0, p.q_col_kchunks);
+              }
+            }
           }
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmC, b1, n0 + c, y0);
-            tma_store_2d(&tmC, b3, p.half + n0 + c, y0);
+            if (q) {
+              tma_store_2d(&tmQr, b1, n0 + c, y0);
+              tma_store_2d(&tmQc, b1 + 1024, n0 + c, y0);
+              tma_store_2d(&tmQr, b3, p.half + n0 + c, y0);
+              tma_store_2d(&tmQc, b3 + 1024, p.half + n0 + c, y0);
+            } else {
+              tma_store_2d(&tmC, b1, n0 + c, y0);
+              tma_store_2d(&tmC, b3, p.half + n0 + c, y0);
+            }
             bulk_commit();
           }
         }
@@ -1014,7 +1085,8 @@ moe_status_t make_out_map(CUtensorMap* m, const void* base, uint64_t inner, uint
 }
 
 struct Maps {
-  CUtensorMap a, b, b3, c, c2, in;
+  CUtensorMap a, b, b3, c, c2, in, qr, qc;
+  bool q = false;     // qr / qc set (MX epilogue quantisation)
 };
 
 template <bool MX, bool A_MN, int BLOAD, int EPI, bool GATHER = false>
@@ -1023,7 +1095,8 @@ moe_status_t launch(const Maps& m, const Params& p, int max_tiles, cudaStream_t 
   const size_t smem = EpiCfg<MX, EPI, A_MN>::SMEM;
   MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(kern), smem, "grouped_gemm"));
   const int grid = max(1, min(num_sms(), max_tiles));
-  kern<<<grid, NUM_THREADS, smem, s>>>(m.a, m.b, m.b3, m.c, m.c2, m.in, p);
+  kern<<<grid, NUM_THREADS, smem, s>>>(m.a, m.b, m.b3, m.c, m.c2, m.in, m.q ? m.qr : m.a,
+                                       m.q ? m.qc : m.a, p);
   MOE_CHECK_LAUNCH("grouped_gemm");
   return MOE_OK;
 }
@@ -1198,6 +1271,104 @@ extern "C" moe_status_t moe_grouped_gemm_fwd_gather(const void* x, int T, const 
   MOE_CHECK_ARG(x && src, "gemm_fwd_gather: null x or src");
   return fwd_impl(MOE_BF16, x, nullptr, B, nullptr, B3, nullptr, poff, E, A_pad_max, N, K,
                   epilogue, C, aux, src, T, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// MXFP8 forward GEMM1 with the SwiGLU epilogue whose h leaves as MX codes:
+// along F (h_q / h_s, for the forward GEMM2) and down the rows (hT_q / hT_s,
+// for the GEMM2 weight gradient), from the bf16-rounded h; aux [H1 | H3] as
+// in moe_grouped_gemm_fwd.  h itself is not stored.
+extern "C" moe_status_t moe_grouped_gemm_fwd_swiglu_mxq(
+    const void* A, const uint8_t* A_sc, const void* B, const uint8_t* B_sc, const void* B3,
+    const uint8_t* B3_sc, const int32_t* poff, int E, int A_pad_max, int F, int K, void* aux,
+    uint8_t* h_q, uint8_t* h_s, uint8_t* hT_q, uint8_t* hT_s, int32_t* dev_status,
+    moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_fwd_swiglu_mxq: E must be in [1, %d]", MAX_E);
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_fwd_swiglu_mxq: A_pad_max %% 128");
+  MOE_CHECK_ARG(K > 0 && K % 128 == 0 && F > 0 && F % 128 == 0, "gemm_fwd_swiglu_mxq: K, F %% 128");
+  MOE_CHECK_ARG(A && A_sc && B && B_sc && B3 && B3_sc && poff && aux,
+                "gemm_fwd_swiglu_mxq: null pointer");
+  MOE_CHECK_ARG(h_q && h_s && hT_q && hT_s && aligned16(h_q) && aligned16(hT_q),
+                "gemm_fwd_swiglu_mxq: null or unaligned MX output");
+  Params p = base_params(poff, E, dev_status);
+  p.num_kb = K / 128;
+  p.b_rows_per_e = K;
+  p.a_sc = A_sc;
+  p.a_sc_kchunks = K / 128;
+  p.b_sc = B_sc;
+  p.b3_sc = B3_sc;
+  p.b_sc_kchunks = (int)((long long)E * K / 128);
+  p.n_tiles = F / (BN / 2);
+  p.ldc = F;
+  p.aux = static_cast<__nv_bfloat16*>(aux);
+  p.ld_aux = 2LL * F;
+  p.half = F;
+  p.quant = 1;
+  p.q_sr = h_s;
+  p.q_sc = hT_s;
+  p.q_row_kchunks = F / 128;
+  p.q_col_kchunks = A_pad_max / 128;
+  Maps m;
+  MOE_TRY(make_map(&m.a, A, 1, K, A_pad_max, 128, BM));
+  p.b3d = make_map_mn3(&m.b, B, 1, F, (uint64_t)E * K, 128, (BN / 2) / 128) &&
+          make_map_mn3(&m.b3, B3, 1, F, (uint64_t)E * K, 128, (BN / 2) / 128);
+  if (!p.b3d) {
+    MOE_TRY(make_map(&m.b, B, 1, F, (uint64_t)E * K, 128, 128));
+    MOE_TRY(make_map(&m.b3, B3, 1, F, (uint64_t)E * K, 128, 128));
+  }
+  MOE_TRY(make_out_map(&m.c2, aux, 2ULL * F, A_pad_max));
+  MOE_TRY(make_map(&m.qr, h_q, 1, F, A_pad_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+  MOE_TRY(make_map(&m.qc, hT_q, 1, F, A_pad_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+  m.q = true;
+  m.c = m.in = m.a;
+  const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+  return launch<true, false, B_MN_DUAL_N, EPI_SWIGLU>(m, p, max_tiles, s);
+}
+
+// MXFP8 GEMM2 dgrad with the SwiGLU-backward epilogue whose dA = [dA1 | dA3]
+// [A_pad_max, 2K] leaves as MX codes: along the 2K columns (dA_q / dA_s,
+// for the GEMM1 dgrad) and down the rows (dAT_q / dAT_s, for the GEMM1
+// weight gradient), from the bf16-rounded dA.  dA itself is not stored.
+extern "C" moe_status_t moe_grouped_gemm_dgrad_swiglu_mxq(
+    const void* dC, const uint8_t* dC_sc, const void* B, const uint8_t* B_sc,
+    const int32_t* poff, int E, int A_pad_max, int N, int K, const void* aux, uint8_t* dA_q,
+    uint8_t* dA_s, uint8_t* dAT_q, uint8_t* dAT_s, int32_t* dev_status, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(E > 0 && E <= MAX_E, "gemm_dgrad_swiglu_mxq: E must be in [1, %d]", MAX_E);
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "gemm_dgrad_swiglu_mxq: A_pad_max %% 128");
+  MOE_CHECK_ARG(N > 0 && N % 128 == 0 && K > 0 && K % 256 == 0,
+                "gemm_dgrad_swiglu_mxq: N %% 128, K %% 256");
+  MOE_CHECK_ARG(dC && dC_sc && B && B_sc && poff && aux, "gemm_dgrad_swiglu_mxq: null pointer");
+  MOE_CHECK_ARG(dA_q && dA_s && dAT_q && dAT_s && aligned16(dA_q) && aligned16(dAT_q),
+                "gemm_dgrad_swiglu_mxq: null or unaligned MX output");
+  Params p = base_params(poff, E, dev_status);
+  p.num_kb = N / 128;
+  p.b_rows_per_e = K;
+  p.k_split = N;
+  p.n_tiles = K / BN;
+  p.a_sc = dC_sc;
+  p.a_sc_kchunks = N / 128;
+  p.b_sc = B_sc;
+  p.b_sc_kchunks = N / 128;
+  p.aux = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(aux));
+  p.ld_aux = 2LL * K;
+  p.half = K;
+  p.ldc = 2LL * K;
+  p.quant = 1;
+  p.q_sr = dA_s;
+  p.q_sc = dAT_s;
+  p.q_row_kchunks = 2 * K / 128;
+  p.q_col_kchunks = A_pad_max / 128;
+  Maps m;
+  MOE_TRY(make_map(&m.a, dC, 1, N, A_pad_max, 128, BM));
+  MOE_TRY(make_map(&m.b, B, 1, N, (uint64_t)E * K, 128, BN));
+  MOE_TRY(make_out_map(&m.in, aux, 2ULL * K, A_pad_max));
+  MOE_TRY(make_map(&m.qr, dA_q, 1, 2ULL * K, A_pad_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+  MOE_TRY(make_map(&m.qc, dAT_q, 1, 2ULL * K, A_pad_max, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
+  m.q = true;
+  m.c = m.b3 = m.c2 = m.a;
+  const int max_tiles = (A_pad_max / BM) * p.n_tiles;
+  return launch<true, false, B_K, EPI_SWIGLU_BWD>(m, p, max_tiles, s);
 }
 
 extern "C" moe_status_t moe_grouped_gemm_dgrad(int dt, const void* dC, const uint8_t* dC_sc,

@@ -73,13 +73,15 @@ size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   x.dg = l.take<float>(T * k);
   x.dl = l.take<float>(T * k);
   x.dl_rows = l.take<float>(A);
-  x.Xp = gathers(L) ? nullptr : l.take<__nv_bfloat16>(A * d);
+  // the bf16 permuted copy: only BF16 layers that do not gather need it
+  x.Xp = (L->dtype == MOE_BF16 && !gathers(L)) ? l.take<__nv_bfloat16>(A * d) : nullptr;
   x.H13 = l.take<__nv_bfloat16>(A * 2 * F);
-  x.h = l.take<__nv_bfloat16>(A * F);
+  // MXFP8: h and dA13 leave their GEMM epilogues as MX codes only
+  x.h = L->dtype == MOE_MXFP8 ? nullptr : l.take<__nv_bfloat16>(A * F);
   x.Y = l.take<__nv_bfloat16>(A * d);
   x.dXp = x.Y;   // Y is dead once the combine backward has run
-  x.dY = l.take<__nv_bfloat16>(A * d);
-  x.dA13 = l.take<__nv_bfloat16>(A * 2 * F);
+  x.dY = L->dtype == MOE_MXFP8 ? nullptr : l.take<__nv_bfloat16>(A * d);
+  x.dA13 = L->dtype == MOE_MXFP8 ? nullptr : l.take<__nv_bfloat16>(A * 2 * F);
   if (L->dtype == MOE_MXFP8) {
     x.Xp_q = l.take<uint8_t>(A * d);       x.Xp_s = l.take<uint8_t>(A * d / 32);
     x.W13_q = l.take<uint8_t>(2 * E * d * F); x.W13_s = l.take<uint8_t>(2 * E * d * F / 32);
@@ -224,12 +226,14 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
                                    stream));
     mark(S_GEMM2, true, s);
   } else {
-    const int32_t* nrows = c.poff + E;
     const size_t wq = (size_t)E * d * F;
     uint8_t* W1q = c.W13_q; uint8_t* W3q = c.W13_q + wq;
     uint8_t* W1s = c.W13_s; uint8_t* W3s = c.W13_s + wq / 32;
+    // rowwise dispatch straight into MX codes: along d (GEMM1) and down
+    // the rows (GEMM1 weight gradient); no bf16 permuted copy
     mark(S_PERMUTE, false, s);
-    MOE_TRY(moe_permute(x, c.dst, c.offsets, c.poff, T, k, d, E, A, c.Xp, c.Xp_q, c.Xp_s, stream));
+    MOE_TRY(moe_permute_mx(x, c.src, c.poff, T, d, E, A, c.Xp_q, c.Xp_s, c.XpT_q, c.XpT_s,
+                           stream));
     mark(S_PERMUTE, true, s);
     // every weight along both K axes it is used with, in one pass each:
     // W1/W3 [E*d, F] down d (fwd GEMM1) and along F (GEMM1 dgrad); W2
@@ -240,14 +244,13 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
                              W3s, stream));
     MOE_TRY(mx_quantize_dual(w->W2, E * F, d, nullptr, c.W2t_q, c.W2t_s, c.W2_q, c.W2_s, stream));
     mark(S_QW, true, s);
+    // GEMM1 + SwiGLU; its epilogue quantises h along F (fwd GEMM2) and down
+    // the rows (GEMM2 wgrad) in place of storing it
     mark(S_GEMM1, false, s);
-    MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.Xp_q, c.Xp_s, W1q, W1s, W3q, W3s, c.poff, E, A, F, d,
-                                 MOE_EPI_SWIGLU, c.h, c.H13, dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_fwd_swiglu_mxq(c.Xp_q, c.Xp_s, W1q, W1s, W3q, W3s, c.poff, E, A, F,
+                                            d, c.H13, c.h_q, c.h_s, c.hT_q, c.hT_s, dev_status,
+                                            stream));
     mark(S_GEMM1, true, s);
-    // h along F (fwd GEMM2) and down its rows (GEMM2 wgrad)
-    mark(S_QH, false, s);
-    MOE_TRY(mx_quantize_dual(c.h, A, F, nrows, c.h_q, c.h_s, c.hT_q, c.hT_s, stream));
-    mark(S_QH, true, s);
     mark(S_GEMM2, false, s);
     MOE_TRY(moe_grouped_gemm_fwd(MOE_MXFP8, c.h_q, c.h_s, c.W2_q, c.W2_s, nullptr, nullptr, c.poff,
                                  E, A, d, F, MOE_EPI_NONE, c.Y, nullptr, dev_status, stream));
@@ -275,9 +278,11 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   // W_r^T [E, d] (fp32) in the workspace: the GEMM1 dgrad epilogue adds
   // dl_rows[r] * W_r[:, e] to each row r of expert e
   float* wrT = router ? static_cast<float*>(c.ws) : nullptr;
+  // dg, dl, dl_rows (and in BF16 the gate-scaled rows dY)
   mark(S_COMBINE_BWD, false, s);
-  MOE_TRY(moe_combine_bwd(dout, c.Y, c.gates, c.dst, c.offsets, c.poff, T, k, d, E, c.dY, c.dg,
-                          router ? c.dl : nullptr, router ? c.dl_rows : nullptr, stream));
+  MOE_TRY(moe_combine_bwd(dout, c.Y, c.gates, c.dst, c.offsets, c.poff, T, k, d, E,
+                          mx ? nullptr : c.dY, c.dg, router ? c.dl : nullptr,
+                          router ? c.dl_rows : nullptr, stream));
   mark(S_COMBINE_BWD, true, s);
   if (!mx) {
     mark(S_DGRAD2, false, s);
@@ -310,26 +315,25 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                       c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));
     mark(S_WGRAD1, true, s);
   } else {
-    const int32_t* nrows = c.poff + E;
     const size_t wq = (size_t)E * d * F;
     // (weights were quantised along both axes in the forward)
-    // dY along d (GEMM2 dgrad) and down its rows (GEMM2 wgrad)
+    // the gate-scaled rows dY straight into MX codes, along d (GEMM2 dgrad)
+    // and down the rows (GEMM2 wgrad)
     mark(S_QD2, false, s);
-    MOE_TRY(mx_quantize_dual(c.dY, A, d, nrows, c.dY_q, c.dY_s, c.dYT_q, c.dYT_s, stream));
+    MOE_TRY(moe_combine_bwd_mx(dout, c.gates, c.topk_idx, c.src, c.poff, T, k, d, E, A, c.dY_q,
+                               c.dY_s, c.dYT_q, c.dYT_s, stream));
     mark(S_QD2, true, s);
+    // GEMM2 dgrad + SwiGLU backward; its epilogue quantises dA13 along 2F
+    // (GEMM1 dgrad) and down the rows (GEMM1 wgrad) in place of storing it
     mark(S_DGRAD2, false, s);
-    MOE_TRY(moe_grouped_gemm_dgrad(MOE_MXFP8, c.dY_q, c.dY_s, c.W2t_q, c.W2t_s, nullptr, nullptr,
-                                   c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
-                                   dev_status, stream));
+    MOE_TRY(moe_grouped_gemm_dgrad_swiglu_mxq(c.dY_q, c.dY_s, c.W2t_q, c.W2t_s, c.poff, E, A, d, F,
+                                              c.H13, c.dA_q, c.dA_s, c.dAT_q, c.dAT_s, dev_status,
+                                              stream));
     mark(S_DGRAD2, true, s);
     mark(S_WGRAD2, false, s);
     MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff,
                                     c.offsets, E, A, F, d, G->dW2, nullptr, dev_status, s));
     mark(S_WGRAD2, true, s);
-    // dA13 along 2F (GEMM1 dgrad) and down its rows (GEMM1 wgrad)
-    mark(S_QD1, false, s);
-    MOE_TRY(mx_quantize_dual(c.dA13, A, 2 * F, nrows, c.dA_q, c.dA_s, c.dAT_q, c.dAT_s, stream));
-    mark(S_QD1, true, s);
     mark(S_DGRAD1, false, s);
     if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
     MOE_TRY(moe::grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, c.W13t_q, c.W13t_s, c.W13t_q + wq,
@@ -337,10 +341,6 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                c.dXp, router ? c.dl_rows : nullptr, router ? wrT : nullptr,
                                dev_status, s));
     mark(S_DGRAD1, true, s);
-    // Xp down its rows (GEMM1 wgrad)
-    mark(S_QW1, false, s);
-    MOE_TRY(mx_quantize(c.Xp, A, d, 1, c.poff, E, nrows, c.XpT_q, c.XpT_s, stream));
-    mark(S_QW1, true, s);
     mark(S_WGRAD1, false, s);
     MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff,
                                     c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));

@@ -1,0 +1,101 @@
+// MX (MXFP8) element rule shared by the quantisers and the fused GEMM
+// epilogues: E4M3 codes with one E8M0 scale per 32 elements along K.
+//
+// Olmo-core 3 オープン混合エキスパート学習インフラストラクチャ, section
+// "MXFP8による精度最適化": MXFP8 for the expert feed-forward compute.  Rule
+// (OCP MX): X = 2^(floor(log2 amax) - 8), code = RNE-saturating E4M3 of v/X,
+// an all-zero block gets scale byte 0.  For a bf16 (or bf16-valued fp32)
+// block maximum, floor(log2 amax) is the exponent field of amax minus 127,
+// so the scale byte is max(expfield(amax) - 8, 0), and 1/X is the fp32
+// number with exponent field 254 - byte (exact power-of-two scaling).
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// byte offset of the scale of (MN index mn, K block kb) in the tensor-core
+// layout: 512-byte blocks of 128 MN indices x 4 K blocks
+__device__ __forceinline__ size_t mx_sf_offset(int mn, int kb, int kchunks) {
+  return ((size_t)(mn >> 7) * kchunks + (kb >> 2)) * 512 + (mn & 31) * 16 + ((mn >> 5) & 3) * 4 +
+         (kb & 3);
+}
+
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+  const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
+  return ef > 8 ? (uint32_t)(ef - 8) : 0u;
+}
+
+__device__ __forceinline__ float mx_inv_scale(uint32_t byte) {
+  return __uint_as_float((254u - byte) << 23);
+}
+
+// two values -> two E4M3 codes (low byte first)
+__device__ __forceinline__ uint32_t mx_encode2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// 8 values -> 8 E4M3 codes (memory order)
+__device__ __forceinline__ uint2 mx_encode8(const float* f, float inv) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = mx_encode2(f[2 * i] * inv, f[2 * i + 1] * inv);
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// A warp's 32 x 32 block of bf16-valued numbers (lane = row, v[j] = column
+// j) quantised both ways: cr = the lane's row codes (blocks of 32 along the
+// row), cc = its codes under the column scales (blocks of 32 rows down each
+// column), 4 codes per word in column order; br = the row's scale byte,
+// bc = the scale byte of column `lane`.
+__device__ __forceinline__ void mx_quant_block32_regs(const float* v, uint32_t* cr, uint32_t* cc,
+                                                      uint32_t& br, uint32_t& bc) {
+  const int lane = threadIdx.x & 31;
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  br = mx_scale_byte(amax);
+  const float inv = mx_inv_scale(br);
+  bc = 0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // column maximum over the warp's 32 rows (non-negative floats order
+      // like their bit patterns)
+      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + i])));
+      b[i] = mx_scale_byte(__uint_as_float(m));
+      if (lane == j + i) bc = b[i];
+    }
+    cr[j / 4] = mx_encode2(v[j] * inv, v[j + 1] * inv) |
+                (mx_encode2(v[j + 2] * inv, v[j + 3] * inv) << 16);
+    cc[j / 4] = mx_encode2(v[j] * mx_inv_scale(b[0]), v[j + 1] * mx_inv_scale(b[1])) |
+                (mx_encode2(v[j + 2] * mx_inv_scale(b[2]), v[j + 3] * mx_inv_scale(b[3])) << 16);
+  }
+}
+
+// mx_quant_block32_regs with the codes written to two [32 rows x 32 bytes]
+// shared-memory boxes (row r at r * 32; box_r: row codes, box_c: column
+// codes) and the scale bytes to global memory: the row scale of (row,
+// col0/32) with K = the row length (row_kchunks = K / 128), the column
+// scale of (col0 + lane, row0/32) with K = the padded row count
+// (col_kchunks = A_pad_max / 128).
+__device__ __forceinline__ void mx_quant_block32(const float* v, uint8_t* box_r, uint8_t* box_c,
+                                                 uint8_t* scales_r, int row, int col0,
+                                                 int row_kchunks, uint8_t* scales_c, int row0,
+                                                 int col_kchunks) {
+  const int lane = threadIdx.x & 31;
+  uint32_t cr[8], cc[8], br, bc;
+  mx_quant_block32_regs(v, cr, cc, br, bc);
+  *reinterpret_cast<uint4*>(box_r + lane * 32) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+  *reinterpret_cast<uint4*>(box_r + lane * 32 + 16) = make_uint4(cr[4], cr[5], cr[6], cr[7]);
+  *reinterpret_cast<uint4*>(box_c + lane * 32) = make_uint4(cc[0], cc[1], cc[2], cc[3]);
+  *reinterpret_cast<uint4*>(box_c + lane * 32 + 16) = make_uint4(cc[4], cc[5], cc[6], cc[7]);
+  scales_r[mx_sf_offset(row, col0 >> 5, row_kchunks)] = (uint8_t)br;
+  scales_c[mx_sf_offset(col0 + lane, row0 >> 5, col_kchunks)] = (uint8_t)bc;
+}
+
+}  // namespace moe

@@ -13,35 +13,17 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "mx.cuh"
 #include "sm100.cuh"
 
 namespace moe {
 
 __device__ __forceinline__ size_t sf_offset(int mn, int kb, int kchunks) {
-  return ((size_t)(mn >> 7) * kchunks + (kb >> 2)) * 512 + (mn & 31) * 16 + ((mn >> 5) & 3) * 4 +
-         (kb & 3);
+  return mx_sf_offset(mn, kb, kchunks);
 }
-
-__device__ __forceinline__ uint32_t scale_byte(float amax) {
-  const int ef = (__float_as_uint(amax) >> 23) & 0xFF;
-  return ef > 8 ? (uint32_t)(ef - 8) : 0u;
-}
-
-__device__ __forceinline__ float inv_scale(uint32_t byte) {
-  return __uint_as_float((254u - byte) << 23);
-}
-
-// 8 values -> 8 E4M3 codes (memory order)
-__device__ __forceinline__ uint2 encode8(const float* f, float inv) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
-        make_float2(f[2 * i] * inv, f[2 * i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-    w[i] = (uint32_t)c;
-  }
-  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-}
+__device__ __forceinline__ uint32_t scale_byte(float amax) { return mx_scale_byte(amax); }
+__device__ __forceinline__ float inv_scale(uint32_t byte) { return mx_inv_scale(byte); }
+__device__ __forceinline__ uint2 encode8(const float* f, float inv) { return mx_encode8(f, inv); }
 
 // ------------------------------------------- blocks along rows (axis 0)
 // one warp per 256-column segment of one row; 4 lanes per 32-element block
@@ -314,9 +296,121 @@ permute_mx_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
   }
 }
 
+
+// ----------------------- dispatch straight into MX codes, both K axes
+// The expert-contiguous buffer in blocks of 32 rows (a block never crosses
+// a group: groups start on multiples of 128): row r is token src[r], or a
+// zero row for src[r] < 0.  A CTA takes one 32-row block and 256 columns,
+// warp w columns 32w..32w+31, lane = row: the lane loads its 32 values of
+// its token's row, and the warp quantises the 32 x 32 block along the rows
+// (Xq / Xs, K = d: GEMM1) and down the columns (XqT / XsT, K = the padded
+// rows: GEMM1 weight gradient).  The bf16 permuted copy is never written.
+// Rows from poff[E] on are not touched (no GEMM reads them).
+// With a gate (the backward's dY rows): row r of group e is g * x[t] with
+// g = gates[t, j] for the slot j of expert e in topk[t, :], rounded to bf16
+// as the combine backward rounds it.
+constexpr int kGatherWarps = 8;
+
+struct GateRows {
+  const float* gates;     // [T, k], null: no gate
+  const int32_t* topk;    // [T, k]
+  const int32_t* poff;    // [E + 1]
+  int k, E;
+};
+
+__global__ void __launch_bounds__(32 * kGatherWarps)
+permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ src,
+                         const int32_t* __restrict__ poff_end, int d, int A_pad_max,
+                         uint8_t* __restrict__ Xq, uint8_t* __restrict__ Xs,
+                         uint8_t* __restrict__ XqT, uint8_t* __restrict__ XsT, GateRows gr) {
+  const int nrows = min(*poff_end, A_pad_max);
+  const int segs = d / 256;
+  const int nblk = (nrows / 32) * segs;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
+    const int rb = b / segs, seg = b - rb * segs;
+    const int r0 = rb * 32, r = r0 + lane;
+    const int c0 = seg * 256 + warp * 32;
+    const int t = src[r];
+    float v[32];
+    if (t >= 0) {
+      const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)t * d + c0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) unpack8(__ldg(p + j), v + 8 * j);
+      if (gr.gates) {
+        // the block's group (largest e with poff[e] <= r0), then this
+        // token's slot of that expert
+        int lo = 0, hi = gr.E - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (__ldg(gr.poff + mid) <= r0) lo = mid; else hi = mid - 1;
+        }
+        float g = 0.f;
+        for (int j = 0; j < gr.k; ++j)
+          if (__ldg(gr.topk + (size_t)t * gr.k + j) == lo) g = __ldg(gr.gates + (size_t)t * gr.k + j);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(g * v[j]));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    }
+    uint32_t cr[8], cc[8], br, bc;
+    mx_quant_block32_regs(v, cr, cc, br, bc);
+    uint4* qr = reinterpret_cast<uint4*>(Xq + (size_t)r * d + c0);
+    uint4* qc = reinterpret_cast<uint4*>(XqT + (size_t)r * d + c0);
+    qr[0] = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+    qr[1] = make_uint4(cr[4], cr[5], cr[6], cr[7]);
+    qc[0] = make_uint4(cc[0], cc[1], cc[2], cc[3]);
+    qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
+    Xs[mx_sf_offset(r, c0 >> 5, d / 128)] = (uint8_t)br;
+    XsT[mx_sf_offset(c0 + lane, r0 >> 5, A_pad_max / 128)] = (uint8_t)bc;
+  }
+}
+
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" moe_status_t moe_permute_mx(const void* x, const int32_t* src, const int32_t* poff,
+                                       int T, int d, int E, int A_pad_max, uint8_t* Xq,
+                                       uint8_t* Xs, uint8_t* XqT, uint8_t* XsT,
+                                       moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && E > 0 && d > 0 && d % 256 == 0, "moe_permute_mx: d %% 256");
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "moe_permute_mx: A_pad_max %% 128");
+  MOE_CHECK_ARG(x && src && poff && Xq && Xs && XqT && XsT, "moe_permute_mx: null pointer");
+  MOE_CHECK_ARG(aligned16(x) && aligned16(Xq) && aligned16(XqT), "moe_permute_mx: unaligned buffer");
+  const long long blocks = (long long)(A_pad_max / 32) * (d / 256);
+  const int grid = (int)std::min<long long>(blocks, 8LL * num_sms());
+  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(x), src, poff + E, d, A_pad_max, Xq, Xs, XqT, XsT,
+      GateRows{nullptr, nullptr, nullptr, 0, E});
+  MOE_CHECK_LAUNCH("moe_permute_mx");
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
+                                           const int32_t* topk_idx, const int32_t* src,
+                                           const int32_t* poff, int T, int k, int d, int E,
+                                           int A_pad_max, uint8_t* dYq, uint8_t* dYs,
+                                           uint8_t* dYTq, uint8_t* dYTs, moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CHECK_ARG(T > 0 && E > 0 && k > 0 && k <= 16 && d > 0 && d % 256 == 0,
+                "moe_combine_bwd_mx: d %% 256, 0 < k <= 16");
+  MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "moe_combine_bwd_mx: A_pad_max %% 128");
+  MOE_CHECK_ARG(dout && gates && topk_idx && src && poff && dYq && dYs && dYTq && dYTs,
+                "moe_combine_bwd_mx: null pointer");
+  MOE_CHECK_ARG(aligned16(dout) && aligned16(dYq) && aligned16(dYTq),
+                "moe_combine_bwd_mx: unaligned buffer");
+  const long long blocks = (long long)(A_pad_max / 32) * (d / 256);
+  const int grid = (int)std::min<long long>(blocks, 8LL * num_sms());
+  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(dout), src, poff + E, d, A_pad_max, dYq, dYs, dYTq, dYTs,
+      GateRows{gates, topk_idx, poff, k, E});
+  MOE_CHECK_LAUNCH("moe_combine_bwd_mx");
+  return MOE_OK;
+}
 
 moe_status_t moe_permute_mx_launch(const void* x, const int32_t* dst, const int32_t* offsets,
                                    const int32_t* poff, int T, int k, int d, int E, int A_pad_max,

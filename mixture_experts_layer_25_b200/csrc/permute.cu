@@ -33,8 +33,10 @@ __device__ __forceinline__ void zero_pad_rows(const int32_t* offsets, const int3
   const int r1 = poff[e + 1];
   const size_t n = (size_t)(r1 - r0) * d8;
   const uint4 z = make_uint4(0, 0, 0, 0);
-  uint4* base = buf + (size_t)r0 * d8;
-  for (size_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = z;
+  if (buf) {
+    uint4* base = buf + (size_t)r0 * d8;
+    for (size_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = z;
+  }
   if (row_vec)
     for (int r = r0 + (int)threadIdx.x; r < r1; r += blockDim.x) row_vec[r] = 0.f;
 }
@@ -283,7 +285,7 @@ combine_bwd_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ Y,
           sc[i] = g[j] * fd[i];
         }
         dot[j] += sdot;
-        dY[(size_t)r[j] * d8 + c] = pack8(sc);
+        if (dY) dY[(size_t)r[j] * d8 + c] = pack8(sc);
       }
     }
   }
@@ -393,7 +395,7 @@ combine_bwd_pf_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ 
           sc[i] = g[j] * fd[i];
         }
         dot[j] += sdot;
-        dY[(size_t)r[j] * d8 + lt] = pack8(sc);
+        if (dY) dY[(size_t)r[j] * d8 + lt] = pack8(sc);
       }
     }
 #pragma unroll
@@ -630,9 +632,10 @@ extern "C" moe_status_t moe_combine_bwd(const void* dout, const void* Y, const f
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   MOE_CHECK_ARG(T > 0 && k > 0 && k <= kTopKLimit && E > 0 && d > 0 && d % 8 == 0,
                 "moe_combine_bwd: bad sizes");
-  MOE_CHECK_ARG(dout && Y && gates && dst && offsets && poff && dY && dg,
+  MOE_CHECK_ARG(dout && Y && gates && dst && offsets && poff && dg,
                 "moe_combine_bwd: null pointer");
-  MOE_CHECK_ARG(aligned16(dout) && aligned16(Y) && aligned16(dY), "moe_combine_bwd: unaligned");
+  MOE_CHECK_ARG(aligned16(dout) && aligned16(Y) && (!dY || aligned16(dY)),
+                "moe_combine_bwd: unaligned");
   const int tpb = kBlock / team_threads(d / 8);
   const int tok_blocks = (T + tpb - 1) / tpb;
   if (d / 8 <= kBlock && k <= 4) {

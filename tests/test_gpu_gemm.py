@@ -7,7 +7,7 @@ import torch
 
 import moe_inputs
 import oracle
-from gpu_util import f64, rel_err
+from gpu_util import f64, rel_err, scales_to_plain
 
 pytestmark = pytest.mark.gpu
 moe = pytest.importorskip("mixture_experts_layer_25_b200")
@@ -370,3 +370,57 @@ def test_wgrad_gather_equals_wgrad_on_permuted_rows(T, E, k):
     empty = np.nonzero(ref["counts"] == 0)[0]
     for e in empty:
         assert torch.all(g1[e] == 0) and torch.all(g3[e] == 0)
+
+
+def _same_codes(q_fused, q_ref, R, C, axis, P):
+    """Fused-epilogue MX codes and scales equal the quantiser's on rows < P."""
+    (cf, sf), (cr, sr) = q_fused, q_ref
+    assert torch.equal(cf[:P], cr[:P])
+    pf, pr = scales_to_plain(sf, R, C, axis), scales_to_plain(sr, R, C, axis)
+    rows = P if axis == 0 else P // 32
+    np.testing.assert_array_equal(pf[:rows], pr[:rows])
+
+
+def test_fwd_swiglu_mxq_equals_quantised_h():
+    """GEMM1 + SwiGLU in MXFP8 with h quantised in the epilogue: codes and
+    scales along F and down the rows are bit-identical to mx_quantize_dual
+    of the h the plain MX call stores, and [H1 | H3] is the same."""
+    E, K, F = len(COUNTS), 256, 256
+    poff, A, real = _groups(COUNTS)
+    X = _act(A, K, real, 50)
+    W1, W3 = _w(E, K, F, 51), _w(E, K, F, 52)
+    tp = torch.from_numpy(poff).cuda()
+    P = int(poff[-1])
+    Xq, Xs = moe.mx_quantize(X, 0)
+    W1q, W1s = moe.mx_quantize(W1.view(E * K, F), 1)
+    W3q, W3s = moe.mx_quantize(W3.view(E * K, F), 1)
+    h, aux = moe.moe_grouped_gemm_fwd(Xq, W1q.view(E, K, F), tp, E, epilogue=moe.MOE_EPI_SWIGLU,
+                                      B3=W3q.view(E, K, F), A_sc=Xs, B_sc=W1s, B3_sc=W3s)
+    aux2, qrow, qcol = moe.moe_grouped_gemm_fwd_swiglu_mxq(Xq, Xs, W1q.view(E, K, F), W1s,
+                                                           W3q.view(E, K, F), W3s, tp, E)
+    ref_row, ref_col = moe.mx_quantize_dual(h)
+    torch.cuda.synchronize()
+    assert torch.equal(aux2[:P], aux[:P])
+    _same_codes(qrow, ref_row, A, F, 0, P)
+    _same_codes(qcol, ref_col, A, F, 1, P)
+
+
+def test_dgrad_swiglu_mxq_equals_quantised_dA():
+    """GEMM2 dgrad + SwiGLU backward in MXFP8 with dA quantised in the
+    epilogue: bit-identical to mx_quantize_dual of the stored dA."""
+    E, F, d = len(COUNTS), 256, 512
+    poff, A, real = _groups(COUNTS)
+    dY = _act(A, d, real, 53)
+    W2 = _w(E, F, d, 54)
+    H13 = _act(A, 2 * F, real, 55, scale=2.0)
+    P = int(poff[-1])
+    tp = torch.from_numpy(poff).cuda()
+    dYq, dYs = moe.mx_quantize(dY, 0)
+    Wq, Ws = moe.mx_quantize(W2.view(E * F, d), 0)
+    dA = moe.moe_grouped_gemm_dgrad(dYq, Wq.view(E, F, d), tp, E, epilogue=moe.MOE_EPI_SWIGLU_BWD,
+                                    aux=H13, dC_sc=dYs, B_sc=Ws)
+    qrow, qcol = moe.moe_grouped_gemm_dgrad_swiglu_mxq(dYq, dYs, Wq.view(E, F, d), Ws, H13, tp, E)
+    ref_row, ref_col = moe.mx_quantize_dual(dA)
+    torch.cuda.synchronize()
+    _same_codes(qrow, ref_row, A, 2 * F, 0, P)
+    _same_codes(qcol, ref_col, A, 2 * F, 1, P)

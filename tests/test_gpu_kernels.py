@@ -144,6 +144,55 @@ def test_permute_fused_mx_codes():
     np.testing.assert_array_equal(scales_to_plain(Xs, A, d, 0)[:P], s)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(700, 512, 16, 4), (1, 256, 8, 2), (64, 6144, 384, 8),
+                                     (3000, 2048, 128, 4)])
+def test_permute_mx_codes_both_axes(T, d, E, k):
+    """Dispatch straight into MX codes: along d and down the rows, bit-exact
+    against the oracle's quantisers applied to the oracle's permuted rows."""
+    idx, gates, meta = _meta_for(T, E, k, 6 + T)
+    x = moe_inputs.random_bf16((T, d), 9 + T, device="cuda")
+    x[0, :64] = 0                                   # zero blocks
+    (q, qs), (qT, qTs) = moe.moe_permute_mx(x, meta, E)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    P = int(ref["poff"][E])
+    A = meta["A_pad_max"]
+    Xp64 = oracle.permute_rows(f64(x), ref)
+    c0, s0 = oracle.mx_quantize_rows(Xp64)
+    c1, s1 = oracle.mx_quantize_cols_grouped(Xp64, ref["poff"])
+    np.testing.assert_array_equal(q[:P].cpu().numpy(), c0)
+    np.testing.assert_array_equal(scales_to_plain(qs, A, d, 0)[:P], s0)
+    np.testing.assert_array_equal(qT[:P].cpu().numpy(), c1)
+    np.testing.assert_array_equal(scales_to_plain(qTs, A, d, 1)[:P // 32], s1)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(700, 512, 16, 4), (1, 256, 8, 2), (64, 6144, 384, 8)])
+def test_combine_bwd_mx_codes_both_axes(T, d, E, k):
+    """The backward's gate-scaled rows straight into MX codes: bit-exact
+    against the oracle's quantisers of the bf16-rounded dY rows."""
+    idx, gates, meta = _meta_for(T, E, k, 16 + T)
+    dout = moe_inputs.random_bf16((T, d), 19 + T, device="cuda")
+    (q, qs), (qT, qTs) = moe.moe_combine_bwd_mx(dout, meta["gates"], meta, E)
+    torch.cuda.synchronize()
+    ref = oracle.routing_metadata(idx, E, 128)
+    P = int(ref["poff"][E])
+    A = meta["A_pad_max"]
+    # dY as the kernel forms it, g * dout in fp32 then rounded to bf16: the
+    # codes are integer decisions taken in the kernel's precision
+    g32 = meta["gates"].cpu().numpy().astype(np.float32)
+    d32 = f64(dout).astype(np.float32)
+    dY = np.zeros((P, d))
+    for j in range(k):
+        prod = torch.from_numpy(g32[:, j:j + 1] * d32).to(torch.bfloat16).to(torch.float64)
+        dY[ref["dst"][:, j]] = prod.numpy()
+    c0, s0 = oracle.mx_quantize_rows(dY)
+    c1, s1 = oracle.mx_quantize_cols_grouped(dY, ref["poff"])
+    np.testing.assert_array_equal(q[:P].cpu().numpy(), c0)
+    np.testing.assert_array_equal(scales_to_plain(qs, A, d, 0)[:P], s0)
+    np.testing.assert_array_equal(qT[:P].cpu().numpy(), c1)
+    np.testing.assert_array_equal(scales_to_plain(qTs, A, d, 1)[:P // 32], s1)
+
+
 @pytest.mark.parametrize("R,C,axis", [(256, 512, 0), (512, 384, 1), (128, 128, 0), (384, 2048, 1)])
 def test_mx_quantize_bit_exact(R, C, axis):
     g = torch.Generator(device="cuda"); g.manual_seed(R + C + axis)
