@@ -279,7 +279,7 @@ MOE_API moe_status_t moe_grouped_gemm_wgrad(int dt, const void* A, const uint8_t
  * GEMM1 operand) and down the rows in blocks of 32 inside each group (XqT
  * [A_pad_max, d], XsT: K = A_pad_max; the GEMM1 weight-gradient operand),
  * bit-identical to mx_quantize_dual of the bf16 permuted buffer.  No bf16
- * copy is written; rows from poff[E] on are not touched.  d % 256 == 0,
+ * copy is written; rows from poff[E] on are not touched.  d % 128 == 0,
  * A_pad_max % 128 == 0, x / Xq / XqT 16-byte aligned. */
 MOE_API moe_status_t moe_permute_mx(const void* x, const int32_t* src, const int32_t* poff,
                                     int T, int d, int E, int A_pad_max, uint8_t* Xq,
@@ -292,7 +292,7 @@ MOE_API moe_status_t moe_permute_mx(const void* x, const int32_t* src, const int
  * e (a zero row for src[r] < 0), written only as MX codes along d (dYq /
  * dYs, K = d: GEMM2 dgrad) and down the rows (dYTq / dYTs, K = A_pad_max:
  * GEMM2 weight gradient); bit-identical to mx_quantize_dual of the dY that
- * moe_combine_bwd writes.  Rows from poff[E] on are not touched.  d % 256
+ * moe_combine_bwd writes.  Rows from poff[E] on are not touched.  d % 128
  * == 0, k <= 16. */
 MOE_API moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
                                         const int32_t* topk_idx, const int32_t* src,

@@ -55,7 +55,10 @@ constexpr int SFB_BYTES = 1024;     // 256 rows x 4 scale bytes
 constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
-enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3 };
+enum Epi { EPI_STORE = 0, EPI_SWIGLU = 1, EPI_SWIGLU_BWD = 2, EPI_ROUTER = 3, EPI_ROUTER4 = 4 };
+// the router epilogue keeps a running top-k of 8 slots (EPI_ROUTER, k <= 8)
+// or 4 slots (EPI_ROUTER4, k <= 4)
+__host__ __device__ constexpr bool is_router(int epi) { return epi == EPI_ROUTER || epi == EPI_ROUTER4; }
 
 // pipeline depth and per-warp staging (boxes of 2 KB) for each epilogue,
 // within the 227 KB of shared memory per CTA: STORE uses one box per warp
@@ -76,11 +79,11 @@ template <bool MX, int EPI, bool WGRAD = false> struct EpiCfg {
   static constexpr int STAGES = EPI == EPI_STORE ? (STORE_BOXES == 1 ? 4 : 3)
                               : EPI == EPI_SWIGLU ? SWIGLU_STAGES : 3;
   static constexpr int BOXES = EPI == EPI_STORE ? STORE_BOXES
-                             : EPI == EPI_ROUTER ? 1
+                             : is_router(EPI) ? 1
                              : EPI == EPI_SWIGLU ? (SWIGLU_STAGES == 4 ? 1 : 3) : 4;
   static constexpr int STG = BOXES * BOX_BYTES;
   // the router stage holds three B tiles (one per weight split) of <= 128 columns
-  static constexpr int B_STAGE = EPI == EPI_ROUTER ? 3 * 128 * 128 : B_BYTES;
+  static constexpr int B_STAGE = is_router(EPI) ? 3 * 128 * 128 : B_BYTES;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_STAGE +
                                  (MX ? SFA_BYTES + SFB_BYTES : 0)) + NUM_EPI_WARPS * STG;
 };
@@ -378,11 +381,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           // the router's tiles all read the same split weights: each tile
           // starts at its own K block so that they do not stream the same
           // lines at the same time (fp32 sums in a rotated, fixed order)
-          const int kb = EPI == EPI_ROUTER ? (step + tile) % nkb : step;
+          const int kb = is_router(EPI) ? (step + tile) % nkb : step;
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs)) break;
           uint64_t* fb = &full_bar[stage];
           const int nbox = p.b_boxes ? p.b_boxes : BN / MN_CHUNK;
-          if constexpr (EPI == EPI_ROUTER)
+          if constexpr (is_router(EPI))
             mbar_arrive_expect_tx(fb, A_BYTES + 3 * nbox * MN_CHUNK_BYTES);
           else
             mbar_arrive_expect_tx(fb, B_MNMAJOR ? STAGE_TX - (BN / MN_CHUNK - nbox) * MN_CHUNK_BYTES
@@ -402,7 +405,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           // B operand
           const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
-          if constexpr (EPI == EPI_ROUTER) {
+          if constexpr (is_router(EPI)) {
             // rows kb*BK.. of each weight split (split s starts at row s * d)
             for (int sp = 0; sp < 3; ++sp)
               for (int i = 0; i < nbox; ++i)
@@ -517,7 +520,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tmem_cp_32x128b_warpx4(sfb_t, smem_desc(sf + SFA_BYTES, 0, 128, 0));
             tmem_cp_32x128b_warpx4(sfb_t + 4, smem_desc(sf + SFA_BYTES + 512, 0, 128, 0));
           }
-          if constexpr (EPI == EPI_ROUTER) {
+          if constexpr (is_router(EPI)) {
 #pragma unroll
             for (int ks = 0; ks < KSTEPS; ++ks) {
               const uint64_t ad = smem_desc(sa + ks * 32, 16, 1024, 2);
@@ -599,7 +602,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       // epilogue keeps no other large state; otherwise each 32-column chunk
       // is read from TMEM when it is stored and the accumulator is released
       // at the end of the tile (BF16 double-buffers its accumulators).
-      constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU);
+#ifndef MOE_MX_BWD_EARLY
+#define MOE_MX_BWD_EARLY 1
+#endif
+      constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU ||
+                                    (EPI == EPI_SWIGLU_BWD && MOE_MX_BWD_EARLY));
       constexpr int NV = EARLY ? 128 : 32;
       uint32_t av[NV];
       if constexpr (EARLY) {
@@ -783,7 +790,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {  // accumulator = dh, columns [nt*256, +256)
         const int n0 = t.nt * BN + hc * (BN / 2);
         constexpr int NCH = BN / 2 / CHUNK;
-#pragma unroll 1
+#pragma unroll(EARLY ? NCH : 1)
         for (int ci = 0; ci < NCH; ++ci) {
           const int c = ci * CHUNK;
           const int pr = ci & 1;                      // staging pair of this chunk
@@ -797,9 +804,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[ew][pr ^ 1], p.half + n0 + c + CHUNK, y0);
             in_pending |= 1u << (pr ^ 1);
           }
-          uint32_t* v = av;
-          tmem_ld32(tbase + hc * (BN / 2) + c, v);
-          tmem_wait_ld();
+          uint32_t* v = av + (EARLY ? 32 * ci : 0);
+          if constexpr (!EARLY) {
+            tmem_ld32(tbase + hc * (BN / 2) + c, v);
+            tmem_wait_ld();
+          }
           int got = 1;
           if (lane == 0)
             got = mbar_wait(&in_bar[ew][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
@@ -870,13 +879,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
         if (!ok) break;
-      } else {  // EPI_ROUTER: accumulator = fp32 logits, 128 tokens x E experts
+      } else {  // router: accumulator = fp32 logits, 128 tokens x E experts
         // Both column halves of the epilogue warps scan half of the experts
         // each for the running top-k of their token; the second half's list
         // is merged into the first through shared memory.  Ranks inside the
         // tile: each of four warps counts 32 tokens in order, then a prefix
         // over the four warps' counts (same result as one pass in token order).
-        constexpr int KT = 8;                                   // k <= 8
+        constexpr int KT = EPI == EPI_ROUTER4 ? 4 : 8;          // k <= KT
         int* sel_s = reinterpret_cast<int*>(sStg);              // [128][k] chosen experts
         float* mv_s = reinterpret_cast<float*>(sel_s + BM * KT);  // [128][k] second half's list
         int* me_s = reinterpret_cast<int*>(mv_s + BM * KT);
@@ -1144,7 +1153,8 @@ moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int
   MOE_TRY(make_map(&m.a, x, 2, d, T, 64, BM));
   MOE_TRY(make_map(&m.b, wsplit, 2, E, 3ULL * d, 64, 64));
   m.b3 = m.c = m.c2 = m.in = m.a;
-  return launch<false, false, B_MN, EPI_ROUTER>(m, p, (T + BM - 1) / BM, s);
+  return k <= 4 ? launch<false, false, B_MN, EPI_ROUTER4>(m, p, (T + BM - 1) / BM, s)
+                : launch<false, false, B_MN, EPI_ROUTER>(m, p, (T + BM - 1) / BM, s);
 }
 }  // namespace moe
 

@@ -298,18 +298,24 @@ permute_mx_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ dst,
 
 
 // ----------------------- dispatch straight into MX codes, both K axes
-// The expert-contiguous buffer in blocks of 32 rows (a block never crosses
-// a group: groups start on multiples of 128): row r is token src[r], or a
-// zero row for src[r] < 0.  A CTA takes one 32-row block and 256 columns,
-// warp w columns 32w..32w+31, lane = row: the lane loads its 32 values of
-// its token's row, and the warp quantises the 32 x 32 block along the rows
-// (Xq / Xs, K = d: GEMM1) and down the columns (XqT / XsT, K = the padded
-// rows: GEMM1 weight gradient).  The bf16 permuted copy is never written.
-// Rows from poff[E] on are not touched (no GEMM reads them).
+// Items of 128 rows x 128 columns of the expert-contiguous buffer (a
+// 128-row tile never crosses a group: groups start on multiples of 128):
+// row r is token src[r], or a zero row for src[r] < 0.  The item's rows are
+// gathered into shared memory by coalesced 16-byte cp.async copies (two
+// buffers: the next item loads while this one is quantised); each warp then
+// quantises two of the item's sixteen 32 x 32 blocks (lane = row) along the
+// rows (Xq / Xs, K = d: GEMM1) and down the columns (XqT / XsT, K = the
+// padded rows: GEMM1 weight gradient), and the item's scale bytes leave as
+// whole 32-bit words of the tensor-core layout.  The bf16 permuted copy is
+// never written; rows from poff[E] on are not touched (no GEMM reads them).
+//
 // With a gate (the backward's dY rows): row r of group e is g * x[t] with
 // g = gates[t, j] for the slot j of expert e in topk[t, :], rounded to bf16
 // as the combine backward rounds it.
 constexpr int kGatherWarps = 8;
+constexpr int kGTile = 128;                     // rows and columns of an item
+constexpr int kGRowBytes = kGTile * 2 + 16;     // padded shared-memory row (bank spread)
+constexpr int kGBufBytes = kGTile * kGRowBytes;
 
 struct GateRows {
   const float* gates;     // [T, k], null: no gate
@@ -318,54 +324,120 @@ struct GateRows {
   int k, E;
 };
 
-__global__ void __launch_bounds__(32 * kGatherWarps)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_u32(dst)),
+               "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__global__ void __launch_bounds__(32 * kGatherWarps, 2)
 permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ src,
                          const int32_t* __restrict__ poff_end, int d, int A_pad_max,
                          uint8_t* __restrict__ Xq, uint8_t* __restrict__ Xs,
                          uint8_t* __restrict__ XqT, uint8_t* __restrict__ XsT, GateRows gr) {
+  extern __shared__ __align__(16) uint8_t gsm[];          // 2 x kGBufBytes
+  __shared__ int tok_s[2][kGTile];
+  __shared__ float gate_s[kGTile];
+  __shared__ __align__(4) uint8_t srow_s[kGTile][4];      // row scale bytes, 4 K blocks
+  __shared__ __align__(4) uint8_t scol_s[kGTile][4];      // column scale bytes, 4 row blocks
   const int nrows = min(*poff_end, A_pad_max);
-  const int segs = d / 256;
-  const int nblk = (nrows / 32) * segs;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int b = blockIdx.x; b < nblk; b += gridDim.x) {
-    const int rb = b / segs, seg = b - rb * segs;
-    const int r0 = rb * 32, r = r0 + lane;
-    const int c0 = seg * 256 + warp * 32;
-    const int t = src[r];
-    float v[32];
-    if (t >= 0) {
-      const uint4* p = reinterpret_cast<const uint4*>(x + (size_t)t * d + c0);
+  const int ctiles = d / kGTile;
+  const int nitems = (nrows / kGTile) * ctiles;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // gather the item's rows into buffer `buf` (16 threads per 256-byte row)
+  auto issue = [&](int item, int buf) {
+    const int rt = item / ctiles, ct = item - rt * ctiles;
+    const int r0 = rt * kGTile, c0 = ct * kGTile;
+    uint8_t* dst = gsm + buf * kGBufBytes;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) unpack8(__ldg(p + j), v + 8 * j);
-      if (gr.gates) {
-        // the block's group (largest e with poff[e] <= r0), then this
-        // token's slot of that expert
-        int lo = 0, hi = gr.E - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (__ldg(gr.poff + mid) <= r0) lo = mid; else hi = mid - 1;
-        }
-        float g = 0.f;
+    for (int it = 0; it < kGTile * 16 / (32 * kGatherWarps); ++it) {
+      const int i = tid + it * 32 * kGatherWarps;
+      const int row = i >> 4, ch = i & 15;
+      const int t = src[r0 + row];
+      if (ch == 0) tok_s[buf][row] = t;
+      const __nv_bfloat16* s = t >= 0 ? x + (size_t)t * d + c0 + ch * 8 : x;
+      cp_async16(dst + row * kGRowBytes + ch * 16, s, t >= 0);
+    }
+    cp_async_commit();
+  };
+
+  int it = 0;
+  if ((int)blockIdx.x < nitems) issue(blockIdx.x, 0);
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const int nxt = item + gridDim.x;
+    if (nxt < nitems) issue(nxt, buf ^ 1);
+    else cp_async_commit();                    // keep the group count uniform
+    cp_async_wait<1>();                        // this thread's copies of `item` landed
+    __syncthreads();                           // everyone's have
+    const int rt = item / ctiles, ct = item - rt * ctiles;
+    const int r0 = rt * kGTile, c0 = ct * kGTile;
+    if (gr.gates && tid < kGTile) {
+      // the item's group (largest e with poff[e] <= r0), then each row's
+      // token's slot of that expert
+      int lo = 0, hi = gr.E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(gr.poff + mid) <= r0) lo = mid; else hi = mid - 1;
+      }
+      const int t = tok_s[buf][tid];
+      float g = 0.f;
+      if (t >= 0)
         for (int j = 0; j < gr.k; ++j)
           if (__ldg(gr.topk + (size_t)t * gr.k + j) == lo) g = __ldg(gr.gates + (size_t)t * gr.k + j);
+      gate_s[tid] = g;
+    }
+    if (gr.gates) __syncthreads();
+    const uint8_t* tile = gsm + buf * kGBufBytes;
+    const int rb = warp >> 1;                  // this warp's 32-row block
+    const int row = rb * 32 + lane;
+    const float g = gr.gates ? gate_s[row] : 1.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cb = (warp & 1) * 2 + h;       // its 32-column block
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        unpack8(*reinterpret_cast<const uint4*>(tile + row * kGRowBytes + cb * 64 + j * 16), v + 8 * j);
+      if (gr.gates) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(g * v[j]));
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0.f;
+      uint32_t cr[8], cc[8], br, bc;
+      mx_quant_block32_regs(v, cr, cc, br, bc);
+      const size_t off = (size_t)(r0 + row) * d + c0 + cb * 32;
+      uint4* qr = reinterpret_cast<uint4*>(Xq + off);
+      uint4* qc = reinterpret_cast<uint4*>(XqT + off);
+      qr[0] = make_uint4(cr[0], cr[1], cr[2], cr[3]);
+      qr[1] = make_uint4(cr[4], cr[5], cr[6], cr[7]);
+      qc[0] = make_uint4(cc[0], cc[1], cc[2], cc[3]);
+      qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
+      srow_s[row][cb] = (uint8_t)br;
+      scol_s[cb * 32 + lane][rb] = (uint8_t)bc;
     }
-    uint32_t cr[8], cc[8], br, bc;
-    mx_quant_block32_regs(v, cr, cc, br, bc);
-    uint4* qr = reinterpret_cast<uint4*>(Xq + (size_t)r * d + c0);
-    uint4* qc = reinterpret_cast<uint4*>(XqT + (size_t)r * d + c0);
-    qr[0] = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-    qr[1] = make_uint4(cr[4], cr[5], cr[6], cr[7]);
-    qc[0] = make_uint4(cc[0], cc[1], cc[2], cc[3]);
-    qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
-    Xs[mx_sf_offset(r, c0 >> 5, d / 128)] = (uint8_t)br;
-    XsT[mx_sf_offset(c0 + lane, r0 >> 5, A_pad_max / 128)] = (uint8_t)bc;
+    __syncthreads();                           // buffer `buf` and the scale bytes are complete
+    // one word per row (its 4 K blocks of this item) and per column (its 4
+    // row blocks): the tensor-core layout keeps the 4 bytes adjacent
+    if (tid < kGTile) {
+      const int mn = r0 + tid;
+      *reinterpret_cast<uint32_t*>(Xs + mx_sf_offset(mn, c0 >> 5, d / 128)) =
+          *reinterpret_cast<const uint32_t*>(srow_s[tid]);
+    } else {
+      const int c = tid - kGTile, mn = c0 + c;
+      *reinterpret_cast<uint32_t*>(XsT + mx_sf_offset(mn, r0 >> 5, A_pad_max / 128)) =
+          *reinterpret_cast<const uint32_t*>(scol_s[c]);
+    }
+    __syncthreads();                           // scale staging reused by the next item
   }
+  cp_async_wait<0>();
 }
 
 }  // namespace moe
@@ -377,13 +449,15 @@ extern "C" moe_status_t moe_permute_mx(const void* x, const int32_t* src, const 
                                        uint8_t* Xs, uint8_t* XqT, uint8_t* XsT,
                                        moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && E > 0 && d > 0 && d % 256 == 0, "moe_permute_mx: d %% 256");
+  MOE_CHECK_ARG(T > 0 && E > 0 && d > 0 && d % 128 == 0, "moe_permute_mx: d %% 128");
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "moe_permute_mx: A_pad_max %% 128");
   MOE_CHECK_ARG(x && src && poff && Xq && Xs && XqT && XsT, "moe_permute_mx: null pointer");
   MOE_CHECK_ARG(aligned16(x) && aligned16(Xq) && aligned16(XqT), "moe_permute_mx: unaligned buffer");
-  const long long blocks = (long long)(A_pad_max / 32) * (d / 256);
-  const int grid = (int)std::min<long long>(blocks, 8LL * num_sms());
-  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 0, s>>>(
+  const long long items = (long long)(A_pad_max / kGTile) * (d / kGTile);
+  const int grid = (int)std::min<long long>(items, 2LL * num_sms());
+  MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(permute_mx_gather_kernel), 2 * kGBufBytes,
+                         "moe_permute_mx"));
+  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 2 * kGBufBytes, s>>>(
       static_cast<const __nv_bfloat16*>(x), src, poff + E, d, A_pad_max, Xq, Xs, XqT, XsT,
       GateRows{nullptr, nullptr, nullptr, 0, E});
   MOE_CHECK_LAUNCH("moe_permute_mx");
@@ -396,16 +470,18 @@ extern "C" moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
                                            int A_pad_max, uint8_t* dYq, uint8_t* dYs,
                                            uint8_t* dYTq, uint8_t* dYTs, moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && E > 0 && k > 0 && k <= 16 && d > 0 && d % 256 == 0,
-                "moe_combine_bwd_mx: d %% 256, 0 < k <= 16");
+  MOE_CHECK_ARG(T > 0 && E > 0 && k > 0 && k <= 16 && d > 0 && d % 128 == 0,
+                "moe_combine_bwd_mx: d %% 128, 0 < k <= 16");
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "moe_combine_bwd_mx: A_pad_max %% 128");
   MOE_CHECK_ARG(dout && gates && topk_idx && src && poff && dYq && dYs && dYTq && dYTs,
                 "moe_combine_bwd_mx: null pointer");
   MOE_CHECK_ARG(aligned16(dout) && aligned16(dYq) && aligned16(dYTq),
                 "moe_combine_bwd_mx: unaligned buffer");
-  const long long blocks = (long long)(A_pad_max / 32) * (d / 256);
-  const int grid = (int)std::min<long long>(blocks, 8LL * num_sms());
-  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 0, s>>>(
+  const long long items = (long long)(A_pad_max / kGTile) * (d / kGTile);
+  const int grid = (int)std::min<long long>(items, 2LL * num_sms());
+  MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(permute_mx_gather_kernel), 2 * kGBufBytes,
+                         "moe_combine_bwd_mx"));
+  permute_mx_gather_kernel<<<grid, 32 * kGatherWarps, 2 * kGBufBytes, s>>>(
       static_cast<const __nv_bfloat16*>(dout), src, poff + E, d, A_pad_max, dYq, dYs, dYTq, dYTs,
       GateRows{gates, topk_idx, poff, k, E});
   MOE_CHECK_LAUNCH("moe_combine_bwd_mx");
