@@ -65,10 +65,9 @@ moe_status_t grouped_gemm_wgrad(int dt, const void* A, const uint8_t* A_sc, cons
 
 // Weight-gradient grouped GEMM (BF16) on SM pairs (grouped_gemm_pair.cu):
 // dB[e] = A_e^T dC_e (+ dB3 from dC's second N half), reduced over group e
-// up to its last real row; A the padded buffer, or with a_src the
-// unpermuted x [a_rows, K] gathered by row.  K % 256 == 0, N % 256 == 0.
-moe_status_t grouped_gemm_wgrad_pair(const void* A, const int32_t* a_src, int a_rows,
-                                     const void* dC, const int32_t* poff, const int32_t* offsets,
+// up to its last real row; A the padded buffer.  K % 256 == 0, N % 256 == 0.
+moe_status_t grouped_gemm_wgrad_pair(const void* A, const void* dC, const int32_t* poff,
+                                     const int32_t* offsets,
                                      int E, int A_pad_max, int K, int N, void* dB, void* dB3,
                                      int32_t* dev_status, cudaStream_t s);
 

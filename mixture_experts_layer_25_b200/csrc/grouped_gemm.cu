@@ -126,6 +126,7 @@ struct Params {
   // a_src[r] of the unpermuted tokens (a_src[r] < 0: a zero row, read as the
   // out-of-range row a_oob)
   const int32_t* a_src; int a_oob;
+  const __nv_bfloat16* a_x; int a_ld;   // the unpermuted rows and their length (K or M)
   // router epilogue
   const float* r_bias; float* r_logits; int32_t* r_topk; float* r_gates;
   int32_t* r_rank; int32_t* r_hist; int r_k; int r_E;
@@ -247,6 +248,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   __shared__ int poff_s[MAX_E + 1];
   __shared__ int krows_s[A_MN ? MAX_E : 1];  // wgrad: reduction rows of each group
   __shared__ volatile int abort_flag;
+  __shared__ int gtok_s[GATHER ? BM : 1];    // gathered A: token of each row being copied
+  __shared__ __align__(16) float qinv_s[MX ? NUM_EPI_WARPS : 1][32];   // quantising epilogues
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -269,7 +272,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      // gathered A: the B bytes' arrival plus one per producer lane's copies
+      mbar_init(&full_bar[s], GATHER ? 1 + 32 : 1);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -310,40 +314,74 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0 && GATHER) {
     // ------------------------------------------------- producer (gathered A)
-    // The whole warp: lane 0 owns the barriers and the B loads; each lane
-    // gathers four A rows per stage (row mode: rows 4 lane.. of the 128-row
-    // tile; weight-gradient mode: K rows 4 (lane % 16).. of the stage's 64,
-    // for the 64-column chunk lane / 16 of the tile's 128 M columns).
+    // The whole warp copies the A rows from the unpermuted x with 16-byte
+    // cp.async (completion: each lane's cp.async.mbarrier.arrive.noinc on
+    // the stage's full barrier, whose count includes the 32 lanes); lane 0
+    // posts the B bytes and issues the B loads with TMA.  16-byte unit j of a
+    // 128-byte shared-memory row r sits at (j ^ (r & 7)) * 16: the layout of
+    // the TMA 128-byte swizzle the MMA descriptors expect.  A token row < 0
+    // (a pad row) is zero-filled.
+    //  rows mode: the tile's 128 rows x 64 K; lane l copies unit l % 8 of
+    //    rows 4 i + l / 8, i = 0..31;
+    //  weight-gradient mode: the stage's 64 K rows (tokens) x the tile's 128
+    //    M columns, two 64-column chunks; lane l copies unit l % 8 of rows
+    //    4 i + l / 8 of both chunks, i = 0..15.
     int stage = 0;
     uint32_t phase = 0;
     uint32_t used = 0, last_parity = 0;
     bool stop = false;
+    const __nv_bfloat16* xb = p.a_x;
+    const int j = lane & 7;
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
       const Tile t = decode(p, poff_s, tile);
       const int nkb = group_kb(t);
-      int4 rows = make_int4(0, 0, 0, 0);
-      if constexpr (!A_MN) rows = gather_rows(p, t.row0 + 4 * lane);
-      int4 next_rows = rows;
-      if constexpr (A_MN) if (nkb > 0) next_rows = gather_rows(p, t.krow0 + 4 * (lane & 15));
+      if constexpr (!A_MN) {
+        const int4 v = __ldg(reinterpret_cast<const int4*>(p.a_src + t.row0 + 4 * lane));
+        __syncwarp();
+        gtok_s[4 * lane] = v.x; gtok_s[4 * lane + 1] = v.y;
+        gtok_s[4 * lane + 2] = v.z; gtok_s[4 * lane + 3] = v.w;
+        __syncwarp();
+      }
       for (int kb = 0; kb < nkb; ++kb) {
-        if constexpr (A_MN) {
-          rows = next_rows;
-          if (kb + 1 < nkb) next_rows = gather_rows(p, t.krow0 + (kb + 1) * BK + 4 * (lane & 15));
-        }
         int ok = 1;
         if (lane == 0)
           ok = mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { stop = true; break; }
         uint64_t* fb = &full_bar[stage];
-        if (lane == 0) mbar_arrive_expect_tx(fb, STAGE_TX);
-        __syncwarp();
+        if constexpr (A_MN) {
+          __syncwarp();
+          if (lane < 16) {
+            const int4 v = __ldg(reinterpret_cast<const int4*>(p.a_src + t.krow0 + kb * BK + 4 * lane));
+            gtok_s[4 * lane] = v.x; gtok_s[4 * lane + 1] = v.y;
+            gtok_s[4 * lane + 2] = v.z; gtok_s[4 * lane + 3] = v.w;
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mbar_arrive_expect_tx(fb, STAGE_TX - A_BYTES);
         uint8_t* a_dst = sA + stage * A_BYTES;
-        if constexpr (!A_MN)
-          tma_gather4(a_dst + lane * 512, &tmA, fb, kb * BK, rows.x, rows.y, rows.z, rows.w);
-        else
-          tma_gather4(a_dst + (lane >> 4) * MN_CHUNK_BYTES + (lane & 15) * 512, &tmA, fb,
-                      t.m0 + (lane >> 4) * MN_CHUNK, rows.x, rows.y, rows.z, rows.w);
+        if constexpr (!A_MN) {
+#pragma unroll 8
+          for (int i = 0; i < 32; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const int tk = gtok_s[r];
+            const __nv_bfloat16* src = tk >= 0 ? xb + (size_t)tk * p.a_ld + kb * BK + j * 8 : xb;
+            cp_async16(a_dst + r * 128 + ((j ^ (r & 7)) << 4), src, tk >= 0);
+          }
+        } else {
+#pragma unroll 8
+          for (int i = 0; i < 16; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            const int tk = gtok_s[r];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const __nv_bfloat16* src =
+                  tk >= 0 ? xb + (size_t)tk * p.a_ld + t.m0 + c * MN_CHUNK + j * 8 : xb;
+              cp_async16(a_dst + c * MN_CHUNK_BYTES + r * 128 + ((j ^ (r & 7)) << 4), src, tk >= 0);
+            }
+          }
+        }
+        cp_async_arrive_noinc(fb);
         if (lane == 0) {
           uint8_t* b_dst = sB + stage * B_STAGE;
           const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
@@ -361,7 +399,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
-    if (lane == 0)     // every load of the warp has landed before the CTA exits
+    if (lane == 0)     // every copy and load of the warp has landed before the CTA exits
       for (int s = 0; s < STAGES; ++s)
         if (used & (1u << s)) {
           volatile int no_abort = 0;
@@ -510,6 +548,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           tc_fence_after();
+          // gathered A was written by cp.async (generic proxy): order it
+          // before the tensor core's reads (async proxy)
+          if constexpr (GATHER) fence_async_smem();
           const uint32_t sa = a_base + stage * A_BYTES, sb = b_base + stage * B_STAGE;
           uint32_t sfa_t = 0, sfb_t = 0;
           if constexpr (MX) {
@@ -602,11 +643,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       // epilogue keeps no other large state; otherwise each 32-column chunk
       // is read from TMEM when it is stored and the accumulator is released
       // at the end of the tile (BF16 double-buffers its accumulators).
-#ifndef MOE_MX_BWD_EARLY
-#define MOE_MX_BWD_EARLY 1
-#endif
-      constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU ||
-                                    (EPI == EPI_SWIGLU_BWD && MOE_MX_BWD_EARLY));
+      // (the SwiGLU backward keeps the per-chunk path: with its whole slice
+      // in registers it spills, measured 2.3x slower)
+      constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU);
       constexpr int NV = EARLY ? 128 : 32;
       uint32_t av[NV];
       if constexpr (EARLY) {
@@ -746,7 +785,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 hv[2 * i + 1] = f2.y;
               }
               mx_quant_block32(hv, stg, stg + 1024, p.q_sr, y0 + r, n0 + c, p.q_row_kchunks,
-                               p.q_sc, y0, p.q_col_kchunks);
+                               p.q_sc, y0, p.q_col_kchunks, qinv_s[MX ? ew : 0]);
             }
           }
           if constexpr (ONE_BOX) {
@@ -790,7 +829,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {  // accumulator = dh, columns [nt*256, +256)
         const int n0 = t.nt * BN + hc * (BN / 2);
         constexpr int NCH = BN / 2 / CHUNK;
-#pragma unroll(EARLY ? NCH : 1)
+#pragma unroll 1
         for (int ci = 0; ci < NCH; ++ci) {
           const int c = ci * CHUNK;
           const int pr = ci & 1;                      // staging pair of this chunk
@@ -804,11 +843,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tma_load_2d(n1 + BOX_BYTES, &tmIn, &in_bar[ew][pr ^ 1], p.half + n0 + c + CHUNK, y0);
             in_pending |= 1u << (pr ^ 1);
           }
-          uint32_t* v = av + (EARLY ? 32 * ci : 0);
-          if constexpr (!EARLY) {
-            tmem_ld32(tbase + hc * (BN / 2) + c, v);
-            tmem_wait_ld();
-          }
+          uint32_t* v = av;
+          tmem_ld32(tbase + hc * (BN / 2) + c, v);
+          tmem_wait_ld();
           int got = 1;
           if (lane == 0)
             got = mbar_wait(&in_bar[ew][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
@@ -859,7 +896,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 for (int j = 0; j < 4; ++j) unpack8(k4[j], dv + 8 * j);
                 uint8_t* box = o == 0 ? b1 : b3;
                 mx_quant_block32(dv, box, box + 1024, p.q_sr, y0 + r, (o ? p.half : 0) + n0 + c,
-                                 p.q_row_kchunks, p.q_sc, y0, p.q_col_kchunks);
+                                 p.q_row_kchunks, p.q_sc, y0, p.q_col_kchunks, qinv_s[MX ? ew : 0]);
               }
             }
           }
@@ -1218,8 +1255,10 @@ static moe_status_t fwd_impl(int dt, const void* A, const uint8_t* A_sc, const v
   p.C = static_cast<__nv_bfloat16*>(C);
   p.a_src = a_src;
   p.a_oob = a_rows;
+  p.a_x = static_cast<const __nv_bfloat16*>(A);
+  p.a_ld = K;
   Maps m;
-  if (gather) MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));
+  if (gather) MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));   // unused by the gathering producer
   else MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, BM));
   if (epilogue == MOE_EPI_NONE) {
     MOE_CHECK_ARG(N > 0 && N % 256 == 0, "gemm_fwd: N %% 256");
@@ -1493,10 +1532,12 @@ static moe_status_t wgrad_impl(int dt, const void* A, const uint8_t* A_sc, const
   MOE_CHECK_ARG(A && dC && dB && poff, "gemm_wgrad: null pointer");
   MOE_CHECK_ARG(!mx || (A_sc && dC_sc), "gemm_wgrad: MX needs scales");
 #ifndef MOE_NO_PAIR_WGRAD
-  // BF16 with 256-aligned weight shapes: 256 x 256 tiles on SM pairs
-  if (!mx && K % 256 == 0)
-    return grouped_gemm_wgrad_pair(A, a_src, a_rows, dC, poff, offsets, E, A_pad_max, K, N, dB,
-                                   dB3, dev_status, s);
+  // BF16 with 256-aligned weight shapes: 256 x 256 tiles on SM pairs (the
+  // gathered form runs on single SMs: its cp.async copies signal a barrier
+  // of their own CTA only)
+  if (!mx && !gather && K % 256 == 0)
+    return grouped_gemm_wgrad_pair(A, dC, poff, offsets, E, A_pad_max, K, N, dB, dB3, dev_status,
+                                   s);
 #endif
   const int eb = mx ? 1 : 2;
   const int Ncols = dB3 ? 2 * N : N;
@@ -1517,9 +1558,11 @@ static moe_status_t wgrad_impl(int dt, const void* A, const uint8_t* A_sc, const
   p.c_expert_stride = (long long)K * N;
   p.a_src = a_src;
   p.a_oob = a_rows;
+  p.a_x = static_cast<const __nv_bfloat16*>(A);
+  p.a_ld = K;
   Maps m;
   if (gather) {
-    MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));
+    MOE_TRY(make_map(&m.a, A, 2, K, a_rows, 64, 1));   // unused by the gathering producer
   } else {
     p.a3d = make_map_mn3(&m.a, A, eb, K, A_pad_max, 128 / eb, BM * eb / 128);
     if (!p.a3d) MOE_TRY(make_map(&m.a, A, eb, K, A_pad_max, 128 / eb, 128 / eb));

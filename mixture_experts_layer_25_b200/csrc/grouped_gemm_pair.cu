@@ -60,8 +60,6 @@ struct Params {
   int n_tiles;              // tiles along N (Ncols / 256)
   int k_out;                // output rows per expert (K_out)
   int n_split;              // > 0: columns >= n_split go to the second output
-  const int32_t* a_src;     // gathered A: row r is x[a_src[r]] (null: A is the padded buffer)
-  int a_oob;                // out-of-range row index for pad rows (= T)
   int32_t* status;
 };
 
@@ -73,32 +71,11 @@ __device__ __forceinline__ uint32_t sw64(int r, int j) {
   return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
 
-__device__ __forceinline__ int4 gather_rows(const Params& p, int r) {
-  int4 v = __ldg(reinterpret_cast<const int4*>(p.a_src + r));
-  v.x = v.x < 0 ? p.a_oob : v.x;
-  v.y = v.y < 0 ? p.a_oob : v.y;
-  v.z = v.z < 0 ? p.a_oob : v.z;
-  v.w = v.w < 0 ? p.a_oob : v.w;
-  return v;
-}
-
-// 4 rows of a 2-D one-row-box map into this CTA's shared memory, completion
-// on the leader's mbarrier (shared::cluster address)
-__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* m, uint32_t bar,
-                                                 int x, int y0, int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-      : "memory");
-}
-
 // instruction descriptor: bf16 x bf16 -> fp32, A and B MN-major, M = 256
 // (the pair), N = 256
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
-template <bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
@@ -182,9 +159,7 @@ wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // lane 0 owns the barriers and the B loads (and the A loads unless they
-    // are gathered, in which case every lane gathers 4 of the 64 K rows of
-    // one of the two 64-column A chunks)
+    // lane 0 owns the barriers and issues both operands' loads
     const uint32_t full_leader0 = map_to_rank(&full_bar[0], 0);
     int stage = 0;
     uint32_t phase = 0;
@@ -196,8 +171,6 @@ wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int nkb = nkb_of(e);
       const int krow0 = poff_s[e];
       for (int kb = 0; kb < nkb; ++kb) {
-        int4 rows = make_int4(0, 0, 0, 0);
-        if constexpr (GATHER) rows = gather_rows(p, krow0 + kb * BK + 4 * (lane & 15));
         int ok = 1;
         if (lane == 0)
           ok = mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, p.status, kWaitLimitNs);
@@ -208,14 +181,10 @@ wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         __syncwarp();
         uint8_t* a_dst = sA + stage * A_BYTES;
         uint8_t* b_dst = sB + stage * B_BYTES;
-        if constexpr (GATHER) {
-          tma_gather4_pair(a_dst + (lane >> 4) * CHUNK_BYTES + (lane & 15) * 512, &tmA, fb,
-                           m0 + (lane >> 4) * 64, rows.x, rows.y, rows.z, rows.w);
-        } else if (lane == 0) {
+        if (lane == 0) {
           tma_load_3d_pair(a_dst, &tmA, fb, 0, krow0 + kb * BK, m0 / 64);
-        }
-        if (lane == 0)
           tma_load_3d_pair(b_dst, &tmB, fb, 0, krow0 + kb * BK, (nt * BN + (int)rank * (BN / 2)) / 64);
+        }
         used |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -390,10 +359,9 @@ bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATHER>
 moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                     const CUtensorMap& c2, const Params& p, int tiles, cudaStream_t s) {
-  auto kern = wgrad_pair_kernel<GATHER>;
+  auto kern = wgrad_pair_kernel;
   MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(kern), SMEM, "wgrad_pair"));
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -428,20 +396,16 @@ moe_status_t launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
 // Weight-gradient grouped GEMM (BF16) on SM pairs: dB[e] = A_e^T dC_e (and
 // dB3 from dC's second half when dB3 is given), reduced over the rows of
 // group e up to its last real row (offsets, or every padded row).  A is the
-// padded buffer [A_pad_max, K], or with a_src the unpermuted x [a_rows, K]
-// gathered by row (a_src[r] < 0: zero row).  K % 256 == 0, N % 256 == 0.
-moe_status_t grouped_gemm_wgrad_pair(const void* A, const int32_t* a_src, int a_rows,
-                                     const void* dC, const int32_t* poff, const int32_t* offsets,
+// padded buffer [A_pad_max, K].  K % 256 == 0, N % 256 == 0.
+moe_status_t grouped_gemm_wgrad_pair(const void* A, const void* dC, const int32_t* poff,
+                                     const int32_t* offsets,
                                      int E, int A_pad_max, int K, int N, void* dB, void* dB3,
                                      int32_t* dev_status, cudaStream_t s) {
   using namespace gp;
-  const bool gather = a_src != nullptr;
   MOE_CHECK_ARG(E > 0 && E <= MAX_E, "wgrad_pair: E must be in [1, %d]", MAX_E);
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "wgrad_pair: A_pad_max %% 128");
   MOE_CHECK_ARG(K > 0 && K % 256 == 0 && N > 0 && N % 256 == 0, "wgrad_pair: K, N %% 256");
   MOE_CHECK_ARG(A && dC && dB && poff, "wgrad_pair: null pointer");
-  MOE_CHECK_ARG(!gather || (a_rows > 0 && aligned16(a_src) && aligned16(A)),
-                "wgrad_pair: gathered A needs T > 0 and 16-byte aligned x and src");
   const int Ncols = dB3 ? 2 * N : N;
   Params p{};
   p.poff = poff;
@@ -451,12 +415,9 @@ moe_status_t grouped_gemm_wgrad_pair(const void* A, const int32_t* a_src, int a_
   p.n_tiles = Ncols / BN;
   p.k_out = K;
   p.n_split = dB3 ? N : 0;
-  p.a_src = a_src;
-  p.a_oob = a_rows;
   p.status = dev_status;
   CUtensorMap ma, mb, mc, mc2;
-  bool ok = gather ? map_2d(&ma, A, K, a_rows, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)
-                   : map_mn3(&ma, A, K, A_pad_max, BK, 2);
+  bool ok = map_mn3(&ma, A, K, A_pad_max, BK, 2);
   ok = ok && map_mn3(&mb, dC, Ncols, A_pad_max, BK, 2);
   ok = ok && map_2d(&mc, dB, N, (uint64_t)E * K, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   ok = ok && (dB3 ? map_2d(&mc2, dB3, N, (uint64_t)E * K, CHUNK, 32, CU_TENSOR_MAP_SWIZZLE_64B)
@@ -466,8 +427,7 @@ moe_status_t grouped_gemm_wgrad_pair(const void* A, const int32_t* a_src, int a_
     return MOE_ERR_CUDA;
   }
   const int tiles = E * p.m_tiles * p.n_tiles;
-  return gather ? launch<true>(ma, mb, mc, mc2, p, tiles, s)
-                : launch<false>(ma, mb, mc, mc2, p, tiles, s);
+  return launch(ma, mb, mc, mc2, p, tiles, s);
 }
 
 }  // namespace moe

@@ -53,7 +53,12 @@ bool tokens_n(const moe_layer_desc* L);
 
 // The BF16 layer on the main grouped GEMM reads the token rows straight
 // from x (row gathers in the GEMM1 producers): no permuted copy Xp.
-bool gathers(const moe_layer_desc* L) { return false && L->dtype == MOE_BF16 && !tokens_n(L); }
+#ifndef MOE_GATHER_DISPATCH
+#define MOE_GATHER_DISPATCH 1
+#endif
+bool gathers(const moe_layer_desc* L) {
+  return MOE_GATHER_DISPATCH && L->dtype == MOE_BF16 && !tokens_n(L);
+}
 
 size_t layout(const moe_layer_desc* L, void* base, moe_ctx_view* v) {
   Layout l;
@@ -149,10 +154,13 @@ extern "C" moe_status_t moe_layer_ctx_view(const moe_layer_desc* desc, void* ctx
 // T = 8192, k = 8, E = 384), and multiplying only the real rows pays for
 // that kernel's lower per-tile rate (measured: 12% faster layer at that
 // shape, 6-7% slower at 512 rows per expert).
+#ifndef MOE_TN_MIN_ROWS
+#define MOE_TN_MIN_ROWS 256     // mean rows per expert below which the tokens-N kernel runs
+#endif
 namespace {
 bool tokens_n(const moe_layer_desc* L) {
-  return L->dtype == MOE_BF16 && (long long)L->T * L->k < 256LL * L->E && L->d % 128 == 0 &&
-         L->F % 64 == 0;
+  return L->dtype == MOE_BF16 && (long long)L->T * L->k < (long long)MOE_TN_MIN_ROWS * L->E &&
+         L->d % 128 == 0 && L->F % 64 == 0;
 }
 }  // namespace
 

@@ -49,31 +49,36 @@ __device__ __forceinline__ uint2 mx_encode8(const float* f, float inv) {
 // j) quantised both ways: cr = the lane's row codes (blocks of 32 along the
 // row), cc = its codes under the column scales (blocks of 32 rows down each
 // column), 4 codes per word in column order; br = the row's scale byte,
-// bc = the scale byte of column `lane`.
+// bc = the scale byte of column `lane`.  Each lane works out only its own
+// column's scale and the 32 reciprocal scales reach every lane through
+// inv_s (32 floats of this warp's shared memory).
 __device__ __forceinline__ void mx_quant_block32_regs(const float* v, uint32_t* cr, uint32_t* cc,
-                                                      uint32_t& br, uint32_t& bc) {
+                                                      uint32_t& br, uint32_t& bc, float* inv_s) {
   const int lane = threadIdx.x & 31;
   float amax = 0.f;
 #pragma unroll
   for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
   br = mx_scale_byte(amax);
   const float inv = mx_inv_scale(br);
-  bc = 0;
+  // column maxima over the warp's 32 rows (non-negative floats order like
+  // their bit patterns); lane j keeps column j's
+  uint32_t mine = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(v[j]) & 0x7fffffffu);
+    mine = lane == j ? m : mine;
+  }
+  bc = mx_scale_byte(__uint_as_float(mine));
+  __syncwarp();
+  inv_s[lane] = mx_inv_scale(bc);
+  __syncwarp();
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
-    uint32_t b[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      // column maximum over the warp's 32 rows (non-negative floats order
-      // like their bit patterns)
-      const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j + i])));
-      b[i] = mx_scale_byte(__uint_as_float(m));
-      if (lane == j + i) bc = b[i];
-    }
+    const float4 ic = *reinterpret_cast<const float4*>(inv_s + j);
     cr[j / 4] = mx_encode2(v[j] * inv, v[j + 1] * inv) |
                 (mx_encode2(v[j + 2] * inv, v[j + 3] * inv) << 16);
-    cc[j / 4] = mx_encode2(v[j] * mx_inv_scale(b[0]), v[j + 1] * mx_inv_scale(b[1])) |
-                (mx_encode2(v[j + 2] * mx_inv_scale(b[2]), v[j + 3] * mx_inv_scale(b[3])) << 16);
+    cc[j / 4] = mx_encode2(v[j] * ic.x, v[j + 1] * ic.y) |
+                (mx_encode2(v[j + 2] * ic.z, v[j + 3] * ic.w) << 16);
   }
 }
 
@@ -82,14 +87,14 @@ __device__ __forceinline__ void mx_quant_block32_regs(const float* v, uint32_t* 
 // codes) and the scale bytes to global memory: the row scale of (row,
 // col0/32) with K = the row length (row_kchunks = K / 128), the column
 // scale of (col0 + lane, row0/32) with K = the padded row count
-// (col_kchunks = A_pad_max / 128).
+// (col_kchunks = A_pad_max / 128).  inv_s: as in mx_quant_block32_regs.
 __device__ __forceinline__ void mx_quant_block32(const float* v, uint8_t* box_r, uint8_t* box_c,
                                                  uint8_t* scales_r, int row, int col0,
                                                  int row_kchunks, uint8_t* scales_c, int row0,
-                                                 int col_kchunks) {
+                                                 int col_kchunks, float* inv_s) {
   const int lane = threadIdx.x & 31;
   uint32_t cr[8], cc[8], br, bc;
-  mx_quant_block32_regs(v, cr, cc, br, bc);
+  mx_quant_block32_regs(v, cr, cc, br, bc, inv_s);
   *reinterpret_cast<uint4*>(box_r + lane * 32) = make_uint4(cr[0], cr[1], cr[2], cr[3]);
   *reinterpret_cast<uint4*>(box_r + lane * 32 + 16) = make_uint4(cr[4], cr[5], cr[6], cr[7]);
   *reinterpret_cast<uint4*>(box_c + lane * 32) = make_uint4(cc[0], cc[1], cc[2], cc[3]);

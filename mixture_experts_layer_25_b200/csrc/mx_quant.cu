@@ -324,11 +324,7 @@ struct GateRows {
   int k, E;
 };
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sm100::smem_u32(dst)),
-               "l"(src), "r"(valid ? 16 : 0)
-               : "memory");
-}
+using sm100::cp_async16;
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -347,6 +343,7 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
   __shared__ float gate_s[kGTile];
   __shared__ __align__(4) uint8_t srow_s[kGTile][4];      // row scale bytes, 4 K blocks
   __shared__ __align__(4) uint8_t scol_s[kGTile][4];      // column scale bytes, 4 row blocks
+  __shared__ __align__(16) float qinv_s[kGatherWarps][32];  // each warp's column scales
   const int nrows = min(*poff_end, A_pad_max);
   const int ctiles = d / kGTile;
   const int nitems = (nrows / kGTile) * ctiles;
@@ -412,7 +409,7 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
         for (int j = 0; j < 32; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(g * v[j]));
       }
       uint32_t cr[8], cc[8], br, bc;
-      mx_quant_block32_regs(v, cr, cc, br, bc);
+      mx_quant_block32_regs(v, cr, cc, br, bc, qinv_s[warp]);
       const size_t off = (size_t)(r0 + row) * d + c0 + cb * 32;
       uint4* qr = reinterpret_cast<uint4*>(Xq + off);
       uint4* qc = reinterpret_cast<uint4*>(XqT + off);
