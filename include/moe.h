@@ -136,7 +136,8 @@ MOE_API void moe_set_stage_events(void* const* events, int n);
  *   lower index, slot j = j-th largest), gates = softmax of the k chosen
  *   logits (fp32); writes topk_idx [T,k] and gates [T,k].  With E <= 128,
  *   E % 8 == 0, k <= 8 and d % 64 == 0 the logits run on the tensor cores:
- *   W_r is split exactly into three bf16 parts (w0 + w1 + w2 = W_r, each
+ *   W_r is split into two bf16 parts (w0 + w1 = W_r within 2^-17 |W_r|,
+ *   below the fp32 accumulation error of a sum over d >= 32 terms; each
  *   product exact) accumulated in fp32; otherwise fp32 FMA on CUDA cores.
  * mode MOE_ROUTE_GIVEN: topk_idx and gates are INPUTS (random-routing stress
  *   workload, [OC3-ja] "実証されたスケール"); x and W_r are not read.  An index

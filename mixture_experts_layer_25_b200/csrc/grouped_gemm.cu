@@ -77,13 +77,14 @@ template <bool MX, int EPI, bool WGRAD = false> struct EpiCfg {
   static constexpr int SWIGLU_STAGES = MX ? 3 : MOE_GG_SWIGLU_STAGES;
   static constexpr int STORE_BOXES = WGRAD ? MOE_GG_WGRAD_BOXES : MOE_GG_STORE_BOXES;
   static constexpr int STAGES = EPI == EPI_STORE ? (STORE_BOXES == 1 ? 4 : 3)
-                              : EPI == EPI_SWIGLU ? SWIGLU_STAGES : 3;
+                              : EPI == EPI_SWIGLU ? SWIGLU_STAGES
+                              : is_router(EPI) ? 4 : 3;
   static constexpr int BOXES = EPI == EPI_STORE ? STORE_BOXES
                              : is_router(EPI) ? 1
                              : EPI == EPI_SWIGLU ? (SWIGLU_STAGES == 4 ? 1 : 3) : 4;
   static constexpr int STG = BOXES * BOX_BYTES;
-  // the router stage holds three B tiles (one per weight split) of <= 128 columns
-  static constexpr int B_STAGE = is_router(EPI) ? 3 * 128 * 128 : B_BYTES;
+  // the router stage holds two B tiles (one per weight split) of <= 128 columns
+  static constexpr int B_STAGE = is_router(EPI) ? 2 * 128 * 128 : B_BYTES;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_STAGE +
                                  (MX ? SFA_BYTES + SFB_BYTES : 0)) + NUM_EPI_WARPS * STG;
 };
@@ -424,7 +425,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           uint64_t* fb = &full_bar[stage];
           const int nbox = p.b_boxes ? p.b_boxes : BN / MN_CHUNK;
           if constexpr (is_router(EPI))
-            mbar_arrive_expect_tx(fb, A_BYTES + 3 * nbox * MN_CHUNK_BYTES);
+            mbar_arrive_expect_tx(fb, A_BYTES + 2 * nbox * MN_CHUNK_BYTES);
           else
             mbar_arrive_expect_tx(fb, B_MNMAJOR ? STAGE_TX - (BN / MN_CHUNK - nbox) * MN_CHUNK_BYTES
                                                 : STAGE_TX);
@@ -445,7 +446,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const int brow = p.wgrad ? t.krow0 : t.e * p.b_rows_per_e;
           if constexpr (is_router(EPI)) {
             // rows kb*BK.. of each weight split (split s starts at row s * d)
-            for (int sp = 0; sp < 3; ++sp)
+            for (int sp = 0; sp < 2; ++sp)
               for (int i = 0; i < nbox; ++i)
                 tma_load_2d(b_dst + sp * SPLIT_BYTES + i * MN_CHUNK_BYTES, &tmB, fb, i * MN_CHUNK,
                             sp * p.split_rows + kb * BK);
@@ -566,7 +567,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int ks = 0; ks < KSTEPS; ++ks) {
               const uint64_t ad = smem_desc(sa + ks * 32, 16, 1024, 2);
 #pragma unroll
-              for (int sp = 0; sp < 3; ++sp) {
+              for (int sp = 0; sp < 2; ++sp) {
                 const uint64_t bd =
                     smem_desc(sb + sp * SPLIT_BYTES + ks * MMA_K * 128, MN_CHUNK_BYTES, 1024, 2);
                 mma_bf16(d_tmem, ad, bd, idesc, (kb > 0 || ks > 0 || sp > 0) ? 1u : 0u);
@@ -1065,6 +1066,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     }
   }
 
+  // every warp reconverges first: lanes that skipped a one-lane role loop
+  // (producer, MMA issue) must not reach the CTA barrier, or the warp-wide
+  // TMEM free after it, ahead of that lane
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -1162,9 +1167,9 @@ static Params base_params(const int32_t* poff, int E, int32_t* status) {
 }
 
 // Router logits on the tensor cores: x [T, d] (bf16) times W_r split exactly
-// into three bf16 parts stacked as wsplit [3d, E] (w0 + w1 + w2 = W_r): each
-// stage holds one x tile and the three split tiles of the same K rows, and
-// all three products accumulate into one fp32 TMEM accumulator; top-k,
+// into two bf16 parts stacked as wsplit [2d, E] (w0 + w1 = W_r to within
+// 2^-17 |W_r|): each stage holds one x tile and the two split tiles of the
+// same K rows, and both products accumulate into one fp32 TMEM accumulator; top-k,
 // gates, per-128-token-block ranks and histogram in the epilogue.
 namespace moe {
 moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int T, int d, int E,
@@ -1188,7 +1193,7 @@ moe_status_t router_tc(const void* x, const void* wsplit, const float* bias, int
   p.r_E = E;
   Maps m;
   MOE_TRY(make_map(&m.a, x, 2, d, T, 64, BM));
-  MOE_TRY(make_map(&m.b, wsplit, 2, E, 3ULL * d, 64, 64));
+  MOE_TRY(make_map(&m.b, wsplit, 2, E, 2ULL * d, 64, 64));
   m.b3 = m.c = m.c2 = m.in = m.a;
   return k <= 4 ? launch<false, false, B_MN, EPI_ROUTER4>(m, p, (T + BM - 1) / BM, s)
                 : launch<false, false, B_MN, EPI_ROUTER>(m, p, (T + BM - 1) / BM, s);

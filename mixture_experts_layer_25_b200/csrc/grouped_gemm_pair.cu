@@ -323,6 +323,10 @@ wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     while (globaltimer_ns() - t0 < 100000ull) {
     }
   }
+  // every warp reconverges first: lanes that skipped a one-lane role loop
+  // (producer, MMA issue) must not reach the cluster barrier, or the warp-wide
+  // TMEM free after it, ahead of that lane
+  __syncwarp();
   tc_fence_before();
   cluster_sync_all();
   if (warp == 1) {

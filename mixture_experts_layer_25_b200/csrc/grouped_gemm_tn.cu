@@ -438,6 +438,11 @@ gemm_tn_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ 
     if (lane == 0) bulk_wait_all();
   }
 
+  // every warp reconverges first: lanes that skipped a one-lane role loop
+  // (producer, MMA issue) must not reach the CTA barrier, or the warp-wide
+  // TMEM free after it, ahead of that lane
+  __syncwarp();
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

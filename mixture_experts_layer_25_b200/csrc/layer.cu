@@ -54,7 +54,7 @@ bool tokens_n(const moe_layer_desc* L);
 // The BF16 layer on the main grouped GEMM reads the token rows straight
 // from x (row gathers in the GEMM1 producers): no permuted copy Xp.
 #ifndef MOE_GATHER_DISPATCH
-#define MOE_GATHER_DISPATCH 1
+#define MOE_GATHER_DISPATCH 0     // measured slower than the permute pass: off
 #endif
 bool gathers(const moe_layer_desc* L) {
   return MOE_GATHER_DISPATCH && L->dtype == MOE_BF16 && !tokens_n(L);

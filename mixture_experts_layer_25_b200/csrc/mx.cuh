@@ -37,11 +37,18 @@ __device__ __forceinline__ uint32_t mx_encode2(float a, float b) {
   return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
 }
 
+// two values scaled by (power-of-two, so exact) factors -> two E4M3 codes;
+// one packed fp32 multiply for the pair
+__device__ __forceinline__ uint32_t mx_encode2s(float a, float b, float sa, float sb) {
+  const float2 q = __fmul2_rn(make_float2(a, b), make_float2(sa, sb));
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+}
+
 // 8 values -> 8 E4M3 codes (memory order)
 __device__ __forceinline__ uint2 mx_encode8(const float* f, float inv) {
   uint32_t w[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = mx_encode2(f[2 * i] * inv, f[2 * i + 1] * inv);
+  for (int i = 0; i < 4; ++i) w[i] = mx_encode2s(f[2 * i], f[2 * i + 1], inv, inv);
   return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
 
@@ -75,10 +82,10 @@ __device__ __forceinline__ void mx_quant_block32_regs(const float* v, uint32_t* 
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     const float4 ic = *reinterpret_cast<const float4*>(inv_s + j);
-    cr[j / 4] = mx_encode2(v[j] * inv, v[j + 1] * inv) |
-                (mx_encode2(v[j + 2] * inv, v[j + 3] * inv) << 16);
-    cc[j / 4] = mx_encode2(v[j] * ic.x, v[j + 1] * ic.y) |
-                (mx_encode2(v[j + 2] * ic.z, v[j + 3] * ic.w) << 16);
+    cr[j / 4] = mx_encode2s(v[j], v[j + 1], inv, inv) |
+                (mx_encode2s(v[j + 2], v[j + 3], inv, inv) << 16);
+    cc[j / 4] = mx_encode2s(v[j], v[j + 1], ic.x, ic.y) |
+                (mx_encode2s(v[j + 2], v[j + 3], ic.z, ic.w) << 16);
   }
 }
 

@@ -110,11 +110,7 @@ __device__ __forceinline__ void unpack4(const uint2& v, float* f) {
 }
 
 __device__ __forceinline__ uint32_t encode4(const float* f, const float* inv) {
-  const __nv_fp8x2_storage_t c0 = __nv_cvt_float2_to_fp8x2(
-      make_float2(f[0] * inv[0], f[1] * inv[1]), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(
-      make_float2(f[2] * inv[2], f[3] * inv[3]), __NV_SATFINITE, __NV_E4M3);
-  return (uint32_t)c0 | ((uint32_t)c1 << 16);
+  return mx_encode2s(f[0], f[1], inv[0], inv[1]) | (mx_encode2s(f[2], f[3], inv[2], inv[3]) << 16);
 }
 
 // ------------------------------ both axes, TMA-fed persistent variant

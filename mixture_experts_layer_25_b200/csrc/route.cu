@@ -10,8 +10,10 @@
 //      assignments to the same expert (token order), and the block's
 //      per-expert histogram.  Router mode runs on the tensor cores when it
 //      can (E <= 128, E % 8 == 0, k <= 8, d % 64 == 0; blocks of 128 tokens):
-//      W_r is split exactly into three bf16 parts w0 + w1 + w2 and the logits
-//      are one K = 3d product [x|x|x] [w0;w1;w2] accumulated in fp32.  The
+//      W_r is split into two bf16 parts w0 + w1 (equal to W_r within
+//      2^-17 |W_r|, below the fp32 accumulation error of a length-d sum for
+//      d >= 32) and the logits are one K = 2d product [x|x] [w0;w1]
+//      accumulated in fp32.  The
 //      fallback (and given-mode) kernels use blocks of 32 tokens and fp32
 //      FMA.
 //   2. route_scan (one CTA): per-expert exclusive scan of the block
@@ -208,21 +210,17 @@ route_given_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
 }
 
 // ---------------------------------------------------------------------------
-// W_r [d, E] fp32 -> wsplit [3d, E] bf16 with w0 = bf16(W), w1 = bf16(W - w0),
-// w2 = bf16(W - w0 - w1): each difference is exact in fp32 and the last part
-// holds at most 8 significant bits, so w0 + w1 + w2 == W (normal range).
+// W_r [d, E] fp32 -> wsplit [2d, E] bf16 with w0 = bf16(W), w1 = bf16(W - w0):
+// the difference is exact in fp32 and w0 + w1 keeps 16 significant bits, so
+// |W - w0 - w1| <= 2^-17 |W| (normal range).
 __global__ void router_split_kernel(const float* __restrict__ Wr, int n,
                                     __nv_bfloat16* __restrict__ ws) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float w = Wr[i];
   const __nv_bfloat16 w0 = __float2bfloat16_rn(w);
-  const float r1 = w - __bfloat162float(w0);
-  const __nv_bfloat16 w1 = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(w1);
   ws[i] = w0;
-  ws[n + i] = w1;
-  ws[2 * n + i] = __float2bfloat16_rn(r2);
+  ws[n + i] = __float2bfloat16_rn(w - __bfloat162float(w0));
 }
 
 // ---------------------------------------------------------------------------
@@ -353,7 +351,7 @@ extern "C" size_t moe_route_workspace_size(int T, int d, int E) {
   const size_t simt = round_up((size_t)((T + kTok - 1) / kTok) * E * sizeof(int32_t), 256);
   // tensor-core router: histograms of 128-token blocks + the split W_r
   const size_t tc = round_up((size_t)((T + 127) / 128) * E * sizeof(int32_t), 256) +
-                    round_up((size_t)3 * d * E * sizeof(__nv_bfloat16), 256);
+                    round_up((size_t)2 * d * E * sizeof(__nv_bfloat16), 256);
   return simt > tc ? simt : tc;
 }
 

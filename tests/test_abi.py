@@ -41,8 +41,8 @@ def test_host_size_queries():
     lib = _lib.lib()
     # given routing (d = 0): 32-token block histograms
     assert lib.moe_route_workspace_size(16384, 0, 128) == 512 * 128 * 4
-    # tensor-core router: 128-token block histograms + W_r split in 3 bf16 parts
-    assert lib.moe_route_workspace_size(16384, 2048, 128) == 128 * 128 * 4 + 3 * 2048 * 128 * 2
+    # tensor-core router: 128-token block histograms + W_r split in 2 bf16 parts
+    assert lib.moe_route_workspace_size(16384, 2048, 128) == 128 * 128 * 4 + 2 * 2048 * 128 * 2
     assert lib.moe_route_workspace_size(0, 2048, 128) == 0
     assert lib.moe_unpermute_sum_workspace_size(2048, 128) == 2048 * 128 * 4
     d = _lib.LayerDesc(16384, 2048, 128, 4, 1024, 128, 0, 0)
