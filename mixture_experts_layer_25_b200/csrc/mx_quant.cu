@@ -234,99 +234,6 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
   }
 }
 
-// ------------------------- both axes, 32 x 32 blocks (weights, in-step)
-// Persistent CTAs of 8 warps walk 128 x 128 tiles, each arriving by TMA in
-// two 64-column boxes with the 128-byte swizzle (so that the 32 lanes of a
-// warp, one row each, read a block's row segments without bank conflicts),
-// double-buffered.  Warp w quantises two of the tile's sixteen 32 x 32
-// blocks both ways with mx_quant_block32_regs; codes leave straight from
-// registers (32 bytes per lane and block), the tile's scale bytes as whole
-// words of the tensor-core layouts.  Rows at and beyond nrows keep their
-// codes and row scales; a 32-row block wholly beyond it gets column scale 0.
-constexpr int kDual2Warps = 8;
-
-__global__ void __launch_bounds__(32 * kDual2Warps, 2)
-mx_quant_dual_kernel(const __grid_constant__ CUtensorMap tin, int rows, int cols,
-                     const int32_t* __restrict__ nrows_dev, uint8_t* __restrict__ codes_r,
-                     uint8_t* __restrict__ scales_r, uint8_t* __restrict__ codes_c,
-                     uint8_t* __restrict__ scales_c) {
-  using namespace sm100;
-  extern __shared__ __align__(1024) uint8_t qsm2[];
-  __shared__ __align__(8) uint64_t full[2];
-  __shared__ volatile int abort_flag;
-  __shared__ __align__(4) uint8_t srow_s[kDualTile][4];
-  __shared__ __align__(4) uint8_t scol_s[kDualTile][4];
-  __shared__ __align__(16) float qinv_s[kDual2Warps][32];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qsm2) + 1023) &
-                                             ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nrows = nrows_dev ? min(*nrows_dev, rows) : rows;
-  const int tiles_r = (nrows + kDualTile - 1) / kDualTile, tiles_c = cols / kDualTile;
-  const int ntiles = tiles_r * tiles_c;
-  if (tid == 0) {
-    abort_flag = 0;
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  auto issue = [&](int tile, int buf) {
-    const int tr = tile / tiles_c, tc = tile % tiles_c;
-    uint8_t* dst = smem + buf * kDualTileBytes;
-    mbar_arrive_expect_tx(&full[buf], kDualTileBytes);
-    tma_load_2d(dst, &tin, &full[buf], tc * kDualTile, tr * kDualTile);
-    tma_load_2d(dst + kDualTileBytes / 2, &tin, &full[buf], tc * kDualTile + 64, tr * kDualTile);
-  };
-  if (tid == 0 && (int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
-  uint32_t phase = 0;
-  int it = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int buf = it & 1;
-    if (tid == 0 && tile + (int)gridDim.x < ntiles) issue(tile + gridDim.x, buf ^ 1);
-    if (!mbar_wait(&full[buf], (phase >> buf) & 1, &abort_flag, nullptr, 2000000000ull)) break;
-    phase ^= 1u << buf;
-    const int tr = tile / tiles_c, tc = tile % tiles_c;
-    const int r0 = tr * kDualTile, c0 = tc * kDualTile;
-    const uint8_t* t = smem + buf * kDualTileBytes;
-    const int rb = warp >> 1, row = rb * 32 + lane;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = (warp & 1) * 2 + h;
-      const uint8_t* rowp = t + (cb >> 1) * (kDualTileBytes / 2) + row * 128;
-      float v[32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = (cb & 1) * 4 + q;
-        unpack8(*reinterpret_cast<const uint4*>(rowp + ((j ^ (row & 7)) << 4)), v + 8 * q);
-      }
-      uint32_t cr[8], cc[8], br, bc;
-      mx_quant_block32_regs(v, cr, cc, br, bc, qinv_s[warp]);
-      if (r0 + row < nrows) {
-        const size_t off = (size_t)(r0 + row) * cols + c0 + cb * 32;
-        uint4* qr = reinterpret_cast<uint4*>(codes_r + off);
-        uint4* qc = reinterpret_cast<uint4*>(codes_c + off);
-        qr[0] = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-        qr[1] = make_uint4(cr[4], cr[5], cr[6], cr[7]);
-        qc[0] = make_uint4(cc[0], cc[1], cc[2], cc[3]);
-        qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
-      }
-      srow_s[row][cb] = (uint8_t)br;
-      scol_s[cb * 32 + lane][rb] = r0 + rb * 32 < nrows ? (uint8_t)bc : (uint8_t)0;
-    }
-    __syncthreads();               // buffer `buf` read; the tile's scale bytes complete
-    if (tid < kDualTile) {
-      if (r0 + tid < nrows)
-        *reinterpret_cast<uint32_t*>(scales_r + mx_sf_offset(r0 + tid, c0 >> 5, cols / 128)) =
-            *reinterpret_cast<const uint32_t*>(srow_s[tid]);
-    } else {
-      const int c = tid - kDualTile;
-      *reinterpret_cast<uint32_t*>(scales_c + mx_sf_offset(c0 + c, r0 >> 5, rows / 128)) =
-          *reinterpret_cast<const uint32_t*>(scol_s[c]);
-    }
-    __syncthreads();               // scale staging and buffer `buf` free for reuse
-  }
-}
-
 // -------------------------------------------- permute fused with MX codes
 constexpr int kMaxK = 16;
 constexpr int kWarps = 8;
@@ -429,7 +336,8 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
                          uint8_t* __restrict__ XqT, uint8_t* __restrict__ XsT, GateRows gr) {
   extern __shared__ __align__(16) uint8_t gsm[];          // 2 x kGBufBytes
   __shared__ int tok_s[2][kGTile];
-  __shared__ float gate_s[kGTile];
+  __shared__ float gate_s[kGTile];           // gates of the rows of row tile gate_rt
+  __shared__ int grp_s;
   __shared__ __align__(4) uint8_t srow_s[kGTile][4];      // row scale bytes, 4 K blocks
   __shared__ __align__(4) uint8_t scol_s[kGTile][4];      // column scale bytes, 4 row blocks
   __shared__ __align__(16) float qinv_s[kGatherWarps][32];  // each warp's column scales
@@ -455,33 +363,40 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
     cp_async_commit();
   };
 
-  int it = 0;
-  if ((int)blockIdx.x < nitems) issue(blockIdx.x, 0);
-  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
+  // each CTA takes a contiguous run of items, so that the gates of a row
+  // tile are looked up once for its d / 128 column tiles
+  const int per = (nitems + gridDim.x - 1) / gridDim.x;
+  const int i0 = min((int)blockIdx.x * per, nitems), i1 = min(i0 + per, nitems);
+  int it = 0, gate_rt = -1;
+  if (i0 < i1) issue(i0, 0);
+  for (int item = i0; item < i1; ++item, ++it) {
     const int buf = it & 1;
-    const int nxt = item + gridDim.x;
-    if (nxt < nitems) issue(nxt, buf ^ 1);
+    if (item + 1 < i1) issue(item + 1, buf ^ 1);
     else cp_async_commit();                    // keep the group count uniform
     cp_async_wait<1>();                        // this thread's copies of `item` landed
     __syncthreads();                           // everyone's have
     const int rt = item / ctiles, ct = item - rt * ctiles;
     const int r0 = rt * kGTile, c0 = ct * kGTile;
-    if (gr.gates && tid < kGTile) {
-      // the item's group (largest e with poff[e] <= r0), then each row's
-      // token's slot of that expert
-      int lo = 0, hi = gr.E - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(gr.poff + mid) <= r0) lo = mid; else hi = mid - 1;
+    if (gr.gates && rt != gate_rt) {
+      // the row tile's group: the one non-empty e with poff[e] <= r0 < poff[e+1]
+      for (int e = tid; e < gr.E; e += blockDim.x)
+        if (__ldg(gr.poff + e) <= r0 && r0 < __ldg(gr.poff + e + 1)) grp_s = e;
+      __syncthreads();
+      if (tid < kGTile) {
+        // each row's token's slot of that expert
+        const int t = tok_s[buf][tid], e = grp_s;
+        float g = 0.f;
+        if (t >= 0) {
+          const int32_t* ti = gr.topk + (size_t)t * gr.k;
+#pragma unroll 4
+          for (int j = 0; j < gr.k; ++j)
+            if (__ldg(ti + j) == e) g = __ldg(gr.gates + (size_t)t * gr.k + j);
+        }
+        gate_s[tid] = g;
       }
-      const int t = tok_s[buf][tid];
-      float g = 0.f;
-      if (t >= 0)
-        for (int j = 0; j < gr.k; ++j)
-          if (__ldg(gr.topk + (size_t)t * gr.k + j) == lo) g = __ldg(gr.gates + (size_t)t * gr.k + j);
-      gate_s[tid] = g;
+      __syncthreads();
+      gate_rt = rt;
     }
-    if (gr.gates) __syncthreads();
     const uint8_t* tile = gsm + buf * kGBufBytes;
     const int rb = warp >> 1;                  // this warp's 32-row block
     const int row = rb * 32 + lane;
@@ -635,26 +550,6 @@ extern "C" moe_status_t mx_quantize_dual(const void* in, int rows, int cols,
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
-#ifndef MOE_QDUAL_V1
-  // 32 x 32 blocks (mx_quant_dual_kernel): 128-byte swizzled boxes
-  if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(in), dims, strides, box, estr,
-         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-    set_error("mx_quantize_dual: tensor map encoding failed");
-    return MOE_ERR_CUDA;
-  }
-  {
-    const size_t smem = 1024 + 2 * (size_t)kDualTileBytes;
-    MOE_TRY(set_smem_limit(reinterpret_cast<const void*>(mx_quant_dual_kernel), smem,
-                           "mx_quantize_dual"));
-    const long long ntiles = (long long)(rows / 128) * (cols / 128);
-    const int grid = (int)std::min<long long>(ntiles, 2LL * num_sms());
-    mx_quant_dual_kernel<<<grid, 32 * kDual2Warps, smem, s>>>(m, rows, cols, nrows_dev, codes_rows,
-                                                              scales_rows, codes_cols, scales_cols);
-    MOE_CHECK_LAUNCH("mx_quantize_dual");
-    return MOE_OK;
-  }
-#endif
   if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(in), dims, strides, box, estr,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
