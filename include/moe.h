@@ -294,7 +294,7 @@ MOE_API moe_status_t moe_permute_mx(const void* x, const int32_t* src, const int
  * dYs, K = d: GEMM2 dgrad) and down the rows (dYTq / dYTs, K = A_pad_max:
  * GEMM2 weight gradient); bit-identical to mx_quantize_dual of the dY that
  * moe_combine_bwd writes.  Rows from poff[E] on are not touched.  d % 128
- * == 0, k <= 16. */
+ * == 0, k <= 16, E <= 1024. */
 MOE_API moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
                                         const int32_t* topk_idx, const int32_t* src,
                                         const int32_t* poff, int T, int k, int d, int E,

@@ -196,7 +196,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z sigmoid(z); the quotient is the 2-ulp fast division (the
+// correctly rounded one costs more than the rest of the epilogue)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 template <bool MX>
 __device__ __forceinline__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
@@ -785,7 +787,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                 hv[2 * i] = f2.x;
                 hv[2 * i + 1] = f2.y;
               }
-              mx_quant_block32(hv, stg, stg + 1024, p.q_sr, y0 + r, n0 + c, p.q_row_kchunks,
+              mx_quant_block32(hv, hbits, stg, stg + 1024, p.q_sr, y0 + r, n0 + c, p.q_row_kchunks,
                                p.q_sc, y0, p.q_col_kchunks, qinv_s[MX ? ew : 0]);
             }
           }
@@ -868,7 +870,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int i = 0; i < 8; ++i) {
               const float dh = __uint_as_float(v[8 * j + i]);
               const float z = f1[i];
-              const float sg = 1.0f / (1.0f + __expf(-z));
+              const float sg = __fdividef(1.0f, 1.0f + __expf(-z));
               o1[i] = dh * f3[i] * sg * (1.0f + z * (1.0f - sg));
               o3[i] = dh * z * sg;
             }
@@ -896,7 +898,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
                 for (int j = 0; j < 4; ++j) unpack8(k4[j], dv + 8 * j);
                 uint8_t* box = o == 0 ? b1 : b3;
-                mx_quant_block32(dv, box, box + 1024, p.q_sr, y0 + r, (o ? p.half : 0) + n0 + c,
+                mx_quant_block32(dv, reinterpret_cast<const uint32_t*>(k4), box, box + 1024, p.q_sr, y0 + r, (o ? p.half : 0) + n0 + c,
                                  p.q_row_kchunks, p.q_sc, y0, p.q_col_kchunks, qinv_s[MX ? ew : 0]);
               }
             }

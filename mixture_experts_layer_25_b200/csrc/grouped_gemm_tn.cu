@@ -103,7 +103,8 @@ __device__ __forceinline__ uint32_t idesc_bf16(bool a_mn, int n) {
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z sigmoid(z) with the 2-ulp fast division (as the rows-mode kernels)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 struct Tile {
   int e, fb;

@@ -312,6 +312,7 @@ constexpr int kGatherWarps = 8;
 constexpr int kGTile = 128;                     // rows and columns of an item
 constexpr int kGRowBytes = kGTile * 2 + 16;     // padded shared-memory row (bank spread)
 constexpr int kGBufBytes = kGTile * kGRowBytes;
+constexpr int kGMaxE = 1024;                    // experts the gated mode accepts
 
 struct GateRows {
   const float* gates;     // [T, k], null: no gate
@@ -336,8 +337,8 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
                          uint8_t* __restrict__ XqT, uint8_t* __restrict__ XsT, GateRows gr) {
   extern __shared__ __align__(16) uint8_t gsm[];          // 2 x kGBufBytes
   __shared__ int tok_s[2][kGTile];
-  __shared__ float gate_s[kGTile];           // gates of the rows of row tile gate_rt
-  __shared__ int grp_s;
+  __shared__ float gate_s[2][kGTile];        // gates of the rows of the item in each buffer
+  __shared__ int poff_s[kGMaxE + 1];         // group offsets (gated mode)
   __shared__ __align__(4) uint8_t srow_s[kGTile][4];      // row scale bytes, 4 K blocks
   __shared__ __align__(4) uint8_t scol_s[kGTile][4];      // column scale bytes, 4 row blocks
   __shared__ __align__(16) float qinv_s[kGatherWarps][32];  // each warp's column scales
@@ -363,57 +364,87 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
     cp_async_commit();
   };
 
-  // each CTA takes a contiguous run of items, so that the gates of a row
-  // tile are looked up once for its d / 128 column tiles
-  const int per = (nitems + gridDim.x - 1) / gridDim.x;
-  const int i0 = min((int)blockIdx.x * per, nitems), i1 = min(i0 + per, nitems);
-  int it = 0, gate_rt = -1;
-  if (i0 < i1) issue(i0, 0);
-  for (int item = i0; item < i1; ++item, ++it) {
+  // the gate of row `row` of the row tile at r0, whose token is t: the
+  // tile's group is the largest e with poff[e] <= r0 (a non-empty one, as
+  // r0 < poff[E]), the gate the token's slot of that expert
+  auto group_of = [&](int r0) {
+    int lo = 0, hi = gr.E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (poff_s[mid] <= r0) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
+  auto gate_of = [&](int e, int t) {
+    float g = 0.f;
+    if (t >= 0)
+      for (int j = 0; j < gr.k; ++j)
+        if (__ldg(gr.topk + (size_t)t * gr.k + j) == e) g = __ldg(gr.gates + (size_t)t * gr.k + j);
+    return g;
+  };
+  if (gr.gates)
+    for (int e = tid; e <= gr.E; e += blockDim.x) poff_s[e] = __ldg(gr.poff + e);
+
+  int it = 0;
+  if ((int)blockIdx.x < nitems) issue(blockIdx.x, 0);
+  for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++it) {
     const int buf = it & 1;
-    if (item + 1 < i1) issue(item + 1, buf ^ 1);
+    const int nxt = item + gridDim.x;
+    if (nxt < nitems) issue(nxt, buf ^ 1);
     else cp_async_commit();                    // keep the group count uniform
     cp_async_wait<1>();                        // this thread's copies of `item` landed
     __syncthreads();                           // everyone's have
     const int rt = item / ctiles, ct = item - rt * ctiles;
     const int r0 = rt * kGTile, c0 = ct * kGTile;
-    if (gr.gates && rt != gate_rt) {
-      // the row tile's group: the one non-empty e with poff[e] <= r0 < poff[e+1]
-      for (int e = tid; e < gr.E; e += blockDim.x)
-        if (__ldg(gr.poff + e) <= r0 && r0 < __ldg(gr.poff + e + 1)) grp_s = e;
-      __syncthreads();
-      if (tid < kGTile) {
-        // each row's token's slot of that expert
-        const int t = tok_s[buf][tid], e = grp_s;
-        float g = 0.f;
-        if (t >= 0) {
-          const int32_t* ti = gr.topk + (size_t)t * gr.k;
-#pragma unroll 4
-          for (int j = 0; j < gr.k; ++j)
-            if (__ldg(ti + j) == e) g = __ldg(gr.gates + (size_t)t * gr.k + j);
-        }
-        gate_s[tid] = g;
+    // gated mode: the first item's gates now; every later item's are
+    // prefetched (k <= 4: topk and gate words loaded here, used after the
+    // quantisation below) and written to gate_s one item ahead
+    int pe[4] = {-1, -1, -1, -1};
+    float pg[4] = {0.f, 0.f, 0.f, 0.f};
+    if (gr.gates) {
+      if (it == 0) {
+        if (tid < kGTile) gate_s[buf][tid] = gate_of(group_of(r0), tok_s[buf][tid]);
+        __syncthreads();
       }
-      __syncthreads();
-      gate_rt = rt;
+      if (tid < kGTile && nxt < nitems && gr.k <= 4) {
+        const int tn = tok_s[buf ^ 1][tid];
+        if (tn >= 0) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < gr.k) {
+              pe[j] = __ldg(gr.topk + (size_t)tn * gr.k + j);
+              pg[j] = __ldg(gr.gates + (size_t)tn * gr.k + j);
+            }
+          }
+        }
+      }
     }
     const uint8_t* tile = gsm + buf * kGBufBytes;
     const int rb = warp >> 1;                  // this warp's 32-row block
     const int row = rb * 32 + lane;
-    const float g = gr.gates ? gate_s[row] : 1.f;
+    const float g = gr.gates ? gate_s[buf][row] : 1.f;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int cb = (warp & 1) * 2 + h;       // its 32-column block
       float v[32];
+      uint4 w[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        unpack8(*reinterpret_cast<const uint4*>(tile + row * kGRowBytes + cb * 64 + j * 16), v + 8 * j);
+      for (int j = 0; j < 4; ++j) {
+        w[j] = *reinterpret_cast<const uint4*>(tile + row * kGRowBytes + cb * 64 + j * 16);
+        unpack8(w[j], v + 8 * j);
+      }
       if (gr.gates) {
+        // the bf16 product of the gate and the row, as the unfused dY holds it
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(g * v[j]));
+        for (int j = 0; j < 32; ++j) v[j] *= g;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          w[j] = pack8(v + 8 * j);
+          unpack8(w[j], v + 8 * j);
+        }
       }
       uint32_t cr[8], cc[8], br, bc;
-      mx_quant_block32_regs(v, cr, cc, br, bc, qinv_s[warp]);
+      mx_quant_block32_regs(v, reinterpret_cast<const uint32_t*>(w), cr, cc, br, bc, qinv_s[warp]);
       const size_t off = (size_t)(r0 + row) * d + c0 + cb * 32;
       uint4* qr = reinterpret_cast<uint4*>(Xq + off);
       uint4* qc = reinterpret_cast<uint4*>(XqT + off);
@@ -423,6 +454,18 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
       qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
       srow_s[row][cb] = (uint8_t)br;
       scol_s[cb * 32 + lane][rb] = (uint8_t)bc;
+    }
+    if (gr.gates && tid < kGTile && nxt < nitems) {
+      const int rn = (nxt / ctiles) * kGTile;
+      const int e = group_of(rn);
+      float gn = 0.f;
+      if (gr.k <= 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) gn = pe[j] == e ? pg[j] : gn;
+      } else {
+        gn = gate_of(e, tok_s[buf ^ 1][tid]);
+      }
+      gate_s[buf ^ 1][tid] = gn;
     }
     __syncthreads();                           // buffer `buf` and the scale bytes are complete
     // one word per row (its 4 K blocks of this item) and per column (its 4
@@ -471,8 +514,8 @@ extern "C" moe_status_t moe_combine_bwd_mx(const void* dout, const float* gates,
                                            int A_pad_max, uint8_t* dYq, uint8_t* dYs,
                                            uint8_t* dYTq, uint8_t* dYTs, moe_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  MOE_CHECK_ARG(T > 0 && E > 0 && k > 0 && k <= 16 && d > 0 && d % 128 == 0,
-                "moe_combine_bwd_mx: d %% 128, 0 < k <= 16");
+  MOE_CHECK_ARG(T > 0 && E > 0 && E <= kGMaxE && k > 0 && k <= 16 && d > 0 && d % 128 == 0,
+                "moe_combine_bwd_mx: d %% 128, 0 < k <= 16, E <= 1024");
   MOE_CHECK_ARG(A_pad_max > 0 && A_pad_max % 128 == 0, "moe_combine_bwd_mx: A_pad_max %% 128");
   MOE_CHECK_ARG(dout && gates && topk_idx && src && poff && dYq && dYs && dYTq && dYTs,
                 "moe_combine_bwd_mx: null pointer");
