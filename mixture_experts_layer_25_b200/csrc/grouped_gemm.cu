@@ -241,6 +241,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr int ACC_BUFS = MX ? 1 : 2;
   constexpr int SF_COL0 = 256 * ACC_BUFS;        // TMEM column of the first scale stage
   constexpr uint32_t TMEM_COLS = MX ? 512 : 512;
+  // MXFP8 SwiGLU backward: bf16 copy of the accumulator (128 columns)
+  constexpr int PARK_COL = 384;
+  static_assert(!MX || SF_COL0 + 12 * Cfg::STAGES <= PARK_COL, "parked dh overlaps the scales");
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + (MX ? SFA_BYTES + SFB_BYTES : 0);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -649,8 +652,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       // (the SwiGLU backward keeps the per-chunk path: with its whole slice
       // in registers it spills, measured 2.3x slower)
       constexpr bool EARLY = MX && (EPI == EPI_STORE || EPI == EPI_SWIGLU);
+      // PARK (MXFP8 SwiGLU backward, whose working set leaves no room for
+      // the slice in registers): dh is the bf16 output of GEMM2's dgrad, so
+      // the slice is rounded to bf16 pairs and parked in TMEM columns the
+      // MMA does not use (PARK_COL + 64 hc + [0, 64), past the accumulator
+      // and the scale stages); the accumulator is handed back at once and
+      // each chunk reads its 16 packed columns from the parked copy
+      constexpr bool PARK = MX && EPI == EPI_SWIGLU_BWD;
       constexpr int NV = EARLY ? 128 : 32;
       uint32_t av[NV];
+      const uint32_t park = tmem_base + ((uint32_t)(q * 32) << 16) + PARK_COL + hc * 64;
+      if constexpr (PARK) {
+        if (!empty) {
+#pragma unroll 1
+          for (int i = 0; i < 4; ++i) {
+            tmem_ld32(tbase + hc * (BN / 2) + 32 * i, av);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+              pk[m] = bf16x2_bits(__uint_as_float(av[2 * m]), __uint_as_float(av[2 * m + 1]));
+            tmem_st16(park + 16 * i, pk);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      }
       if constexpr (EARLY) {
         if (!empty) {
 #pragma unroll
@@ -847,8 +876,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             in_pending |= 1u << (pr ^ 1);
           }
           uint32_t* v = av;
-          tmem_ld32(tbase + hc * (BN / 2) + c, v);
-          tmem_wait_ld();
+          if constexpr (PARK) {
+            // this chunk's dh: 16 parked bf16 pairs -> 32 fp32 bit patterns
+            uint32_t pk[16];
+            if (!empty) {
+              tmem_ld16(park + 16 * ci, pk);
+              tmem_wait_ld();
+            } else {
+#pragma unroll
+              for (int m = 0; m < 16; ++m) pk[m] = 0u;
+            }
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+              v[2 * m] = pk[m] << 16;
+              v[2 * m + 1] = pk[m] & 0xffff0000u;
+            }
+          } else {
+            tmem_ld32(tbase + hc * (BN / 2) + c, v);
+            tmem_wait_ld();
+          }
           int got = 1;
           if (lane == 0)
             got = mbar_wait(&in_bar[ew][pr], (in_phase >> pr) & 1, &abort_flag, p.status,
@@ -1050,7 +1096,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         named_bar_sync(1, 256);                  // shared memory is reused by the next tile
       }
-      if constexpr (!EARLY) {
+      if constexpr (!EARLY && !PARK) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);

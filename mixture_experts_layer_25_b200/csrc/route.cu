@@ -227,6 +227,7 @@ __global__ void router_split_kernel(const float* __restrict__ Wr, int n,
 // One CTA: hist[b][e] -> exclusive offset of block b inside expert e;
 // counts, offsets, poff.
 constexpr int kScanThreads = 1024;
+constexpr int kScanBatch = 8;
 
 __global__ void __launch_bounds__(kScanThreads)
 route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
@@ -240,12 +241,19 @@ route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
   int* tot = sm + G * E;                // [E]
   const int chunk = (nblk + G - 1) / G;
 
+  // the column of a (group, expert) work item is read kScanBatch blocks at
+  // a time, all loads of a batch in flight together
   for (int w = tid; w < G * E; w += kScanThreads) {
     const int g = w / E, e = w % E;
     const int b0 = g * chunk, b1 = min(nblk, b0 + chunk);
     int s = 0;
-#pragma unroll 4
-    for (int b = b0; b < b1; ++b) s += hist[(size_t)b * E + e];
+    for (int b = b0; b < b1; b += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) v[i] = b + i < b1 ? hist[(size_t)(b + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) s += v[i];
+    }
     part[g * E + e] = s;
   }
   __syncthreads();
@@ -264,11 +272,15 @@ route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
     const int g = w / E, e = w % E;
     const int b0 = g * chunk, b1 = min(nblk, b0 + chunk);
     int run = part[g * E + e];
-    for (int b = b0; b < b1; ++b) {
-      const size_t o = (size_t)b * E + e;
-      const int v = hist[o];
-      hist[o] = run;
-      run += v;
+    for (int b = b0; b < b1; b += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) v[i] = b + i < b1 ? hist[(size_t)(b + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kScanBatch; ++i) {
+        if (b + i < b1) hist[(size_t)(b + i) * E + e] = run;
+        run += v[i];
+      }
     }
   }
   // exclusive scans over experts (serial per thread-chunk, then across chunks)

@@ -362,9 +362,11 @@ def layer_backward(ctx, dout):
         dh[a:b] = gemm2_dgrad(dYe, W2[e], mx)
         dW2[e] = gemm2_wgrad(he, dYe, mx)
         if mx:
+            # an MXFP8 GEMM accumulates in fp32 and outputs bf16, dh included;
             # the saved activations enter the backward at their stored (bf16)
             # precision, and dA is stored in bf16 before it is quantised, so
             # the quantised dA operands are the device's
+            dh[a:b] = round_bf16(dh[a:b])
             g1, g3 = swiglu_backward(dh[a:b], round_bf16(H1[a:b]), round_bf16(H3[a:b]))
             dA1[a:b], dA3[a:b] = round_bf16(g1), round_bf16(g3)
         else:

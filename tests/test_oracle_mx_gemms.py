@@ -199,7 +199,7 @@ def test_mx_layer_every_gemm_against_brute_force_quantisation():
     """Forward and backward of a tiny MX layer (router mode, ragged groups
     padded to 32 rows): each GEMM output against the brute-force GEMM of
     its own inputs, each operand quantised along that GEMM's K after the
-    device's bf16 rounding (h, dY, the saved H1/H3 and dA are stored in
+    device's bf16 rounding (h, dY, the saved H1/H3, dh and dA are stored in
     bf16 first; x and the weights are bf16 inputs)."""
     rng = np.random.default_rng(20)
     T, d, E, F, k = 72, 64, 4, 64, 2
@@ -233,7 +233,7 @@ def test_mx_layer_every_gemm_against_brute_force_quantisation():
         _close(ctx["Y"][a:b], _brute_gemm(he, W2[e]), "GEMM2")
         dYe = dY[a:b]
         dh = g["dh"][a:b]
-        _close(dh, _brute_gemm(dYe, W2[e].T), "GEMM2 dgrad")
+        _close(dh, _bf16(_brute_gemm(dYe, W2[e].T)), "GEMM2 dgrad (bf16 output)")
         _close(g["dW2"][e], _brute_gemm(he.T, dYe), "GEMM2 wgrad")
         # SwiGLU backward from the stored H1/H3, result stored in bf16
         z, u = _bf16(H1), _bf16(H3)
