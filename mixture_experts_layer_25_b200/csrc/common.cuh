@@ -129,29 +129,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// fp32 -> bf16 round to nearest even on the integer ALU, the bf16 in the
-// high 16 bits of the result: adding 0x7fff plus the lowest kept bit carries
-// into the kept bits exactly when the dropped half is above one half, or
-// equal to it with the kept value odd.  Identical to the conversion
-// instruction for every number and infinity; a NaN keeps its upper payload
-// with the quiet bit set.  For kernels whose conversion unit is their
-// bottleneck (the MXFP8 epilogues convert every element to E4M3 as well).
-__device__ __forceinline__ uint32_t bf16_rne_hi(float f) {
-  const uint32_t u = __float_as_uint(f);
-  const uint32_t r = u + 0x7fffu + ((u >> 16) & 1u);
-  return (u & 0x7fffffffu) > 0x7f800000u ? (u | 0x00400000u) : r;
-}
-
-// pack2 on the integer ALU (a in the low half)
-__device__ __forceinline__ uint32_t pack2_alu(float a, float b) {
-  return __byte_perm(bf16_rne_hi(a), bf16_rne_hi(b), 0x7632);
-}
-
-__device__ __forceinline__ uint4 pack8_alu(const float* f) {
-  return make_uint4(pack2_alu(f[0], f[1]), pack2_alu(f[2], f[3]), pack2_alu(f[4], f[5]),
-                    pack2_alu(f[6], f[7]));
-}
-
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"

@@ -189,13 +189,7 @@ __device__ __forceinline__ Tile decode(const Params& p, const int* poff_s, int t
   return t;
 }
 
-// fp32 pair -> bf16 pair (a low).  MXFP8 epilogues round on the integer ALU
-// (their conversion unit is busy with the E4M3 codes); BF16 ones convert.
-template <bool MX>
-__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
-  if constexpr (MX) return pack2_alu(a, b);
-  else return pack2(a, b);
-}
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) { return pack2(a, b); }
 
 // barrier over a subset of the CTA's warps (id 0 is __syncthreads')
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -677,7 +671,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             uint32_t pk[16];
 #pragma unroll
             for (int m = 0; m < 16; ++m)
-              pk[m] = bf16x2_bits<MX>(__uint_as_float(av[2 * m]), __uint_as_float(av[2 * m + 1]));
+              pk[m] = bf16x2_bits(__uint_as_float(av[2 * m]), __uint_as_float(av[2 * m + 1]));
             tmem_st16(park + 16 * i, pk);
           }
           tmem_wait_st();
@@ -749,10 +743,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               f[6] = fmaf(rs, c1.z, f[6]); f[7] = fmaf(rs, c1.w, f[7]);
             }
             uint4 w;
-            w.x = bf16x2_bits<MX>(f[0], f[1]);
-            w.y = bf16x2_bits<MX>(f[2], f[3]);
-            w.z = bf16x2_bits<MX>(f[4], f[5]);
-            w.w = bf16x2_bits<MX>(f[6], f[7]);
+            w.x = bf16x2_bits(f[0], f[1]);
+            w.y = bf16x2_bits(f[2], f[3]);
+            w.z = bf16x2_bits(f[4], f[5]);
+            w.w = bf16x2_bits(f[6], f[7]);
             *reinterpret_cast<uint4*>(buf + sw64(r, j)) = w;
           }
           fence_async_smem();
@@ -795,9 +789,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               const float g1 = __uint_as_float(g[8 * j + 2 * i + 1]);
               const float u0 = __uint_as_float(u[8 * j + 2 * i]);
               const float u1 = __uint_as_float(u[8 * j + 2 * i + 1]);
-              hp[i] = bf16x2_bits<MX>(silu_f(g0) * u0, silu_f(g1) * u1);
-              gp[i] = bf16x2_bits<MX>(g0, g1);
-              up[i] = bf16x2_bits<MX>(u0, u1);
+              hp[i] = bf16x2_bits(silu_f(g0) * u0, silu_f(g1) * u1);
+              gp[i] = bf16x2_bits(g0, g1);
+              up[i] = bf16x2_bits(u0, u1);
             }
             if constexpr (ONE_BOX) {
               hkeep[j] = hw; gkeep[j] = gw; ukeep[j] = uw;
@@ -926,7 +920,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               o1[i] = dh * f3[i] * sg * (1.0f + z * (1.0f - sg));
               o3[i] = dh * z * sg;
             }
-            const uint4 w1 = MX ? pack8_alu(o1) : pack8(o1), w3 = MX ? pack8_alu(o3) : pack8(o3);
+            const uint4 w1 = pack8(o1), w3 = pack8(o3);
             if constexpr (MX) {
               o1k[j] = w1;
               o3k[j] = w3;

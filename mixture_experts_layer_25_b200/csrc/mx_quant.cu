@@ -439,7 +439,7 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
         for (int j = 0; j < 32; ++j) v[j] *= g;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          w[j] = pack8_alu(v + 8 * j);
+          w[j] = pack8(v + 8 * j);
           unpack8(w[j], v + 8 * j);
         }
       }
