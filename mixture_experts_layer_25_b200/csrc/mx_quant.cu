@@ -119,7 +119,9 @@ __device__ __forceinline__ uint32_t encode4(const float* f, const float* inv) {
 // tile is quantised, so the bytes in flight do not depend on registers.
 // Warp w takes rows 16w..16w+15 of the tile (half of one 32-row MX column
 // block; warps 2b and 2b+1 combine their column maxima through shared
-// memory), lane L columns 4L..4L+3; both passes read shared memory.
+// memory), two rows per step with 16 lanes of 8 columns each (a 32-column
+// row block is 4 lanes).  The first pass writes the row codes and keeps the
+// raw rows in registers for the column codes of the second.
 constexpr int kDualTile = 128;
 constexpr int kDualTileBytes = kDualTile * kDualTile * 2;
 constexpr int kDualWarps = 8;
@@ -136,13 +138,14 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
   extern __shared__ __align__(128) uint8_t qsm[];
   __shared__ __align__(8) uint64_t full[2];
   __shared__ volatile int abort_flag;
-  __shared__ float camax[kDualWarps][kDualTile];   // per-warp column maxima
-  __shared__ uint32_t cbyte[4][kDualTile];         // column scale byte per 32-row block
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ __align__(16) float camax[kDualWarps][kDualTile];  // per-warp column maxima
+  __shared__ __align__(4) uint8_t srow_s[kDualTile][4];          // row scale bytes, 4 K blocks
+  __shared__ __align__(4) uint8_t scol_s[kDualTile][4];          // column scale bytes, 4 row blocks
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = nrows_dev ? min(*nrows_dev, rows) : rows;
   const int tiles_r = (nrows + kDualTile - 1) / kDualTile, tiles_c = cols / kDualTile;
   const int ntiles = tiles_r * tiles_c;
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     abort_flag = 0;
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
@@ -156,81 +159,90 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
     tma_load_2d(dst, &tin, &full[buf], tc * kDualTile, tr * kDualTile);
     tma_load_2d(dst + kDualTileBytes / 2, &tin, &full[buf], tc * kDualTile + 64, tr * kDualTile);
   };
-  if (threadIdx.x == 0 && (int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+  if (tid == 0 && (int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
+  // lane L: 16-byte chunk c = L % 16 (columns 8c..8c+7: box c / 8, slot c % 8)
+  // of row 2s + L / 16 of the warp's 16 rows, s = 0..7
+  const int c = lane & 15, hrow = lane >> 4;
   uint32_t phase = 0;   // bit b: parity of full[b]
   int it = 0;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int buf = it & 1;
-    if (threadIdx.x == 0 && tile + (int)gridDim.x < ntiles) issue(tile + gridDim.x, buf ^ 1);
+    if (tid == 0 && tile + (int)gridDim.x < ntiles) issue(tile + gridDim.x, buf ^ 1);
     if (!mbar_wait(&full[buf], (phase >> buf) & 1, &abort_flag, nullptr, 2000000000ull)) break;
     phase ^= 1u << buf;
     const int tr = tile / tiles_c, tc = tile % tiles_c;
-    const uint8_t* t = qsm + buf * kDualTileBytes;
-    // lane L: columns 4L..4L+3 of the tile: box L/16, 8-byte slot L%16 of a 128-byte row
-    const uint8_t* base = t + (lane >> 4) * (kDualTileBytes / 2) + (lane & 15) * 8;
-    const int rl0 = warp * 16;                         // first tile row of this warp
-    const int r0 = tr * kDualTile + rl0;
-    const int col = tc * kDualTile + lane * 4;
-    float amax[4] = {0, 0, 0, 0};
-    uint32_t rs[16];
+    const uint8_t* base = qsm + buf * kDualTileBytes + (c >> 3) * (kDualTileBytes / 2) + (c & 7) * 16;
+    const int rl0 = warp * 16;                          // first tile row of this warp
+    const int col = tc * kDualTile + 8 * c;
+    // pass 1: row scales and row codes; the raw rows stay in registers
+    uint4 raw[8];
+    float cm[8];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float f[4];
-      unpack4(*reinterpret_cast<const uint2*>(base + (rl0 + r) * 128), f);
+    for (int i = 0; i < 8; ++i) cm[i] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int rl = rl0 + 2 * s + hrow;
+      raw[s] = *reinterpret_cast<const uint4*>(base + rl * 128);
+      float f[8];
+      unpack8(raw[s], f);
       float ra = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        amax[i] = fmaxf(amax[i], fabsf(f[i]));
+      for (int i = 0; i < 8; ++i) {
+        cm[i] = fmaxf(cm[i], fabsf(f[i]));
         ra = fmaxf(ra, fabsf(f[i]));
       }
+      // a 32-column block is 4 lanes
       ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 1));
       ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 2));
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 4));
-      rs[r] = scale_byte(ra);
-      // the word of row r0+r for this tile's 4 column blocks: lanes 0, 8, 16, 24
-      const uint32_t b1 = __shfl_down_sync(0xffffffffu, rs[r], 8);
-      const uint32_t b2 = __shfl_down_sync(0xffffffffu, rs[r], 16);
-      const uint32_t b3 = __shfl_down_sync(0xffffffffu, rs[r], 24);
-      if (lane == 0 && r0 + r < nrows) {
-        const int mn = r0 + r;
-        const size_t off = ((size_t)(mn >> 7) * (cols / 128) + tc) * 512 + (mn & 31) * 16 +
-                           ((mn >> 5) & 3) * 4;
-        *reinterpret_cast<uint32_t*>(scales_r + off) = rs[r] | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      }
+      const uint32_t br = mx_scale_byte(ra);
+      const int row = tr * kDualTile + rl;
+      if (row < nrows)
+        *reinterpret_cast<uint2*>(codes_r + (size_t)row * cols + col) = mx_encode8(f, mx_inv_scale(br));
+      if ((c & 3) == 0) srow_s[rl][c >> 2] = (uint8_t)br;
     }
+    // column maxima: the warp's 16 rows, then the partner warp's 16
 #pragma unroll
-    for (int i = 0; i < 4; ++i) camax[warp][lane * 4 + i] = amax[i];
-    __syncthreads();
-    float inv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a = fmaxf(amax[i], camax[warp ^ 1][lane * 4 + i]);
-      const uint32_t b = scale_byte(a);
-      inv[i] = inv_scale(b);
-      if ((warp & 1) == 0) cbyte[warp >> 1][lane * 4 + i] = (r0 < nrows) ? b : 0u;
-    }
-    if (r0 < nrows) {
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float f[4];
-        unpack4(*reinterpret_cast<const uint2*>(base + (rl0 + r) * 128), f);
-        const float ir = inv_scale(rs[r]);
-        const float irr[4] = {ir, ir, ir, ir};
-        *reinterpret_cast<uint32_t*>(codes_c + (size_t)(r0 + r) * cols + col) = encode4(f, inv);
-        *reinterpret_cast<uint32_t*>(codes_r + (size_t)(r0 + r) * cols + col) = encode4(f, irr);
-      }
+    for (int i = 0; i < 8; ++i) cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 16));
+    if (hrow == 0) {
+      *reinterpret_cast<float4*>(&camax[warp][8 * c]) = make_float4(cm[0], cm[1], cm[2], cm[3]);
+      *reinterpret_cast<float4*>(&camax[warp][8 * c + 4]) = make_float4(cm[4], cm[5], cm[6], cm[7]);
     }
     __syncthreads();
-    // column scales: the tile's four 32-row blocks of one column form one word
-    if (threadIdx.x < kDualTile) {
-      const int c = threadIdx.x;
-      const uint32_t word = cbyte[0][c] | (cbyte[1][c] << 8) | (cbyte[2][c] << 16) | (cbyte[3][c] << 24);
-      const int mn = tc * kDualTile + c;
-      const size_t off = ((size_t)(mn >> 7) * (rows / 128) + tr) * 512 + (mn & 31) * 16 +
-                         ((mn >> 5) & 3) * 4;
-      *reinterpret_cast<uint32_t*>(scales_c + off) = word;
+    const bool blk_live = tr * kDualTile + (warp >> 1) * 32 < nrows;
+    float ic[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t b = mx_scale_byte(fmaxf(cm[i], camax[warp ^ 1][8 * c + i]));
+      ic[i] = mx_inv_scale(b);
+      if ((warp & 1) == 0 && hrow == 0) scol_s[8 * c + i][warp >> 1] = blk_live ? (uint8_t)b : 0;
     }
-    __syncthreads();   // buffer `buf`, camax and cbyte are free for the next tile
+    // pass 2: column codes from the registers
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const int row = tr * kDualTile + rl0 + 2 * s + hrow;
+      float f[8];
+      unpack8(raw[s], f);
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = mx_encode2s(f[2 * i], f[2 * i + 1], ic[2 * i], ic[2 * i + 1]);
+      if (row < nrows)
+        *reinterpret_cast<uint2*>(codes_c + (size_t)row * cols + col) =
+            make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+    }
+    __syncthreads();   // buffer `buf` read; the tile's scale bytes complete
+    // one word per row (its 4 K blocks of this tile) and per column (its 4
+    // row blocks): the tensor-core layout keeps the 4 bytes adjacent
+    if (tid < kDualTile) {
+      const int mn = tr * kDualTile + tid;
+      if (mn < nrows)
+        *reinterpret_cast<uint32_t*>(scales_r + mx_sf_offset(mn, tc * 4, cols / 128)) =
+            *reinterpret_cast<const uint32_t*>(srow_s[tid]);
+    } else {
+      const int cc = tid - kDualTile, mn = tc * kDualTile + cc;
+      *reinterpret_cast<uint32_t*>(scales_c + mx_sf_offset(mn, tr * 4, rows / 128)) =
+          *reinterpret_cast<const uint32_t*>(scol_s[cc]);
+    }
+    __syncthreads();   // camax and the scale staging are free for the next tile
   }
 }
 
