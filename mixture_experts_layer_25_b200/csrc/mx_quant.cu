@@ -113,6 +113,101 @@ __device__ __forceinline__ uint32_t encode4(const float* f, const float* inv) {
   return mx_encode2s(f[0], f[1], inv[0], inv[1]) | (mx_encode2s(f[2], f[3], inv[2], inv[3]) << 16);
 }
 
+// One 128 x 128 bf16 tile in shared memory quantised along both axes by 8
+// warps: warp w takes rows 16w..16w+15 (half of one 32-row MX column block;
+// warps 2b and 2b+1 combine their column maxima through `camax`), two rows
+// per step with 16 lanes of 8 columns each (a 32-column row block is 4
+// lanes).  The first pass writes the row codes (16 lanes x 8 bytes = one
+// 128-byte row segment) and keeps the raw rows in registers for the column
+// codes of the second; the scale bytes are gathered in shared memory and
+// leave as whole words of the tensor-core layouts.  `chunk(rl, c)` is the
+// shared address of 16-byte chunk c (columns 8c..8c+7) of tile row rl.
+// `gate` (nullable, by tile row): the rows are first replaced by the bf16
+// product gate x row.  Rows at and beyond `nrows` are not written (their
+// column blocks still see them; a 32-row block wholly beyond gets scale 0).
+// Contains three __syncthreads: every thread of the CTA calls it.
+template <class Chunk>
+__device__ __forceinline__ void mx_tile_both_axes(
+    Chunk chunk, const float* gate, int r0, int c0, int nrows, int cols, int col_kchunks,
+    uint8_t* __restrict__ codes_r, uint8_t* __restrict__ scales_r, uint8_t* __restrict__ codes_c,
+    uint8_t* __restrict__ scales_c, float (*camax)[128], uint8_t (*srow_s)[4],
+    uint8_t (*scol_s)[4]) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = lane & 15, hrow = lane >> 4;
+  const int rl0 = warp * 16;
+  const int col = c0 + 8 * c;
+  uint4 raw[8];
+  float cm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) cm[i] = 0.f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int rl = rl0 + 2 * s + hrow;
+    raw[s] = *reinterpret_cast<const uint4*>(chunk(rl, c));
+    float f[8];
+    unpack8(raw[s], f);
+    if (gate) {
+      const float g = gate[rl];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] *= g;
+      raw[s] = pack8(f);
+      unpack8(raw[s], f);
+    }
+    float ra = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cm[i] = fmaxf(cm[i], fabsf(f[i]));
+      ra = fmaxf(ra, fabsf(f[i]));
+    }
+    ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 1));
+    ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 2));
+    const uint32_t br = mx_scale_byte(ra);
+    const int row = r0 + rl;
+    if (row < nrows)
+      *reinterpret_cast<uint2*>(codes_r + (size_t)row * cols + col) = mx_encode8(f, mx_inv_scale(br));
+    if ((c & 3) == 0) srow_s[rl][c >> 2] = (uint8_t)br;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 16));
+  if (hrow == 0) {
+    *reinterpret_cast<float4*>(&camax[warp][8 * c]) = make_float4(cm[0], cm[1], cm[2], cm[3]);
+    *reinterpret_cast<float4*>(&camax[warp][8 * c + 4]) = make_float4(cm[4], cm[5], cm[6], cm[7]);
+  }
+  __syncthreads();
+  const bool blk_live = r0 + (warp >> 1) * 32 < nrows;
+  float ic[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t b = mx_scale_byte(fmaxf(cm[i], camax[warp ^ 1][8 * c + i]));
+    ic[i] = mx_inv_scale(b);
+    if ((warp & 1) == 0 && hrow == 0) scol_s[8 * c + i][warp >> 1] = blk_live ? (uint8_t)b : 0;
+  }
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int row = r0 + rl0 + 2 * s + hrow;
+    float f[8];
+    unpack8(raw[s], f);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = mx_encode2s(f[2 * i], f[2 * i + 1], ic[2 * i], ic[2 * i + 1]);
+    if (row < nrows)
+      *reinterpret_cast<uint2*>(codes_c + (size_t)row * cols + col) =
+          make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+  }
+  __syncthreads();   // the tile is read; the scale bytes are complete
+  if (tid < 128) {
+    const int mn = r0 + tid;
+    if (mn < nrows)
+      *reinterpret_cast<uint32_t*>(scales_r + mx_sf_offset(mn, c0 >> 5, cols / 128)) =
+          *reinterpret_cast<const uint32_t*>(srow_s[tid]);
+  } else if (tid < 256) {
+    const int cc = tid - 128;
+    *reinterpret_cast<uint32_t*>(scales_c + mx_sf_offset(c0 + cc, r0 >> 5, col_kchunks)) =
+        *reinterpret_cast<const uint32_t*>(scol_s[cc]);
+  }
+  __syncthreads();   // camax and the scale staging are free again
+}
+
 // ------------------------------ both axes, TMA-fed persistent variant
 // Persistent CTAs of 8 warps walk 128 x 128 tiles; each tile arrives in
 // shared memory by TMA (two 64-column boxes, no swizzle) while the previous
@@ -141,7 +236,7 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
   __shared__ __align__(16) float camax[kDualWarps][kDualTile];  // per-warp column maxima
   __shared__ __align__(4) uint8_t srow_s[kDualTile][4];          // row scale bytes, 4 K blocks
   __shared__ __align__(4) uint8_t scol_s[kDualTile][4];          // column scale bytes, 4 row blocks
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int nrows = nrows_dev ? min(*nrows_dev, rows) : rows;
   const int tiles_r = (nrows + kDualTile - 1) / kDualTile, tiles_c = cols / kDualTile;
   const int ntiles = tiles_r * tiles_c;
@@ -160,9 +255,6 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
     tma_load_2d(dst + kDualTileBytes / 2, &tin, &full[buf], tc * kDualTile + 64, tr * kDualTile);
   };
   if (tid == 0 && (int)blockIdx.x < ntiles) issue(blockIdx.x, 0);
-  // lane L: 16-byte chunk c = L % 16 (columns 8c..8c+7: box c / 8, slot c % 8)
-  // of row 2s + L / 16 of the warp's 16 rows, s = 0..7
-  const int c = lane & 15, hrow = lane >> 4;
   uint32_t phase = 0;   // bit b: parity of full[b]
   int it = 0;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
@@ -171,78 +263,13 @@ mx_quant_dual_tma_kernel(const __grid_constant__ CUtensorMap tin, int rows, int 
     if (!mbar_wait(&full[buf], (phase >> buf) & 1, &abort_flag, nullptr, 2000000000ull)) break;
     phase ^= 1u << buf;
     const int tr = tile / tiles_c, tc = tile % tiles_c;
-    const uint8_t* base = qsm + buf * kDualTileBytes + (c >> 3) * (kDualTileBytes / 2) + (c & 7) * 16;
-    const int rl0 = warp * 16;                          // first tile row of this warp
-    const int col = tc * kDualTile + 8 * c;
-    // pass 1: row scales and row codes; the raw rows stay in registers
-    uint4 raw[8];
-    float cm[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) cm[i] = 0.f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int rl = rl0 + 2 * s + hrow;
-      raw[s] = *reinterpret_cast<const uint4*>(base + rl * 128);
-      float f[8];
-      unpack8(raw[s], f);
-      float ra = 0.f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cm[i] = fmaxf(cm[i], fabsf(f[i]));
-        ra = fmaxf(ra, fabsf(f[i]));
-      }
-      // a 32-column block is 4 lanes
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 1));
-      ra = fmaxf(ra, __shfl_xor_sync(0xffffffffu, ra, 2));
-      const uint32_t br = mx_scale_byte(ra);
-      const int row = tr * kDualTile + rl;
-      if (row < nrows)
-        *reinterpret_cast<uint2*>(codes_r + (size_t)row * cols + col) = mx_encode8(f, mx_inv_scale(br));
-      if ((c & 3) == 0) srow_s[rl][c >> 2] = (uint8_t)br;
-    }
-    // column maxima: the warp's 16 rows, then the partner warp's 16
-#pragma unroll
-    for (int i = 0; i < 8; ++i) cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 16));
-    if (hrow == 0) {
-      *reinterpret_cast<float4*>(&camax[warp][8 * c]) = make_float4(cm[0], cm[1], cm[2], cm[3]);
-      *reinterpret_cast<float4*>(&camax[warp][8 * c + 4]) = make_float4(cm[4], cm[5], cm[6], cm[7]);
-    }
-    __syncthreads();
-    const bool blk_live = tr * kDualTile + (warp >> 1) * 32 < nrows;
-    float ic[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t b = mx_scale_byte(fmaxf(cm[i], camax[warp ^ 1][8 * c + i]));
-      ic[i] = mx_inv_scale(b);
-      if ((warp & 1) == 0 && hrow == 0) scol_s[8 * c + i][warp >> 1] = blk_live ? (uint8_t)b : 0;
-    }
-    // pass 2: column codes from the registers
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const int row = tr * kDualTile + rl0 + 2 * s + hrow;
-      float f[8];
-      unpack8(raw[s], f);
-      uint32_t w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) w[i] = mx_encode2s(f[2 * i], f[2 * i + 1], ic[2 * i], ic[2 * i + 1]);
-      if (row < nrows)
-        *reinterpret_cast<uint2*>(codes_c + (size_t)row * cols + col) =
-            make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-    }
-    __syncthreads();   // buffer `buf` read; the tile's scale bytes complete
-    // one word per row (its 4 K blocks of this tile) and per column (its 4
-    // row blocks): the tensor-core layout keeps the 4 bytes adjacent
-    if (tid < kDualTile) {
-      const int mn = tr * kDualTile + tid;
-      if (mn < nrows)
-        *reinterpret_cast<uint32_t*>(scales_r + mx_sf_offset(mn, tc * 4, cols / 128)) =
-            *reinterpret_cast<const uint32_t*>(srow_s[tid]);
-    } else {
-      const int cc = tid - kDualTile, mn = tc * kDualTile + cc;
-      *reinterpret_cast<uint32_t*>(scales_c + mx_sf_offset(mn, tr * 4, rows / 128)) =
-          *reinterpret_cast<const uint32_t*>(scol_s[cc]);
-    }
-    __syncthreads();   // camax and the scale staging are free for the next tile
+    // TMA boxes: 64 columns x 128 rows each, rows of 128 bytes
+    const uint8_t* t = qsm + buf * kDualTileBytes;
+    auto chunk = [t](int rl, int c) {
+      return t + (c >> 3) * (kDualTileBytes / 2) + rl * 128 + (c & 7) * 16;
+    };
+    mx_tile_both_axes(chunk, nullptr, tr * kDualTile, tc * kDualTile, nrows, cols, rows / 128,
+                      codes_r, scales_r, codes_c, scales_c, camax, srow_s, scol_s);
   }
 }
 
@@ -353,11 +380,11 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
   __shared__ int poff_s[kGMaxE + 1];         // group offsets (gated mode)
   __shared__ __align__(4) uint8_t srow_s[kGTile][4];      // row scale bytes, 4 K blocks
   __shared__ __align__(4) uint8_t scol_s[kGTile][4];      // column scale bytes, 4 row blocks
-  __shared__ __align__(16) float qinv_s[kGatherWarps][32];  // each warp's column scales
+  __shared__ __align__(16) float camax[kGatherWarps][kGTile];  // per-warp column maxima
   const int nrows = min(*poff_end, A_pad_max);
   const int ctiles = d / kGTile;
   const int nitems = (nrows / kGTile) * ctiles;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
 
   // gather the item's rows into buffer `buf` (16 threads per 256-byte row)
   auto issue = [&](int item, int buf) {
@@ -432,42 +459,12 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
       }
     }
     const uint8_t* tile = gsm + buf * kGBufBytes;
-    const int rb = warp >> 1;                  // this warp's 32-row block
-    const int row = rb * 32 + lane;
-    const float g = gr.gates ? gate_s[buf][row] : 1.f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int cb = (warp & 1) * 2 + h;       // its 32-column block
-      float v[32];
-      uint4 w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        w[j] = *reinterpret_cast<const uint4*>(tile + row * kGRowBytes + cb * 64 + j * 16);
-        unpack8(w[j], v + 8 * j);
-      }
-      if (gr.gates) {
-        // the bf16 product of the gate and the row, as the unfused dY holds it
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= g;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          w[j] = pack8(v + 8 * j);
-          unpack8(w[j], v + 8 * j);
-        }
-      }
-      uint32_t cr[8], cc[8], br, bc;
-      mx_quant_block32_regs(v, reinterpret_cast<const uint32_t*>(w), cr, cc, br, bc, qinv_s[warp]);
-      const size_t off = (size_t)(r0 + row) * d + c0 + cb * 32;
-      uint4* qr = reinterpret_cast<uint4*>(Xq + off);
-      uint4* qc = reinterpret_cast<uint4*>(XqT + off);
-      qr[0] = make_uint4(cr[0], cr[1], cr[2], cr[3]);
-      qr[1] = make_uint4(cr[4], cr[5], cr[6], cr[7]);
-      qc[0] = make_uint4(cc[0], cc[1], cc[2], cc[3]);
-      qc[1] = make_uint4(cc[4], cc[5], cc[6], cc[7]);
-      srow_s[row][cb] = (uint8_t)br;
-      scol_s[cb * 32 + lane][rb] = (uint8_t)bc;
-    }
+    auto chunk = [tile](int rl, int c) { return tile + rl * kGRowBytes + c * 16; };
+    // gated rows: bf16(g * dout row), as the unfused dY holds it
+    mx_tile_both_axes(chunk, gr.gates ? gate_s[buf] : nullptr, r0, c0, nrows, d, A_pad_max / 128,
+                      Xq, Xs, XqT, XsT, camax, srow_s, scol_s);
     if (gr.gates && tid < kGTile && nxt < nitems) {
+      // the next item's gates (read after the next item's first barrier)
       const int rn = (nxt / ctiles) * kGTile;
       const int e = group_of(rn);
       float gn = 0.f;
@@ -479,19 +476,6 @@ permute_mx_gather_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __r
       }
       gate_s[buf ^ 1][tid] = gn;
     }
-    __syncthreads();                           // buffer `buf` and the scale bytes are complete
-    // one word per row (its 4 K blocks of this item) and per column (its 4
-    // row blocks): the tensor-core layout keeps the 4 bytes adjacent
-    if (tid < kGTile) {
-      const int mn = r0 + tid;
-      *reinterpret_cast<uint32_t*>(Xs + mx_sf_offset(mn, c0 >> 5, d / 128)) =
-          *reinterpret_cast<const uint32_t*>(srow_s[tid]);
-    } else {
-      const int c = tid - kGTile, mn = c0 + c;
-      *reinterpret_cast<uint32_t*>(XsT + mx_sf_offset(mn, r0 >> 5, A_pad_max / 128)) =
-          *reinterpret_cast<const uint32_t*>(scol_s[c]);
-    }
-    __syncthreads();                           // scale staging reused by the next item
   }
   cp_async_wait<0>();
 }
