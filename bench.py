@@ -454,9 +454,15 @@ def run_ours(args):
         "route": T * d * bpe + d * E * 4 + T * E * 4 + T * k * 16,
         "permute": T * d * bpe + A * d * bpe,
         "combine": A * d * bpe + T * d * bpe,
-        "combine_bwd": T * d * bpe + 2 * A * d * bpe,
+        # the MXFP8 layer writes no bf16 dY here (its dY leaves as MX codes)
+        "combine_bwd": T * d * bpe + (1 if cfg.mx else 2) * A * d * bpe,
         "unpermute_sum": A * d * bpe + T * d * bpe,
     }
+    if cfg.mx:
+        # codes along both K axes (1 byte each) plus one scale byte per 32
+        wq = 3 * E * d * F
+        mem_bytes["quant_w_fwd"] = wq * bpe + 2 * wq + 2 * wq // 32
+        mem_bytes["quant_dgrad2"] = T * d * bpe + 2 * A * d + 2 * A * d // 32
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     mem = {n: {"GB_s": round(b / (stage_ms[n] * 1e-3) / 1e9, 1),
                "frac_of_hbm": round(b / (stage_ms[n] * 1e-3) / 1e9 / hbm, 3),
