@@ -126,48 +126,6 @@ enum Stage { S_ROUTE, S_PERMUTE, S_QW, S_GEMM1, S_QH, S_GEMM2, S_COMBINE, S_COMB
              S_QD2, S_DGRAD2, S_QW2, S_WGRAD2, S_QD1, S_DGRAD1, S_QW1, S_WGRAD1, S_UNPERMUTE,
              S_ROUTER_WGRAD };
 
-// A second stream per device for the MXFP8 forward's weight quantisation,
-// which needs nothing the routing or the dispatch produce (non-blocking,
-// created on first use and kept until the process exits; null if it cannot
-// be made, and the work then stays on the caller's stream).
-constexpr int kMaxSideDevices = 64;
-std::mutex g_side_mu;
-cudaStream_t g_side_stream[kMaxSideDevices] = {};
-
-cudaStream_t side_stream() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_side_mu);
-  if (!g_side_stream[dev] &&
-      cudaStreamCreateWithFlags(&g_side_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
-    g_side_stream[dev] = nullptr;
-  return g_side_stream[dev];
-}
-
-// fork / join of one call's side work
-struct Fork {
-  cudaEvent_t fork = nullptr, join = nullptr;
-  cudaStream_t side = nullptr;   // null: no split, everything on the caller's stream
-  ~Fork() {
-    if (fork) cudaEventDestroy(fork);   // released by the driver once the event has completed
-    if (join) cudaEventDestroy(join);
-  }
-  // the side stream, ordered after everything already on s (or s itself)
-  cudaStream_t open(cudaStream_t s) {
-    cudaStream_t q = side_stream();
-    if (q && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) == cudaSuccess &&
-        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) == cudaSuccess &&
-        cudaEventRecord(fork, s) == cudaSuccess && cudaStreamWaitEvent(q, fork, 0) == cudaSuccess)
-      side = q;
-    return side ? side : s;
-  }
-  // s waits for the side work
-  bool close(cudaStream_t s) {
-    return !side || (cudaEventRecord(join, side) == cudaSuccess &&
-                     cudaStreamWaitEvent(s, join, 0) == cudaSuccess);
-  }
-};
-
 }  // namespace
 
 extern "C" void moe_set_stage_events(void* const* events, int n) {
@@ -242,22 +200,6 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
       return MOE_ERR_CUDA;
     }
   }
-  // MXFP8: every weight along both K axes it is used with, one pass each
-  // (W1/W3 [E*d, F] down d for GEMM1 and along F for the GEMM1 dgrad; W2
-  // [E*F, d] down F for GEMM2 and along d for the GEMM2 dgrad), on the side
-  // stream so that it overlaps the routing and the dispatch
-  Fork qw;
-  if (mx) {
-    const size_t wq = (size_t)E * d * F;
-    cudaStream_t q = qw.open(s);
-    moe_stream_t qs = reinterpret_cast<moe_stream_t>(q);
-    mark(S_QW, false, q);
-    MOE_TRY(mx_quantize_dual(w->W1, E * d, F, nullptr, c.W13t_q, c.W13t_s, c.W13_q, c.W13_s, qs));
-    MOE_TRY(mx_quantize_dual(w->W3, E * d, F, nullptr, c.W13t_q + wq, c.W13t_s + wq / 32,
-                             c.W13_q + wq, c.W13_s + wq / 32, qs));
-    MOE_TRY(mx_quantize_dual(w->W2, E * F, d, nullptr, c.W2t_q, c.W2t_s, c.W2_q, c.W2_s, qs));
-    mark(S_QW, true, q);
-  }
   mark(S_ROUTE, false, s);
   MOE_TRY(moe_route(x, w->Wr, w->bias, T, d, E, k, L->align, L->route_mode, c.topk_idx, c.gates,
                     c.counts, c.offsets, c.poff, c.dst, c.src, A, c.logits, c.ws, c.ws_bytes,
@@ -301,10 +243,15 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
     MOE_TRY(moe_permute_mx(x, c.src, c.poff, T, d, E, A, c.Xp_q, c.Xp_s, c.XpT_q, c.XpT_s,
                            stream));
     mark(S_PERMUTE, true, s);
-    if (!qw.close(s)) {
-      set_error("moe_layer_fwd: joining the weight quantisation failed");
-      return MOE_ERR_CUDA;
-    }
+    // every weight along both K axes it is used with, in one pass each:
+    // W1/W3 [E*d, F] down d (fwd GEMM1) and along F (GEMM1 dgrad); W2
+    // [E*F, d] down F (fwd GEMM2) and along d (GEMM2 dgrad)
+    mark(S_QW, false, s);
+    MOE_TRY(mx_quantize_dual(w->W1, E * d, F, nullptr, c.W13t_q, c.W13t_s, W1q, W1s, stream));
+    MOE_TRY(mx_quantize_dual(w->W3, E * d, F, nullptr, c.W13t_q + wq, c.W13t_s + wq / 32, W3q,
+                             W3s, stream));
+    MOE_TRY(mx_quantize_dual(w->W2, E * F, d, nullptr, c.W2t_q, c.W2t_s, c.W2_q, c.W2_s, stream));
+    mark(S_QW, true, s);
     // GEMM1 + SwiGLU; its epilogue quantises h along F (fwd GEMM2) and down
     // the rows (GEMM2 wgrad) in place of storing it
     mark(S_GEMM1, false, s);
