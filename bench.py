@@ -480,15 +480,17 @@ def run_ours(args):
     if not args.no_e2e:
         xh = x.cpu().pin_memory(); dh = dout.cpu().pin_memory()
         oh = torch.empty_like(xh).pin_memory(); dxh = torch.empty_like(xh).pin_memory()
-        bufs = [torch.empty_like(x) for _ in range(4)]
-        for _ in range(2):
-            layer.step_host(xh, dh, oh, dxh, *bufs)
+        # two alternating sets of device buffers: a step's uploads run under
+        # the previous step's backward
+        bufs = [[torch.empty_like(x) for _ in range(4)] for _ in range(2)]
+        for i in range(2):
+            layer.step_host(xh, dh, oh, dxh, *bufs[i % 2])
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True); b = torch.cuda.Event(enable_timing=True)
         _barrier(world)
         a.record(stream)
-        for _ in range(args.steps):
-            layer.step_host(xh, dh, oh, dxh, *bufs)
+        for i in range(args.steps):
+            layer.step_host(xh, dh, oh, dxh, *bufs[i % 2])
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = _maxreduce(a.elapsed_time(b), world)

@@ -512,13 +512,20 @@ MOE_API moe_status_t moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_w
 /* One training step of the layer from HOST buffers: copies x and dout
  * (pinned host memory recommended) to the device buffers x_dev / dout_dev,
  * runs moe_layer_fwd and moe_layer_bwd, and copies out and dx back to
- * out_host / dx_host.  x and dx move on `stream`; dout and out move on a
- * copy stream the library creates once per device (non-blocking, kept until
- * exit) and orders with events, so that the dout upload overlaps the forward
- * and the out download overlaps the backward.  The call returns once the
- * work is enqueued and leaves `stream` ordered after every copy: synchronise
- * `stream` before reading the host outputs.  The call creates and releases
- * four CUDA events per call; it allocates no device memory.
+ * out_host / dx_host.  The copies run on two streams the library creates
+ * once per device (non-blocking, kept until exit), one for uploads and one
+ * for downloads, ordered with events: out moves to the host under the
+ * backward, and dx under the backward's weight gradients (the backward
+ * forms dx before them).  An upload into a device input buffer waits only
+ * until the earlier host-buffer step that used that buffer has finished
+ * its backward (the library keeps one event per buffer for the last 32
+ * buffers), or, for a buffer it has not seen, until the work already on
+ * `stream` is done: a caller that alternates two sets of device buffers
+ * gets the next step's uploads under the current step's backward.  Write
+ * x_dev / dout_dev only through this call.  The call returns once the work
+ * is enqueued and leaves `stream` ordered after every copy of the step:
+ * synchronise `stream` before reading the host outputs.  It creates six
+ * CUDA events per call and keeps two; it allocates no device memory.
  * ([OC3-th] scaling/optimisation section: the host queues the work without
  * waiting for copies.)
  */

@@ -270,10 +270,15 @@ extern "C" moe_status_t moe_layer_fwd(const moe_layer_desc* L, const moe_layer_w
   return MOE_OK;
 }
 
-extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w,
-                                      const void* x, void* ctx, size_t ctx_bytes,
-                                      const void* dout, void* dx, moe_layer_grads* G,
-                                      int32_t* dev_status, moe_stream_t stream) {
+namespace {
+
+// moe_layer_bwd; dx_ready (nullable) is recorded on the stream once dx is
+// complete, which is before the GEMM1 weight gradient and the router's
+// weight gradient (a host-buffer step downloads dx under them)
+moe_status_t layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w, const void* x,
+                       void* ctx, size_t ctx_bytes, const void* dout, void* dx,
+                       moe_layer_grads* G, int32_t* dev_status, moe_stream_t stream,
+                       cudaEvent_t dx_ready) {
   MOE_TRY(check_common(L, w, ctx, ctx_bytes));
   MOE_CHECK_ARG(x && dout && dx && G && G->dW1 && G->dW3 && G->dW2, "moe_layer_bwd: null pointer");
   const bool router = L->route_mode == MOE_ROUTE_ROUTER;
@@ -283,6 +288,21 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   const bool mx = L->dtype == MOE_MXFP8;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // dx = the plain sum of each token's k rows of dXp: the router's share,
+  // sum_j dl[t, j] W_r[:, e_j], was added to the rows of dXp by the GEMM1
+  // dgrad epilogue.  Taken right after that dgrad, before the weight
+  // gradients, which do not need it.
+  auto dx_sum = [&]() -> moe_status_t {
+    mark(S_UNPERMUTE, false, s);
+    MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, nullptr, nullptr, nullptr, T, k, d, E, dx, nullptr,
+                              0, stream));
+    mark(S_UNPERMUTE, true, s);
+    if (dx_ready && cudaEventRecord(dx_ready, s) != cudaSuccess) {
+      set_error("moe_layer_bwd: recording dx failed");
+      return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  };
   // W_r^T [E, d] (fp32) in the workspace: the GEMM1 dgrad epilogue adds
   // dl_rows[r] * W_r[:, e] to each row r of expert e
   float* wrT = router ? static_cast<float*>(c.ws) : nullptr;
@@ -314,6 +334,7 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                       router ? c.dl_rows : nullptr, router ? wrT : nullptr,
                                       dev_status, s));
     mark(S_DGRAD1, true, s);
+    MOE_TRY(dx_sum());
     mark(S_WGRAD1, false, s);
     if (gathers(L))
       MOE_TRY(moe_grouped_gemm_wgrad_gather(x, T, c.src, c.dA13, c.poff, c.offsets, E, A, d, F,
@@ -349,17 +370,12 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
                                c.dXp, router ? c.dl_rows : nullptr, router ? wrT : nullptr,
                                dev_status, s));
     mark(S_DGRAD1, true, s);
+    MOE_TRY(dx_sum());
     mark(S_WGRAD1, false, s);
     MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff,
                                     c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));
     mark(S_WGRAD1, true, s);
   }
-  mark(S_UNPERMUTE, false, s);
-  // the router's share of dx, sum_j dl[t, j] W_r[:, e_j], was added to the
-  // rows of dXp by the GEMM1 dgrad epilogue: dx is the plain sum of k rows
-  MOE_TRY(moe_unpermute_sum(c.dXp, c.dst, nullptr, nullptr, nullptr, T, k, d, E, dx, nullptr, 0,
-                            stream));
-  mark(S_UNPERMUTE, true, s);
   if (router && G->dWr) {
     mark(S_ROUTER_WGRAD, false, s);
     MOE_TRY(moe_router_wgrad(x, c.src, c.dl_rows, c.offsets, c.poff, T, d, E, A, G->dWr, c.ws,
@@ -369,33 +385,94 @@ extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_w
   return MOE_OK;
 }
 
+}  // namespace
+
+extern "C" moe_status_t moe_layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w,
+                                      const void* x, void* ctx, size_t ctx_bytes,
+                                      const void* dout, void* dx, moe_layer_grads* G,
+                                      int32_t* dev_status, moe_stream_t stream) {
+  return layer_bwd(L, w, x, ctx, ctx_bytes, dout, dx, G, dev_status, stream, nullptr);
+}
+
 namespace {
 
 constexpr int kMaxCopyDevices = 64;
 std::mutex g_copy_mu;
-cudaStream_t g_copy_stream[kMaxCopyDevices] = {};
+cudaStream_t g_copy_stream[2][kMaxCopyDevices] = {};   // [0]: uploads, [1]: downloads
 
-// The library's copy stream on the current device (non-blocking, created on
-// first use and kept until the process exits).
-moe_status_t copy_stream(cudaStream_t* out) {
+// The library's copy streams on the current device (non-blocking, created
+// on first use and kept until the process exits): uploads and downloads on
+// separate streams, so that one call's uploads never queue behind the
+// previous call's downloads.
+moe_status_t copy_streams(cudaStream_t* up, cudaStream_t* down, int* dev_out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxCopyDevices) {
     set_error("moe_layer_step_host: no usable current device");
     return MOE_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lock(g_copy_mu);
-  if (!g_copy_stream[dev] &&
-      cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking) != cudaSuccess) {
-    g_copy_stream[dev] = nullptr;
-    set_error("moe_layer_step_host: copy stream creation failed");
-    return MOE_ERR_CUDA;
-  }
-  *out = g_copy_stream[dev];
+  for (int i = 0; i < 2; ++i)
+    if (!g_copy_stream[i][dev] &&
+        cudaStreamCreateWithFlags(&g_copy_stream[i][dev], cudaStreamNonBlocking) != cudaSuccess) {
+      g_copy_stream[i][dev] = nullptr;
+      set_error("moe_layer_step_host: copy stream creation failed");
+      return MOE_ERR_CUDA;
+    }
+  *up = g_copy_stream[0][dev];
+  *down = g_copy_stream[1][dev];
+  *dev_out = dev;
   return MOE_OK;
 }
 
+// Device input buffers of earlier host-buffer steps, each with the event
+// after which that step was done reading it.  An upload into a known buffer
+// waits only for that event, so a call given the other of two alternating
+// buffer sets uploads its inputs under the previous call's backward; an
+// unknown buffer waits for all work already on the caller's stream.
+struct BufDone {
+  int dev = -1;
+  const void* ptr = nullptr;
+  cudaEvent_t ev = nullptr;
+};
+constexpr int kBufSlots = 32;
+std::mutex g_buf_mu;
+BufDone g_buf[kBufSlots];
+int g_buf_next = 0;
+
+// q waits until buffer p of device dev is free; false if p is unknown
+bool wait_buf(cudaStream_t q, int dev, const void* p, bool* ok) {
+  std::lock_guard<std::mutex> lock(g_buf_mu);
+  for (BufDone& b : g_buf)
+    if (b.ev && b.dev == dev && b.ptr == p) {
+      *ok = cudaStreamWaitEvent(q, b.ev, 0) == cudaSuccess;
+      return true;
+    }
+  return false;
+}
+
+// records on q the point after which buffer p is free (the slot owns the event)
+bool mark_buf(cudaStream_t q, int dev, const void* p) {
+  cudaEvent_t ev = nullptr;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return false;
+  if (cudaEventRecord(ev, q) != cudaSuccess) {
+    cudaEventDestroy(ev);
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(g_buf_mu);
+  BufDone* slot = nullptr;
+  for (BufDone& b : g_buf)
+    if (b.ev && b.dev == dev && b.ptr == p) slot = &b;
+  if (!slot) {
+    slot = &g_buf[g_buf_next];
+    g_buf_next = (g_buf_next + 1) % kBufSlots;
+  }
+  if (slot->ev) cudaEventDestroy(slot->ev);   // every wait on it is already enqueued
+  *slot = BufDone{dev, p, ev};
+  return true;
+}
+
 struct Events {
-  cudaEvent_t ev[4] = {};
+  cudaEvent_t ev[6] = {};
   ~Events() {
     for (cudaEvent_t e : ev)
       if (e) cudaEventDestroy(e);   // released by the driver once the event has completed
@@ -420,8 +497,9 @@ extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_l
   MOE_CHECK_ARG(x_host && dout_host && out_host && dx_host && x_dev && dout_dev && out_dev && dx_dev,
                 "moe_layer_step_host: null pointer");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaStream_t c = nullptr;
-  MOE_TRY(copy_stream(&c));
+  cudaStream_t up = nullptr, down = nullptr;
+  int dev = -1;
+  MOE_TRY(copy_streams(&up, &down, &dev));
   Events E;
   for (cudaEvent_t& e : E.ev)
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
@@ -429,36 +507,49 @@ extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_l
       set_error("moe_layer_step_host: event creation failed");
       return MOE_ERR_CUDA;
     }
-  cudaEvent_t start = E.ev[0], dout_in = E.ev[1], fwd_done = E.ev[2], out_out = E.ev[3];
+  cudaEvent_t start = E.ev[0], in = E.ev[1], fwd_done = E.ev[2], out_out = E.ev[3],
+              dx_ready = E.ev[4], dx_out = E.ev[5];
   const size_t bytes = (size_t)L->T * L->d * 2;
   auto fail = [](const char* what) {
     set_error("moe_layer_step_host: %s failed", what);
     return MOE_ERR_CUDA;
   };
-  if (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(c, start, 0) != cudaSuccess)
-    return fail("ordering the copy stream");
-  if (cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, c) != cudaSuccess ||
-      cudaEventRecord(dout_in, c) != cudaSuccess)
-    return fail("host-to-device copy of dout");
-  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-    return fail("host-to-device copy of x");
-  // from here on every error path still joins the copy stream into s
+  // uploads: each input buffer once the step that last read it is done
+  // with it (or, for a buffer not seen before, after the caller's stream)
+  bool ok = cudaEventRecord(start, s) == cudaSuccess;
+  for (const void* p : {static_cast<const void*>(x_dev), static_cast<const void*>(dout_dev)}) {
+    bool waited = true;
+    if (ok && !wait_buf(up, dev, p, &waited)) waited = cudaStreamWaitEvent(up, start, 0) == cudaSuccess;
+    ok = ok && waited;
+  }
+  if (!ok) return fail("ordering the uploads");
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, up) != cudaSuccess ||
+      cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, up) != cudaSuccess ||
+      cudaEventRecord(in, up) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess)
+    return fail("host-to-device copy of x and dout");
+  // from here on every error path still joins the download stream into s
   moe_status_t st = moe_layer_fwd(L, w, x_dev, out_dev, ctx, ctx_bytes, dev_status, stream);
   const bool rec = cudaEventRecord(fwd_done, s) == cudaSuccess;
-  const bool waited = rec && cudaStreamWaitEvent(c, fwd_done, 0) == cudaSuccess;
+  const bool waited = rec && cudaStreamWaitEvent(down, fwd_done, 0) == cudaSuccess;
   bool copied_out = false;
   if (st == MOE_OK && waited)
-    copied_out = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, c) == cudaSuccess;
-  const bool rec_out = cudaEventRecord(out_out, c) == cudaSuccess;
-  if (st == MOE_OK) {
-    if (cudaStreamWaitEvent(s, dout_in, 0) != cudaSuccess) st = fail("ordering the backward");
-    else st = moe_layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream);
-  }
-  if (st == MOE_OK &&
-      cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    st = fail("device-to-host copy of dx");
-  if ((!rec_out || cudaStreamWaitEvent(s, out_out, 0) != cudaSuccess) && st == MOE_OK)
-    st = fail("joining the copy stream");
+    copied_out = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess;
+  const bool rec_out = cudaEventRecord(out_out, down) == cudaSuccess;
+  // the backward records dx_ready before its weight gradients: dx moves to
+  // the host under them
+  if (st == MOE_OK)
+    st = layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream, dx_ready);
+  bool copied_dx = false;
+  if (st == MOE_OK && cudaStreamWaitEvent(down, dx_ready, 0) == cudaSuccess)
+    copied_dx = cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess;
+  const bool rec_dx = cudaEventRecord(dx_out, down) == cudaSuccess;
+  // x and dout are read until the end of the backward
+  if (st == MOE_OK && !(mark_buf(s, dev, x_dev) && mark_buf(s, dev, dout_dev)))
+    st = fail("recording the input buffers' release");
+  if ((!rec_out || !rec_dx || cudaStreamWaitEvent(s, out_out, 0) != cudaSuccess ||
+       cudaStreamWaitEvent(s, dx_out, 0) != cudaSuccess) && st == MOE_OK)
+    st = fail("joining the download stream");
   if (st == MOE_OK && !(waited && copied_out)) st = fail("device-to-host copy of out");
+  if (st == MOE_OK && !copied_dx) st = fail("device-to-host copy of dx");
   return st;
 }

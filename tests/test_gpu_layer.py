@@ -178,3 +178,36 @@ def test_host_buffer_step_matches_device_step():
     L.step_host(xh, dh, oh, dxh, *bufs)
     torch.cuda.synchronize()
     assert torch.equal(oh, out.cpu()) and torch.equal(dxh, dx.cpu())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mx", [False, True])
+def test_host_buffer_steps_back_to_back(mx):
+    """Four host-buffer steps queued without a host sync, on three different
+    inputs and two alternating sets of device buffers (each step's uploads
+    may run under the previous step's backward): every step's out and dx,
+    and the last step's weight gradients, equal the device-resident step on
+    the same input."""
+    cfg = moe_inputs.CONFIGS["olmo128"].with_(T=4096, mx=mx)
+    inp = moe_inputs.make_layer_inputs(cfg, "cuda")
+    xs = [torch.roll(inp["x"], 37 * i, 0).contiguous() for i in range(3)]
+    ds = [torch.roll(inp["dout"], 101 * i, 0).contiguous() for i in range(3)]
+    order = [0, 1, 2, 1]
+    ref = {}
+    for i in sorted(set(order)):
+        Li, oi, di = _run(cfg, dict(inp, x=xs[i], dout=ds[i]))
+        ref[i] = (oi.cpu(), di.cpu(), Li.dW1.cpu(), Li.dW2.cpu())
+        del Li
+    L = _layer(cfg, inp)
+    host = [(xs[i].cpu().pin_memory(), ds[i].cpu().pin_memory()) for i in range(3)]
+    outs = [(torch.empty_like(host[0][0]).pin_memory(), torch.empty_like(host[0][0]).pin_memory())
+            for _ in order]
+    bufs = [[torch.empty_like(inp["x"]) for _ in range(4)] for _ in range(2)]
+    for n, i in enumerate(order):
+        L.step_host(host[i][0], host[i][1], outs[n][0], outs[n][1], *bufs[n % 2])
+    torch.cuda.synchronize()
+    assert L.status.item() == 0
+    for n, i in enumerate(order):
+        assert torch.equal(outs[n][0], ref[i][0]), ("out", n)
+        assert torch.equal(outs[n][1], ref[i][1]), ("dx", n)
+    assert torch.equal(L.dW1.cpu(), ref[order[-1]][2]) and torch.equal(L.dW2.cpu(), ref[order[-1]][3])
