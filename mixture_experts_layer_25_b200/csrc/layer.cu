@@ -6,11 +6,10 @@
 //           gate-weighted combine.  (MXFP8 and the tokens-N GEMMs take a
 //           separate permute pass that writes Xp.)
 // Backward: combine bwd (dY = g dout, dg, dl) -> GEMM2 dgrad fused with the
-//           SwiGLU backward -> GEMM1 dgrad (+ the router's share of dx as a
-//           rank-1 epilogue term) -> unpermute-sum (dx) -> GEMM2 wgrad ->
-//           GEMM1 wgrad -> router weight grad (dx is complete before the
-//           three weight gradients, which a host-buffer step downloads it
-//           under).
+//           SwiGLU backward -> GEMM2 wgrad -> GEMM1 dgrad (+ the router's
+//           share of dx as a rank-1 epilogue term) -> unpermute-sum (dx) ->
+//           GEMM1 wgrad -> router weight grad (a host-buffer step downloads
+//           dx under the last two).
 // In MXFP8 mode every GEMM operand is quantised along that GEMM's K first
 // (weights included, inside the step); operands used by two GEMMs with
 // different K axes are quantised along both in one pass.  BF16 layers whose
@@ -320,6 +319,10 @@ moe_status_t layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w, cons
                                    c.poff, E, A, d, F, MOE_EPI_SWIGLU_BWD, c.H13, c.dA13,
                                    dev_status, stream));
     mark(S_DGRAD2, true, s);
+    mark(S_WGRAD2, false, s);
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, c.offsets, E,
+                                    A, F, d, G->dW2, nullptr, dev_status, s));
+    mark(S_WGRAD2, true, s);
     mark(S_DGRAD1, false, s);
     if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
     if (tokens_n(L))
@@ -333,10 +336,6 @@ moe_status_t layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w, cons
                                       dev_status, s));
     mark(S_DGRAD1, true, s);
     MOE_TRY(dx_sum());
-    mark(S_WGRAD2, false, s);
-    MOE_TRY(moe::grouped_gemm_wgrad(MOE_BF16, c.h, nullptr, c.dY, nullptr, c.poff, c.offsets, E,
-                                    A, F, d, G->dW2, nullptr, dev_status, s));
-    mark(S_WGRAD2, true, s);
     mark(S_WGRAD1, false, s);
     if (gathers(L))
       MOE_TRY(moe_grouped_gemm_wgrad_gather(x, T, c.src, c.dA13, c.poff, c.offsets, E, A, d, F,
@@ -361,6 +360,10 @@ moe_status_t layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w, cons
                                               c.H13, c.dA_q, c.dA_s, c.dAT_q, c.dAT_s, dev_status,
                                               stream));
     mark(S_DGRAD2, true, s);
+    mark(S_WGRAD2, false, s);
+    MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff,
+                                    c.offsets, E, A, F, d, G->dW2, nullptr, dev_status, s));
+    mark(S_WGRAD2, true, s);
     mark(S_DGRAD1, false, s);
     if (router) MOE_TRY(moe::transpose_f32(w->Wr, d, E, wrT, s));
     MOE_TRY(moe::grouped_gemm_dgrad(MOE_MXFP8, c.dA_q, c.dA_s, c.W13t_q, c.W13t_s, c.W13t_q + wq,
@@ -369,10 +372,6 @@ moe_status_t layer_bwd(const moe_layer_desc* L, const moe_layer_weights* w, cons
                                dev_status, s));
     mark(S_DGRAD1, true, s);
     MOE_TRY(dx_sum());
-    mark(S_WGRAD2, false, s);
-    MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.hT_q, c.hT_s, c.dYT_q, c.dYT_s, c.poff,
-                                    c.offsets, E, A, F, d, G->dW2, nullptr, dev_status, s));
-    mark(S_WGRAD2, true, s);
     mark(S_WGRAD1, false, s);
     MOE_TRY(moe::grouped_gemm_wgrad(MOE_MXFP8, c.XpT_q, c.XpT_s, c.dAT_q, c.dAT_s, c.poff,
                                     c.offsets, E, A, d, F, G->dW1, G->dW3, dev_status, s));
