@@ -103,15 +103,6 @@ __global__ void mx_quant_cols_kernel(const __nv_bfloat16* __restrict__ in, int r
 // (one word = 4 consecutive K blocks of one MN index): a column's word holds
 // the four 32-row sub-blocks of a 128-row block, a row's word four
 // consecutive 32-column blocks.
-__device__ __forceinline__ void unpack4(const uint2& v, float* f) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-  const float2 a = __bfloat1622float2(h[0]), b = __bfloat1622float2(h[1]);
-  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
-}
-
-__device__ __forceinline__ uint32_t encode4(const float* f, const float* inv) {
-  return mx_encode2s(f[0], f[1], inv[0], inv[1]) | (mx_encode2s(f[2], f[3], inv[2], inv[3]) << 16);
-}
 
 // One 128 x 128 bf16 tile in shared memory quantised along both axes by 8
 // warps: warp w takes rows 16w..16w+15 (half of one 32-row MX column block;
