@@ -236,6 +236,32 @@ def test_mx_quantize_dual_equals_both_axes(R, C):
     np.testing.assert_array_equal(scales_to_plain(sc, R, C, 1), s1)
 
 
+@pytest.mark.parametrize("R,C,n", [(384, 256, 200), (256, 512, 129), (512, 128, 64)])
+def test_mx_quantize_dual_partial_rows(R, C, n):
+    """mx_quantize_dual with a device row count n < R: rows below n get the
+    codes and row scales of the full quantisation; a 32-row column block
+    that starts below n gets the full block's column scale (rows at and
+    beyond n are still part of its maximum); a block of a processed 128-row
+    tile that starts at or beyond n gets scale byte 0."""
+    g = torch.Generator(device="cuda"); g.manual_seed(R + C + n)
+    v = (torch.randn((R, C), generator=g, device="cuda") *
+         torch.exp(torch.randn((R, 1), generator=g, device="cuda") * 2)).to(torch.bfloat16)
+    nrows = torch.tensor([n], dtype=torch.int32, device="cuda")
+    (cr, sr), (cc, sc) = moe.mx_quantize_dual(v, nrows=nrows)
+    torch.cuda.synchronize()
+    v64 = f64(v)
+    c0, s0 = oracle.mx_quantize_rows(v64)
+    c1, s1 = oracle.mx_quantize_cols_grouped(v64, np.array([0, R]))
+    np.testing.assert_array_equal(cr.cpu().numpy()[:n], c0[:n])
+    np.testing.assert_array_equal(scales_to_plain(sr, R, C, 0)[:n], s0[:n])
+    np.testing.assert_array_equal(cc.cpu().numpy()[:n], c1[:n])
+    col = scales_to_plain(sc, R, C, 1)          # [R / 32, C]
+    live = -(-n // 32)                          # blocks starting below n
+    np.testing.assert_array_equal(col[:live], s1[:live])
+    tiles_end = -(-n // 128) * 4                # blocks of the processed tiles
+    assert np.all(col[live:tiles_end] == 0)
+
+
 def _every_finite_bf16_in_blocks():
     """Blocks of 32 that hold every finite bf16 value (both zeros and the
     subnormals included) in several roles, as float64 [n_blocks, 32]:
