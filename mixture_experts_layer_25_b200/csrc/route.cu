@@ -283,8 +283,11 @@ route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
       }
     }
   }
-  // exclusive scans over experts (serial per thread-chunk, then across chunks)
-  __shared__ int csum[kScanThreads], psum[kScanThreads];
+  // exclusive scans over experts: serial within each thread's chunk, then
+  // across the threads by shuffles within each warp and over the 32 warp
+  // totals
+  static_assert(kScanThreads == 32 * 32, "two-level shuffle scan");
+  __shared__ int wc[32], wp[32];
   const int per = (E + kScanThreads - 1) / kScanThreads;
   const int e0 = tid * per, e1 = min(E, e0 + per);
   int c = 0, p = 0;
@@ -292,28 +295,38 @@ route_scan_kernel(int32_t* __restrict__ hist, int nblk, int E, int align,
     c += tot[e];
     p += (tot[e] + align - 1) / align * align;
   }
-  csum[tid] = c;
-  psum[tid] = p;
-  __syncthreads();
-  for (int o = 1; o < kScanThreads; o <<= 1) {   // Hillis-Steele inclusive scan
-    int a = 0, b = 0;
-    if (tid >= o) { a = csum[tid - o]; b = psum[tid - o]; }
-    __syncthreads();
-    csum[tid] += a;
-    psum[tid] += b;
-    __syncthreads();
+  const int lane = tid & 31, wid = tid >> 5;
+  int ci = c, pi = p;   // inclusive over the warp's threads
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, ci, o), b = __shfl_up_sync(0xffffffffu, pi, o);
+    if (lane >= o) { ci += a; pi += b; }
   }
-  c = tid ? csum[tid - 1] : 0;
-  p = tid ? psum[tid - 1] : 0;
+  if (lane == 31) { wc[wid] = ci; wp[wid] = pi; }
+  __syncthreads();
+  if (wid == 0) {
+    int x = wc[lane], y = wp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, x, o), b = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) { x += a; y += b; }
+    }
+    wc[lane] = x;   // inclusive over the warps
+    wp[lane] = y;
+  }
+  __syncthreads();
+  ci += wid ? wc[wid - 1] : 0;
+  pi += wid ? wp[wid - 1] : 0;
+  int oc = ci - c, op = pi - p;   // exclusive: the sums of all earlier chunks
   for (int e = e0; e < e1; ++e) {
-    offsets[e] = c;
-    poff[e] = p;
-    c += tot[e];
-    p += (tot[e] + align - 1) / align * align;
+    offsets[e] = oc;
+    poff[e] = op;
+    oc += tot[e];
+    op += (tot[e] + align - 1) / align * align;
   }
   if (tid == kScanThreads - 1) {
-    offsets[E] = csum[tid];
-    poff[E] = psum[tid];
+    offsets[E] = ci;
+    poff[E] = pi;
   }
 }
 
