@@ -99,20 +99,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
-// Row gather (tile::gather4): four rows y0..y3 of a 2-D map whose box is
-// one row high, columns [x, x + box width), land as four consecutive box
-// rows at dst (with the map's swizzle); rows outside the tensor read as
-// zero.  Completion on `bar` as transaction bytes.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
-                                            int y0, int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
-      "r"(y3)
-      : "memory");
-}
-
 // 16-byte global -> shared copy (cp.async, L2 only); valid = false fills
 // the 16 bytes with zeros and reads nothing
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
