@@ -32,10 +32,6 @@ __device__ __forceinline__ float mx_inv_scale(uint32_t byte) {
   return __uint_as_float((254u - byte) << 23);
 }
 
-// two values -> two E4M3 codes (low byte first)
-__device__ __forceinline__ uint32_t mx_encode2(float a, float b) {
-  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
-}
 
 // two values scaled by (power-of-two, so exact) factors -> two E4M3 codes;
 // one packed fp32 multiply for the pair

@@ -297,17 +297,9 @@ __device__ __forceinline__ void cluster_sync_all() {
                ::: "memory");
 }
 
-// 2-D / 3-D tiled loads into this CTA's shared memory whose completion is
+// 3-D tiled load into this CTA's shared memory whose completion is
 // signalled on an mbarrier of either CTA of the pair (shared::cluster
 // address `bar_cluster`, here the leader's)
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m,
-                                                 uint32_t bar_cluster, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m,
                                                  uint32_t bar_cluster, int x, int y, int z) {
   asm volatile(
