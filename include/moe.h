@@ -515,17 +515,21 @@ MOE_API moe_status_t moe_layer_bwd(const moe_layer_desc* desc, const moe_layer_w
  * out_host / dx_host.  The copies run on two streams the library creates
  * once per device (non-blocking, kept until exit), one for uploads and one
  * for downloads, ordered with events: out moves to the host under the
- * backward, and dx under the backward's weight gradients (the backward
- * forms dx before them).  An upload into a device input buffer waits only
- * until the earlier host-buffer step that used that buffer has finished
- * its backward (the library keeps one event per buffer for the last 32
- * buffers), or, for a buffer it has not seen, until the work already on
- * `stream` is done: a caller that alternates two sets of device buffers
- * gets the next step's uploads under the current step's backward.  Write
- * x_dev / dout_dev only through this call.  The call returns once the work
- * is enqueued and leaves `stream` ordered after every copy of the step:
- * synchronise `stream` before reading the host outputs.  It creates six
- * CUDA events per call and keeps two; it allocates no device memory.
+ * backward, and dx under the backward's last weight gradients (the backward
+ * forms dx before them).  Each device buffer is ordered only against the
+ * earlier host-buffer step that used it (the library keeps one event per
+ * buffer for the last 32 buffers): an upload into x_dev / dout_dev waits
+ * for that step's backward, and the forward / backward rewrite out_dev /
+ * dx_dev only after that step's downloads; a buffer the library has not
+ * seen waits for the work already on `stream`.  `stream` itself never waits
+ * for the downloads, so a caller that alternates two sets of device buffers
+ * gets each step's uploads under the previous step's backward and its
+ * forward under the previous step's downloads.  Write the device buffers
+ * only through this call.  The call returns once the work is enqueued; the
+ * host outputs (and the reads of the host inputs) are complete after
+ * moe_layer_step_host_sync(stream) and a synchronisation of `stream` (or of
+ * the device).  It creates four CUDA events per call and keeps four; it
+ * allocates no device memory.
  * ([OC3-th] scaling/optimisation section: the host queues the work without
  * waiting for copies.)
  */
@@ -535,6 +539,14 @@ MOE_API moe_status_t moe_layer_step_host(const moe_layer_desc* desc, const moe_l
                                  void* dx_dev, void* ctx, size_t ctx_bytes,
                                  moe_layer_grads* grads, int32_t* dev_status,
                                  moe_stream_t stream);
+
+/* Makes `stream` wait for every download moe_layer_step_host has queued on
+ * the current device so far: after it, synchronising `stream` leaves every
+ * earlier step's host outputs complete.  Enqueues only; returns
+ * MOE_ERR_CUDA if the library's copy streams cannot be made or ordered.
+ * (No counterpart in the pages: the host-side half of the asynchronous
+ * step above.) */
+MOE_API moe_status_t moe_layer_step_host_sync(moe_stream_t stream);
 
 #ifdef __cplusplus
 }

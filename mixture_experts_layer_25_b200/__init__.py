@@ -360,12 +360,20 @@ class MoELayer:
 
     def step_host(self, x_host, dout_host, out_host, dx_host, x_dev, dout_dev, out_dev, dx_dev,
                   stream=None):
-        """fwd + bwd from host buffers (copies inside the call, on `stream`)."""
+        """fwd + bwd from host buffers (copies inside the call; the host
+        outputs are complete after step_host_sync and a stream sync)."""
         hp = lambda t: ctypes.c_void_p(t.data_ptr())
         _lib.call("moe_layer_step_host", ctypes.byref(self.desc), ctypes.byref(self.weights),
                   hp(x_host), hp(dout_host), hp(out_host), hp(dx_host), _p(x_dev), _p(dout_dev),
                   _p(out_dev), _p(dx_dev), ctypes.c_void_p(self._ctx_ptr), self.ctx_bytes,
                   ctypes.byref(self.grads), _p(self.status), _s(stream))
+
+    @staticmethod
+    def step_host_sync(stream=None):
+        """Orders `stream` after every download step_host has queued on the
+        current device; synchronise the stream afterwards to read the host
+        outputs."""
+        _lib.call("moe_layer_step_host_sync", _s(stream))
 
     def ctx_tensor(self, name: str, shape, dtype) -> torch.Tensor:
         """A view of one saved buffer of the context (for inspection)."""

@@ -89,6 +89,7 @@ _SIGS = {
                           ctypes.POINTER(LayerGrads), P, P]),
     "moe_layer_step_host": (I, [ctypes.POINTER(LayerDesc), ctypes.POINTER(LayerWeights), P, P, P, P,
                                 P, P, P, P, P, Z, ctypes.POINTER(LayerGrads), P, P]),
+    "moe_layer_step_host_sync": (I, [P]),
 }
 
 _lib = None

@@ -473,7 +473,7 @@ bool mark_buf(cudaStream_t q, int dev, const void* p) {
 }
 
 struct Events {
-  cudaEvent_t ev[6] = {};
+  cudaEvent_t ev[4] = {};
   ~Events() {
     for (cudaEvent_t e : ev)
       if (e) cudaEventDestroy(e);   // released by the driver once the event has completed
@@ -482,12 +482,17 @@ struct Events {
 
 }  // namespace
 
-// Schedule (s = the caller's stream, c = the library's copy stream):
-//   s: record start | H2D x | fwd | record fwd_done | wait dout_in | bwd | D2H dx | wait out_out
-//   c: wait start   | H2D dout | record dout_in | wait fwd_done | D2H out | record out_out
-// so the dout upload runs under the forward and the out download under the
-// backward; the call leaves s ordered after every copy, as if all of them
-// had been issued on s.
+// Schedule (s = the caller's stream; up / down = the library's upload and
+// download streams; buffer events from the registry above):
+//   up:   wait x_dev, dout_dev free | H2D x, dout | record in
+//   s:    wait out_dev, dx_dev free | wait in | fwd | record fwd_done | bwd
+//         (records dx_ready after the dx sum) | x_dev, dout_dev free
+//   down: wait fwd_done | D2H out | out_dev free | wait dx_ready | D2H dx |
+//         dx_dev free
+// s never waits for the downloads: the next step's forward runs under this
+// step's downloads when it has the other set of device buffers.  The host
+// outputs are complete once s has been made to wait for the downloads
+// (moe_layer_step_host_sync) and then synchronised.
 extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_layer_weights* w,
                                             const void* x_host, const void* dout_host,
                                             void* out_host, void* dx_host, void* x_dev,
@@ -508,8 +513,7 @@ extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_l
       set_error("moe_layer_step_host: event creation failed");
       return MOE_ERR_CUDA;
     }
-  cudaEvent_t start = E.ev[0], in = E.ev[1], fwd_done = E.ev[2], out_out = E.ev[3],
-              dx_ready = E.ev[4], dx_out = E.ev[5];
+  cudaEvent_t start = E.ev[0], in = E.ev[1], fwd_done = E.ev[2], dx_ready = E.ev[3];
   const size_t bytes = (size_t)L->T * L->d * 2;
   auto fail = [](const char* what) {
     set_error("moe_layer_step_host: %s failed", what);
@@ -528,29 +532,50 @@ extern "C" moe_status_t moe_layer_step_host(const moe_layer_desc* L, const moe_l
       cudaMemcpyAsync(dout_dev, dout_host, bytes, cudaMemcpyHostToDevice, up) != cudaSuccess ||
       cudaEventRecord(in, up) != cudaSuccess || cudaStreamWaitEvent(s, in, 0) != cudaSuccess)
     return fail("host-to-device copy of x and dout");
-  // from here on every error path still joins the download stream into s
+  // outputs: a device output buffer is rewritten only after the download
+  // that last read it
+  for (const void* p : {static_cast<const void*>(out_dev), static_cast<const void*>(dx_dev)}) {
+    bool waited = true;
+    if (wait_buf(s, dev, p, &waited) && !waited) return fail("ordering the output buffers");
+  }
   moe_status_t st = moe_layer_fwd(L, w, x_dev, out_dev, ctx, ctx_bytes, dev_status, stream);
   const bool rec = cudaEventRecord(fwd_done, s) == cudaSuccess;
   const bool waited = rec && cudaStreamWaitEvent(down, fwd_done, 0) == cudaSuccess;
   bool copied_out = false;
   if (st == MOE_OK && waited)
-    copied_out = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess;
-  const bool rec_out = cudaEventRecord(out_out, down) == cudaSuccess;
-  // the backward records dx_ready before its weight gradients: dx moves to
-  // the host under them
+    copied_out = cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess &&
+                 mark_buf(down, dev, out_dev);
+  // the backward records dx_ready before its last weight gradients: dx moves
+  // to the host under them
   if (st == MOE_OK)
     st = layer_bwd(L, w, x_dev, ctx, ctx_bytes, dout_dev, dx_dev, G, dev_status, stream, dx_ready);
   bool copied_dx = false;
   if (st == MOE_OK && cudaStreamWaitEvent(down, dx_ready, 0) == cudaSuccess)
-    copied_dx = cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess;
-  const bool rec_dx = cudaEventRecord(dx_out, down) == cudaSuccess;
+    copied_dx = cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, down) == cudaSuccess &&
+                mark_buf(down, dev, dx_dev);
   // x and dout are read until the end of the backward
   if (st == MOE_OK && !(mark_buf(s, dev, x_dev) && mark_buf(s, dev, dout_dev)))
     st = fail("recording the input buffers' release");
-  if ((!rec_out || !rec_dx || cudaStreamWaitEvent(s, out_out, 0) != cudaSuccess ||
-       cudaStreamWaitEvent(s, dx_out, 0) != cudaSuccess) && st == MOE_OK)
-    st = fail("joining the download stream");
   if (st == MOE_OK && !(waited && copied_out)) st = fail("device-to-host copy of out");
   if (st == MOE_OK && !copied_dx) st = fail("device-to-host copy of dx");
   return st;
+}
+
+extern "C" moe_status_t moe_layer_step_host_sync(moe_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t up = nullptr, down = nullptr;
+  int dev = -1;
+  MOE_TRY(copy_streams(&up, &down, &dev));
+  cudaEvent_t ev = nullptr;
+  if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+    set_error("moe_layer_step_host_sync: event creation failed");
+    return MOE_ERR_CUDA;
+  }
+  const bool ok = cudaEventRecord(ev, down) == cudaSuccess && cudaStreamWaitEvent(s, ev, 0) == cudaSuccess;
+  cudaEventDestroy(ev);   // released by the driver once the event has completed
+  if (!ok) {
+    set_error("moe_layer_step_host_sync: ordering the stream after the downloads failed");
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }

@@ -185,9 +185,10 @@ def test_host_buffer_step_matches_device_step():
 def test_host_buffer_steps_back_to_back(mx):
     """Four host-buffer steps queued without a host sync, on three different
     inputs and two alternating sets of device buffers (each step's uploads
-    may run under the previous step's backward): every step's out and dx,
-    and the last step's weight gradients, equal the device-resident step on
-    the same input."""
+    may run under the previous step's backward, its forward under the
+    previous step's downloads): after step_host_sync and a synchronisation
+    of the stream alone, every step's out and dx, and the last step's
+    weight gradients, equal the device-resident step on the same input."""
     cfg = moe_inputs.CONFIGS["olmo128"].with_(T=4096, mx=mx)
     inp = moe_inputs.make_layer_inputs(cfg, "cuda")
     xs = [torch.roll(inp["x"], 37 * i, 0).contiguous() for i in range(3)]
@@ -203,9 +204,11 @@ def test_host_buffer_steps_back_to_back(mx):
     outs = [(torch.empty_like(host[0][0]).pin_memory(), torch.empty_like(host[0][0]).pin_memory())
             for _ in order]
     bufs = [[torch.empty_like(inp["x"]) for _ in range(4)] for _ in range(2)]
+    stream = torch.cuda.current_stream()
     for n, i in enumerate(order):
         L.step_host(host[i][0], host[i][1], outs[n][0], outs[n][1], *bufs[n % 2])
-    torch.cuda.synchronize()
+    L.step_host_sync()                   # the stream, not the device, is synchronised
+    stream.synchronize()
     assert L.status.item() == 0
     for n, i in enumerate(order):
         assert torch.equal(outs[n][0], ref[i][0]), ("out", n)
